@@ -1,0 +1,169 @@
+/*
+ * sparse_attn.h -- C ABI of libsparse_attn.so: block-sparse and index-sparse softmax
+ * attention on one NVIDIA B200 (sm_100a), forward (O, LSE) and backward (dQ, dK, dV),
+ * and the conversion of token-level top-k indices or block masks into the per-tile
+ * lists the kernels walk.
+ *
+ * Sources of the operation (web pages; no formulas are printed there):
+ *  - MagiAttention PR #334, "[WIP]: feat(cutedsl-sm100): BWD LoopK with
+ *    warp-specialized pipeline + IndexSparse/BlockSparse support": Summary (sparse
+ *    attention forward/backward, dQ accumulation), section 1 (backward pipeline, fp32
+ *    dK/dV accumulation, postprocess with softmax_scale), section 2
+ *    (index_attn_indices_to_block_sparse: indices (total_q, NHK, topk) -> block lists
+ *    via a presence matrix; per-M-block N-block lists).
+ *  - MagiAttention PR #331, "feat: support 192/128 and 256/256 ffa_fa4 in magi":
+ *    Summary (head dims (192,128) and (256,256)), "CSR Tile Mapping" (transposed
+ *    key-to-query block lists for the backward).
+ *  - xtuner PR #2096, "[Feature] Add optional TileLang Top-K selector", Main Changes 1:
+ *    int32 top-k indices with -1 for invalid positions (the input of index mode).
+ *  - nvfp4-megamoe-kernel commit log, multi-row softmax notes: online softmax over
+ *    key tiles with a running max and sum, un-normalised P, final O = acc / sum.
+ *
+ * Definition implemented (textbook attention on an allowed key set A_i):
+ *   s_ij = scale * q_i . k_j ;  LSE_i = ln sum_{j in A_i} exp(s_ij) ;
+ *   O_i = sum_j exp(s_ij - LSE_i) v_j ;  dP_ij = dO_i . v_j ;  Delta_i = dO_i . O_i ;
+ *   dS_ij = P_ij (dP_ij - Delta_i) ; dq_i = scale sum_j dS_ij k_j ;
+ *   dk_j = scale sum_{h in group} sum_i dS_ij q_i ; dv_j = sum_{h in group} sum_i P_ij dO_i.
+ *   Query head h uses KV head h / (HQ / HK).  A row with an empty set gets O = 0,
+ *   LSE = -inf and zero gradients.
+ * A_i: block mode -- mask[b][g][i/bs][j/bs] != 0 (bs = 64 or 128); dense mode -- all
+ * keys; index mode -- the set of row i's indices (duplicates collapse, -1 skipped);
+ * with causal != 0 additionally j <= i.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library never
+ *    allocates or frees device memory.  Host pointers are only the parameter structs.
+ *  - Layouts (row-major, last dimension contiguous, no padding):
+ *      q [B][Sq][HQ][Dqk], k [B][Sk][HK][Dqk], v [B][Sk][HK][Dv],
+ *      o, dO [B][Sq][HQ][Dv], dq [B][Sq][HQ][Dqk], dk [B][Sk][HK][Dqk],
+ *      dv [B][Sk][HK][Dv]: bf16.  lse [B][HQ][Sq]: fp32 (natural log).
+ *    Base pointers must be 16-byte aligned.
+ *  - Supported (Dqk, Dv): (64,64), (128,128), (192,128), (256,256).  HQ % HK == 0.
+ *  - Work is enqueued on `stream` and runs asynchronously; the call returns once it
+ *    is enqueued.  Errors found on the host are returned before anything is enqueued.
+ *  - Return value: SA_OK (0) or a negative SA_ERR_* code.  Errors found on the GPU
+ *    (an index outside [-1, Sk), a pipeline wait that timed out) are OR-ed into the
+ *    optional device int32 `dev_status` (bit 1: index, bit 2: timeout); read it after
+ *    synchronising.  No C++ exception crosses this boundary.
+ */
+#ifndef SPARSE_ATTN_H_
+#define SPARSE_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *sa_stream_t; /* the same handle as cudaStream_t */
+
+#define SA_OK 0
+#define SA_ERR_INVALID (-1)     /* null pointer, bad size or inconsistent shape */
+#define SA_ERR_UNSUPPORTED (-2) /* head dims, block size or mode not supported */
+#define SA_ERR_INDEX (-3)       /* reserved: index errors are reported on the device */
+#define SA_ERR_ALIGN (-4)       /* a base pointer is not 16-byte aligned */
+#define SA_ERR_CUDA (-5)        /* a CUDA call or kernel launch failed */
+#define SA_ERR_WORKSPACE (-7)   /* workspace missing or too small */
+
+#define SA_MODE_DENSE 0
+#define SA_MODE_BLOCK 1
+#define SA_MODE_INDEX 2
+
+#define SA_TILE 128 /* every list entry stands for a 128 x 128 (query x key) tile */
+
+/*
+ * Tile lists and the element data the kernels need inside partial tiles.  Filled by
+ * block_mask_to_block_sparse() or index_to_block_sparse(); read by the attention
+ * calls.  With Tm = ceil(Sq/128), Tn = ceil(Sk/128), W = ceil(Sk/32), the caller
+ * allocates (device memory):
+ *   cnt  int32 [B][HK][Tm][2]   (n_full, n_partial) per query tile
+ *   idx  int32 [B][HK][Tm][Tn]  full key tiles ascending, then partial ascending, -1 fill
+ *   tcnt int32 [B][HK][Tn][2]   the same per key tile over query tiles (backward)
+ *   tidx int32 [B][HK][Tn][Tm]
+ *   bitmap uint32 [B][HK][Sq][W] (index mode only): bit j%32 of word j/32 of row i is
+ *          set iff j is one of row i's indices (the presence matrix).
+ * A tile is FULL when every (i, j) in it with i < Sq, j < Sk is allowed and the tile
+ * lies inside [0, Sk); PARTIAL when some (i, j) is allowed otherwise; absent when none
+ * is.  `mask` (block mode) is the caller's mask, kept for partial tiles of bs = 64.
+ */
+typedef struct sa_block_sparse {
+  int32_t mode;   /* SA_MODE_* */
+  int32_t causal; /* non-zero: j <= i is also required */
+  int32_t B, HK;
+  int64_t Sq, Sk;
+  int32_t bs, Mb, Nb;   /* block mode: granularity and mask extents (Mb*bs >= Sq, Nb*bs >= Sk) */
+  const uint8_t *mask;  /* block mode: [B][HK][Mb][Nb]; NULL in dense mode */
+  uint32_t *bitmap;     /* index mode */
+  int32_t *cnt, *idx, *tcnt, *tidx;
+} sa_block_sparse;
+
+/*
+ * index_to_block_sparse -- MagiAttention PR #334, section 2
+ * (index_attn_indices_to_block_sparse and the per-M-block normalisation) and
+ * MagiAttention PR #331, "CSR Tile Mapping" (the transposed lists).
+ *   idx   device int32 [B][Sq][HK][topk]: key positions in [0, Sk) or -1 (padding).
+ *   out   host struct: B, HK, Sq, Sk, causal and the device buffers bitmap, cnt, idx,
+ *         tcnt, tidx must be set by the caller; mode is set to SA_MODE_INDEX.
+ * Fills the bitmap and all four lists.  Values < -1 or >= Sk are skipped and set bit 1
+ * of *dev_status (when dev_status is not NULL).
+ */
+int index_to_block_sparse(const int32_t *idx, int32_t topk, sa_block_sparse *out,
+                          int32_t *dev_status, sa_stream_t stream);
+
+/*
+ * block_mask_to_block_sparse -- the block-mask counterpart (BlockSparse attention of
+ * MagiAttention PR #334; block-sparsity computation of sgl-flash-attn PR #28).
+ *   out   host struct with mode = SA_MODE_BLOCK (mask = device uint8
+ *         [B][HK][Mb][Nb], bs in {64, 128}) or SA_MODE_DENSE (mask unused), plus B, HK,
+ *         Sq, Sk, causal and the device list buffers.  bitmap is unused.
+ */
+int block_mask_to_block_sparse(sa_block_sparse *out, sa_stream_t stream);
+
+typedef struct sparse_attn_params {
+  const void *q, *k, *v; /* bf16 inputs */
+  void *o;               /* bf16 [B][Sq][HQ][Dv]: forward output, backward input */
+  float *lse;            /* fp32 [B][HQ][Sq]: forward output, backward input */
+  const void *dout;      /* bf16 [B][Sq][HQ][Dv]: backward input */
+  void *dq, *dk, *dv;    /* bf16 backward outputs */
+  int32_t B, HQ, HK, Dqk, Dv;
+  int64_t Sq, Sk;
+  float softmax_scale;
+  const sa_block_sparse *sparse; /* host pointer; lists built for the same B, HK, Sq, Sk */
+  int32_t *dev_status;           /* optional device int32 */
+} sparse_attn_params;
+
+/*
+ * sparse_attn_fwd -- forward: O and LSE.  Streams only the listed key tiles of each
+ * 128-query tile through shared memory, computes S = Q K^T and O += P V on the
+ * tensor cores with fp32 accumulation in tensor memory, and runs the online softmax
+ * (running max and sum, un-normalised P, O / sum at the end; nvfp4-megamoe-kernel
+ * multi-row softmax notes).  Reads q, k, v; writes o, lse.
+ */
+int sparse_attn_fwd(const sparse_attn_params *p, sa_stream_t stream);
+
+/* Bytes of device workspace sparse_attn_bwd needs for these shapes (fp32 Delta and
+ * the fp32 dQ accumulator), rounded up to 256 B. */
+size_t sparse_attn_bwd_workspace_size(const sparse_attn_params *p);
+
+/*
+ * sparse_attn_bwd -- backward: dq, dk, dv from q, k, v, o, lse, dout.
+ * Preprocess Delta = rowsum(dO * O); main kernel over key tiles (walking the
+ * transposed lists) recomputing P = exp(scale S - LSE), accumulating dV += P^T dO and
+ * dK += dS^T Q in tensor memory and adding dQ += dS K into an fp32 accumulator;
+ * postprocess scales dQ (and dK) by softmax_scale and casts to bf16 (MagiAttention
+ * PR #334, section 1 and section 3).  `workspace` is device memory of at least
+ * sparse_attn_bwd_workspace_size() bytes, owned by the caller; its contents need not
+ * be initialised.
+ */
+int sparse_attn_bwd(const sparse_attn_params *p, void *workspace, size_t workspace_bytes,
+                    sa_stream_t stream);
+
+/* Static description of an SA_* code. */
+const char *sparse_attn_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_ATTN_H_ */

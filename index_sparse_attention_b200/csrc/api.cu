@@ -1,0 +1,172 @@
+// api.cu -- the C ABI of libsparse_attn.so: argument checks, TMA tensor maps and the
+// launches of the forward and backward kernels.  No device memory is allocated here.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "sa_device.cuh"
+#include "sa_kernels.h"
+
+using namespace sa;
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 4-D map over a [B][S][H][D] bf16 tensor with 64 x 128 (D x S) boxes, 128-byte swizzle.
+// Out-of-range rows read as zeros.
+bool make_map(CUtensorMap* m, const void* base, int D, int64_t S, int H, int B) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S),
+                        static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(H) * D * 2, static_cast<cuuint64_t>(D) * 2,
+                           static_cast<cuuint64_t>(S) * H * D * 2};
+  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool dims_supported(int dqk, int dv) {
+  return (dqk == 64 && dv == 64) || (dqk == 128 && dv == 128) || (dqk == 192 && dv == 128) ||
+         (dqk == 256 && dv == 256);
+}
+
+int fill_args(const sparse_attn_params* p, AttnArgs* a, bool backward) {
+  if (!p || !p->sparse) return SA_ERR_INVALID;
+  const sa_block_sparse* s = p->sparse;
+  if (!p->q || !p->k || !p->v || !p->o || !p->lse) return SA_ERR_INVALID;
+  if (backward && (!p->dout || !p->dq || !p->dk || !p->dv)) return SA_ERR_INVALID;
+  if (p->B <= 0 || p->HQ <= 0 || p->HK <= 0 || p->Sq <= 0 || p->Sk <= 0) return SA_ERR_INVALID;
+  if (p->HQ % p->HK != 0) return SA_ERR_INVALID;
+  if (!dims_supported(p->Dqk, p->Dv)) return SA_ERR_UNSUPPORTED;
+  if (s->B != p->B || s->HK != p->HK || s->Sq != p->Sq || s->Sk != p->Sk) return SA_ERR_INVALID;
+  if (!s->cnt || !s->idx || !s->tcnt || !s->tidx) return SA_ERR_INVALID;
+  if (s->mode == SA_MODE_INDEX && !s->bitmap) return SA_ERR_INVALID;
+  if (s->mode == SA_MODE_BLOCK && (!s->mask || (s->bs != 64 && s->bs != 128)))
+    return SA_ERR_INVALID;
+  if (s->mode != SA_MODE_DENSE && s->mode != SA_MODE_BLOCK && s->mode != SA_MODE_INDEX)
+    return SA_ERR_INVALID;
+  if (!(p->softmax_scale > 0.f)) return SA_ERR_INVALID;
+  const int64_t Tm = (p->Sq + kTile - 1) / kTile, Tn = (p->Sk + kTile - 1) / kTile;
+  if (Tm > 65535 * 32 || Tn > 8192 || p->HQ > 65535 || p->B > 65535) return SA_ERR_UNSUPPORTED;
+  if (p->Sq > 0x7FFFFFFF || p->Sk > 0x7FFFFFFF) return SA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {p->q, p->k, p->v, p->o};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return SA_ERR_ALIGN;
+  if (backward) {
+    const void* bp[] = {p->dout, p->dq, p->dk, p->dv};
+    for (const void* q : bp)
+      if (!aligned16(q)) return SA_ERR_ALIGN;
+  }
+  *a = AttnArgs{};
+  a->o = p->o;
+  a->lse = p->lse;
+  a->dout = p->dout;
+  a->dq = p->dq;
+  a->dk = p->dk;
+  a->dv = p->dv;
+  a->cnt = s->cnt;
+  a->idx = s->idx;
+  a->tcnt = s->tcnt;
+  a->tidx = s->tidx;
+  a->mask = s->mode == SA_MODE_BLOCK ? s->mask : nullptr;
+  a->bitmap = s->mode == SA_MODE_INDEX ? s->bitmap : nullptr;
+  a->Sq = p->Sq;
+  a->Sk = p->Sk;
+  a->B = p->B;
+  a->HQ = p->HQ;
+  a->HK = p->HK;
+  a->Dqk = p->Dqk;
+  a->Dv = p->Dv;
+  a->Tm = static_cast<int>(Tm);
+  a->Tn = static_cast<int>(Tn);
+  a->W = static_cast<int>((p->Sk + 31) / 32);
+  a->mode = s->mode;
+  a->causal = s->causal ? 1 : 0;
+  a->bs = s->mode == SA_MODE_BLOCK ? s->bs : kTile;
+  a->Mb = s->Mb;
+  a->Nb = s->Nb;
+  a->scale = p->softmax_scale;
+  a->scale_log2 = p->softmax_scale * 1.4426950408889634f;
+  a->status = p->dev_status;
+  return SA_OK;
+}
+
+int fill_maps(const sparse_attn_params* p, TensorMaps* m, bool backward) {
+  if (!make_map(&m->q, p->q, p->Dqk, p->Sq, p->HQ, p->B)) return SA_ERR_CUDA;
+  if (!make_map(&m->k, p->k, p->Dqk, p->Sk, p->HK, p->B)) return SA_ERR_CUDA;
+  if (!make_map(&m->v, p->v, p->Dv, p->Sk, p->HK, p->B)) return SA_ERR_CUDA;
+  if (backward) {
+    if (!make_map(&m->o, p->o, p->Dv, p->Sq, p->HQ, p->B)) return SA_ERR_CUDA;
+    if (!make_map(&m->dout, p->dout, p->Dv, p->Sq, p->HQ, p->B)) return SA_ERR_CUDA;
+  }
+  return SA_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+extern "C" const char* sparse_attn_error_string(int code) {
+  switch (code) {
+    case SA_OK: return "ok";
+    case SA_ERR_INVALID: return "invalid argument (null pointer, bad size or inconsistent shape)";
+    case SA_ERR_UNSUPPORTED: return "unsupported head dims, block size, mode or extent";
+    case SA_ERR_INDEX: return "index outside [-1, Sk)";
+    case SA_ERR_ALIGN: return "a tensor base pointer is not 16-byte aligned";
+    case SA_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case SA_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown error code";
+  }
+}
+
+extern "C" int sparse_attn_fwd(const sparse_attn_params* p, sa_stream_t stream) {
+  AttnArgs a;
+  int rc = fill_args(p, &a, false);
+  if (rc) return rc;
+  TensorMaps m;
+  rc = fill_maps(p, &m, false);
+  if (rc) return rc;
+  return launch_fwd(a, m, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" size_t sparse_attn_bwd_workspace_size(const sparse_attn_params* p) {
+  if (!p || p->B <= 0 || p->HQ <= 0 || p->Sq <= 0 || p->Dqk <= 0) return 0;
+  const size_t delta = sizeof(float) * static_cast<size_t>(p->B) * p->HQ * p->Sq;
+  const size_t dq = sizeof(float) * static_cast<size_t>(p->B) * p->Sq * p->HQ * p->Dqk;
+  return round256(delta) + round256(dq);
+}
+
+extern "C" int sparse_attn_bwd(const sparse_attn_params* p, void* workspace,
+                               size_t workspace_bytes, sa_stream_t stream) {
+  AttnArgs a;
+  int rc = fill_args(p, &a, true);
+  if (rc) return rc;
+  const size_t need = sparse_attn_bwd_workspace_size(p);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SA_ERR_WORKSPACE;
+  a.delta = static_cast<float*>(workspace);
+  a.dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                      round256(sizeof(float) * static_cast<size_t>(p->B) * p->HQ *
+                                               p->Sq));
+  TensorMaps m;
+  rc = fill_maps(p, &m, true);
+  if (rc) return rc;
+  return launch_bwd(a, m, reinterpret_cast<cudaStream_t>(stream));
+}

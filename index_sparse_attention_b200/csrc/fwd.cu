@@ -1,0 +1,362 @@
+// fwd.cu -- sparse attention forward on sm_100a: O and LSE.
+//
+// Operation: softmax attention over the allowed key set of each query (IndexSparse /
+// BlockSparse attention, MagiAttention PR #334, Summary and section 2), computed as
+// the online softmax over key tiles that the nvfp4-megamoe-kernel commit log spells
+// out in its multi-row softmax notes: running max and running sum per row,
+// un-normalised P = exp(s - max), accumulate P V, final O = acc / sum.
+//
+// B200 design (one CTA per 128-query tile of one (batch, query head)):
+//   warp 0     TMA producer: Q once, then the K and V tiles of the ACTIVE key tiles
+//              only (the forward list), 128-byte swizzled, double-buffered when
+//              shared memory allows.
+//   warp 1     allocates 512 TMEM columns and issues the tcgen05 MMAs from one
+//              thread: S = Q K^T into one of two TMEM S buffers (so the next S is
+//              computed while the softmax works on the current one), and
+//              O += P V with P read from TMEM (A operand in tensor memory).
+//   warps 2-5  softmax, one query row per thread (thread = TMEM lane): tcgen05.ld the
+//              S row, apply the element mask on partial tiles (range, causal, 64-block
+//              mask or index bitmap), update the running max lazily (O is rescaled in
+//              TMEM only when the max grows by more than 2^8), exponentiate with
+//              ex2, write bf16 P back over the S buffer, and at the end normalise O
+//              and write O (bf16) and LSE (fp32, natural log).
+// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+Dv).
+// Every mbarrier wait is bounded; a timeout sets SA_ERR_TIMEOUT in the status word and
+// the CTA leaves after releasing its tensor memory.
+#include "sa_device.cuh"
+#include "sa_kernels.h"
+
+namespace sa {
+
+template <int DQK, int DV>
+struct FwdCfg {
+  static constexpr int kPanel = 128 * 128;  // one 64-column x 128-row swizzled panel
+  static constexpr int kQBytes = 128 * DQK * 2;
+  static constexpr int kKBytes = 128 * DQK * 2;
+  static constexpr int kVBytes = 128 * DV * 2;
+  static constexpr int kKStages = (DQK == 256) ? 1 : 2;
+  static constexpr int kVStages = (DV == 256) ? 1 : 2;
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + kQBytes;
+  static constexpr int kVOff = kKOff + kKStages * kKBytes;
+  static constexpr int kBarOff = kVOff + kVStages * kVBytes;
+  static constexpr int kSmem = kBarOff + 256 + 1024;  // barriers + alignment slack
+  static constexpr int kThreads = 192;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kOCol = 256;
+  static_assert(kSmem <= 227 * 1024, "shared memory budget");
+  static_assert(kOCol + DV <= kTmemCols, "tensor memory budget");
+};
+
+// barrier slots
+enum : int { kBQ = 0, kBKF = 1, kBKE = 3, kBVF = 5, kBVE = 7, kBSF = 9, kBPF = 11, kBOD = 13,
+             kBDrain = 14, kBOFin = 15, kNumBars = 16 };
+
+template <int DQK, int DV>
+__global__ void __launch_bounds__(192, 1)
+    sparse_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
+  using C = FwdCfg<DQK, DV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::kBarOff;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 8 * kNumBars + 4);
+  auto BAR = [&](int k) { return bar0 + 8u * static_cast<uint32_t>(k); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt = a.Tm - 1 - static_cast<int>(blockIdx.x);  // longest lists first under causal
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int g = h / (a.HQ / a.HK);
+  const int64_t bg = static_cast<int64_t>(b) * a.HK + g;
+  const int64_t lrow = bg * a.Tm + mt;
+  const int n_full = __ldg(a.cnt + 2 * lrow);
+  const int n_iter = n_full + __ldg(a.cnt + 2 * lrow + 1);
+  const int32_t* list = a.idx + lrow * a.Tn;
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(kBQ), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR(kBKF + s), 1);
+      mbar_init(BAR(kBKE + s), 1);
+      mbar_init(BAR(kBVF + s), 1);
+      mbar_init(BAR(kBVE + s), 1);
+      mbar_init(BAR(kBSF + s), 1);
+      mbar_init(BAR(kBPF + s), 128);
+    }
+    mbar_init(BAR(kBOD), 1);
+    mbar_init(BAR(kBDrain), 1);
+    mbar_init(BAR(kBOFin), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0 && n_iter > 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      prefetch_tensormap(&tm_v);
+      mbar_arrive_expect_tx(BAR(kBQ), C::kQBytes);
+      for (int c = 0; c < DQK / 64; ++c)
+        tma_load_4d(sbase + C::kQOff + c * C::kPanel, &tm_q, BAR(kBQ), c * 64, mt * 128, h, b);
+      for (int it = 0; it < n_iter; ++it) {
+        const int nt = __ldg(list + it);
+        const int ks = it % C::kKStages, ku = it / C::kKStages;
+        if (!mbar_wait(BAR(kBKE + ks), (ku & 1) ^ 1, abort_flag, a.status)) break;
+        mbar_arrive_expect_tx(BAR(kBKF + ks), C::kKBytes);
+        for (int c = 0; c < DQK / 64; ++c)
+          tma_load_4d(sbase + C::kKOff + ks * C::kKBytes + c * C::kPanel, &tm_k, BAR(kBKF + ks),
+                      c * 64, nt * 128, g, b);
+        const int vs = it % C::kVStages, vu = it / C::kVStages;
+        if (!mbar_wait(BAR(kBVE + vs), (vu & 1) ^ 1, abort_flag, a.status)) break;
+        mbar_arrive_expect_tx(BAR(kBVF + vs), C::kVBytes);
+        for (int c = 0; c < DV / 64; ++c)
+          tma_load_4d(sbase + C::kVOff + vs * C::kVBytes + c * C::kPanel, &tm_v, BAR(kBVF + vs),
+                      c * 64, nt * 128, g, b);
+      }
+      if (*abort_flag) {
+        // Let the loads already issued land before the CTA may leave (time-limited).
+        mbar_wait_limited(BAR(kBQ), 0);
+        for (int it = max(0, n_iter - 2); it < n_iter; ++it) {
+          mbar_wait_limited(BAR(kBKF + it % C::kKStages), (it / C::kKStages) & 1);
+          mbar_wait_limited(BAR(kBVF + it % C::kVStages), (it / C::kVStages) & 1);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_iter > 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16(128, DV, 0, 1);
+      bool ok = mbar_wait(BAR(kBQ), 0, abort_flag, a.status);
+      auto issue_s = [&](int it) -> bool {
+        const int ks = it % C::kKStages, ku = it / C::kKStages;
+        if (!mbar_wait(BAR(kBKF + ks), ku & 1, abort_flag, a.status)) return false;
+        tc_fence_after();
+        const uint32_t qa = sbase + C::kQOff;
+        const uint32_t kb = sbase + C::kKOff + ks * C::kKBytes;
+        const uint32_t d = tmem + static_cast<uint32_t>((it & 1) * 128);
+#pragma unroll
+        for (int kk = 0; kk < DQK / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kPanel + (kk & 3) * 32;
+          umma_ss(d, sw128_desc(qa + off, 16, 1024), sw128_desc(kb + off, 16, 1024), idesc_qk,
+                  kk > 0 ? 1u : 0u);
+        }
+        umma_commit(BAR(kBSF + (it & 1)));
+        umma_commit(BAR(kBKE + ks));
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int it = 0; ok && it < n_iter; ++it) {
+        if (it + 1 < n_iter && !issue_s(it + 1)) break;
+        const int vs = it % C::kVStages, vu = it / C::kVStages;
+        if (!mbar_wait(BAR(kBPF + (it & 1)), (it >> 1) & 1, abort_flag, a.status)) break;
+        if (!mbar_wait(BAR(kBVF + vs), vu & 1, abort_flag, a.status)) break;
+        tc_fence_after();
+        const uint32_t vb = sbase + C::kVOff + vs * C::kVBytes;
+        const uint32_t pa = tmem + static_cast<uint32_t>((it & 1) * 128);
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          umma_ts(tmem + C::kOCol, pa + kk * 8, sw128_desc(vb + kk * 2048, C::kPanel, 1024),
+                  idesc_pv, (it > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(BAR(kBOD));
+        umma_commit(BAR(kBVE + vs));
+        if (it == n_iter - 1) umma_commit(BAR(kBOFin));  // the final O is complete
+      }
+      if (*abort_flag) {
+        // Drain: wait (time-limited) for the MMAs issued so far before TMEM is released.
+        umma_commit(BAR(kBDrain));
+        mbar_wait_limited(BAR(kBDrain), 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int64_t i = static_cast<int64_t>(mt) * 128 + r;
+    const bool row_ok = i < a.Sq;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int it = 0; it < n_iter; ++it) {
+      const int sb = it & 1;
+      const bool w_ok = mbar_wait(BAR(kBSF + sb), (it >> 1) & 1, abort_flag, a.status);
+      if (!__all_sync(0xFFFFFFFFu, w_ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t u[128];
+      tmem_ld32(tl + sb * 128 + 0, u + 0);
+      tmem_ld32(tl + sb * 128 + 32, u + 32);
+      tmem_ld32(tl + sb * 128 + 64, u + 64);
+      tmem_ld32(tl + sb * 128 + 96, u + 96);
+      tmem_wait_ld();
+      float x[128];
+#pragma unroll
+      for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(u[c]);
+      if (it >= n_full) {
+        // partial tile: element mask
+        const int nt = __ldg(list + it);
+        const int64_t n0 = static_cast<int64_t>(nt) * 128;
+        int64_t lim = a.Sk;
+        if (a.causal) lim = min64(lim, i + 1);
+        const int lim_c = static_cast<int>(max64(0, min64(128, lim - n0)));
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= lim_c) x[c] = -INFINITY;
+        if (row_ok && a.mode == SA_MODE_BLOCK && a.bs == 64) {
+          const uint8_t* mrow = a.mask + (bg * a.Mb + i / 64) * a.Nb;
+          const int c0 = static_cast<int>(n0 / 64);
+          const bool m0 = __ldg(mrow + c0) != 0;
+          const bool m1 = (c0 + 1 < a.Nb) ? (__ldg(mrow + c0 + 1) != 0) : false;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (!(c < 64 ? m0 : m1)) x[c] = -INFINITY;
+        } else if (row_ok && a.mode == SA_MODE_INDEX) {
+          const uint32_t* brow = a.bitmap + (bg * a.Sq + i) * a.W;
+          const int w0 = static_cast<int>(n0 / 32);
+          uint32_t wd[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) wd[k] = (w0 + k < a.W) ? __ldg(brow + w0 + k) : 0u;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (!((wd[c >> 5] >> (c & 31)) & 1u)) x[c] = -INFINITY;
+        }
+      }
+      float mx = x[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+      const float m_tile = mx * a.scale_log2;
+      // Lazy rescale: only when this row's max grows by more than 2^8; the decision is
+      // taken per warp so that the warp-collective TMEM accesses stay converged.
+      const bool need = m_tile > m_run + 8.0f;
+      if (__any_sync(0xFFFFFFFFu, need)) {
+        const float alpha = need ? ex2(m_run - m_tile) : 1.f;  // 0 when m_run = -inf
+        if (it > 0) {
+          // O holds P V up to tile it-1: rescale it in TMEM once that MMA is done.
+          bool w_ok = mbar_wait(BAR(kBOD), (it - 1) & 1, abort_flag, a.status);
+          if (!__all_sync(0xFFFFFFFFu, w_ok)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < DV; c += 32) {
+            uint32_t ov[32];
+            tmem_ld32(tl + C::kOCol + c, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st32(tl + C::kOCol + c, ov);
+          }
+          tmem_wait_st();
+        }
+        if (need) {
+          l_run *= alpha;
+          m_run = m_tile;
+        }
+      }
+      const float m_eff = (m_run == -INFINITY) ? 0.f : m_run;
+      const float sc = a.scale_log2;
+      float psum = 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2(fmaf(x[c0 + 2 * e], sc, -m_eff));
+          const float p1 = ex2(fmaf(x[c0 + 2 * e + 1], sc, -m_eff));
+          psum += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tl + sb * 128 + c0 / 2, pk);
+      }
+      l_run += psum;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(BAR(kBPF + sb));
+    }
+    // ---------------------------------------------------------------- epilogue
+    if (n_iter > 0 && ok) {
+      const bool w_ok = mbar_wait(BAR(kBOFin), 0, abort_flag, a.status);
+      ok = __all_sync(0xFFFFFFFFu, w_ok);
+      tc_fence_after();
+    }
+    const bool have_o = n_iter > 0 && ok;  // warp-uniform
+    const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) +
+                          ((b * a.Sq + i) * a.HQ + h) * static_cast<int64_t>(DV);
+#pragma unroll 1
+    for (int c = 0; c < DV; c += 32) {
+      uint32_t ov[32];
+      if (have_o) {
+        tmem_ld32(tl + C::kOCol + c, ov);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) ov[e] = 0u;
+      }
+      if (row_ok) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv,
+                              __uint_as_float(ov[2 * e + 1]) * inv);
+        uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+      }
+    }
+    if (row_ok) {
+      const float m_eff = (m_run == -INFINITY) ? 0.f : m_run;
+      a.lse[(static_cast<int64_t>(b) * a.HQ + h) * a.Sq + i] =
+          (l_run > 0.f) ? (m_eff + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int DQK, int DV>
+static int launch_fwd_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
+  using C = FwdCfg<DQK, DV>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(sparse_fwd_kernel<DQK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmem) != cudaSuccess)
+      return SA_ERR_CUDA;
+    attr_set = true;
+  }
+  dim3 grid(a.Tm, a.HQ, a.B);
+  sparse_fwd_kernel<DQK, DV><<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.v, a);
+  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+int launch_fwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
+  if (a.Dqk == 64 && a.Dv == 64) return launch_fwd_t<64, 64>(a, m, st);
+  if (a.Dqk == 128 && a.Dv == 128) return launch_fwd_t<128, 128>(a, m, st);
+  if (a.Dqk == 192 && a.Dv == 128) return launch_fwd_t<192, 128>(a, m, st);
+  if (a.Dqk == 256 && a.Dv == 256) return launch_fwd_t<256, 256>(a, m, st);
+  return SA_ERR_UNSUPPORTED;
+}
+
+}  // namespace sa

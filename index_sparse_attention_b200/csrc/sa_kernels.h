@@ -1,0 +1,44 @@
+// sa_kernels.h -- host-side launch interface shared by the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sparse_attn.h"
+
+namespace sa {
+
+// Everything a forward or backward launch needs besides the TMA tensor maps.
+struct AttnArgs {
+  void* o;               // bf16 [B][Sq][HQ][Dv]
+  float* lse;            // fp32 [B][HQ][Sq]
+  const void* dout;      // bf16 [B][Sq][HQ][Dv]
+  void* dq;              // bf16 [B][Sq][HQ][Dqk]
+  void* dk;              // bf16 [B][Sk][HK][Dqk]
+  void* dv;              // bf16 [B][Sk][HK][Dv]
+  float* delta;          // fp32 [B][HQ][Sq]   (backward workspace)
+  float* dq_acc;         // fp32 [B][Sq][HQ][Dqk] (backward workspace)
+  const int32_t* cnt;    // forward lists
+  const int32_t* idx;
+  const int32_t* tcnt;   // backward (transposed) lists
+  const int32_t* tidx;
+  const uint8_t* mask;   // block mode, bs = 64 partial tiles
+  const uint32_t* bitmap;  // index mode
+  int64_t Sq, Sk;
+  int B, HQ, HK, Dqk, Dv;
+  int Tm, Tn, W;
+  int mode, causal, bs, Mb, Nb;
+  float scale;       // softmax_scale
+  float scale_log2;  // softmax_scale * log2(e)
+  int32_t* status;
+};
+
+struct TensorMaps {
+  CUtensorMap q, k, v, o, dout;
+};
+
+int launch_fwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st);
+int launch_bwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st);
+
+}  // namespace sa
