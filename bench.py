@@ -1,0 +1,440 @@
+"""Benchmark: effective fwd+bwd TFLOP/s of block-/index-sparse attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one pass of the whole path over one batch of synthetic input resident in
+HBM: tile lists from the block mask (or top-k indices), the forward (O, LSE) and the
+backward (Delta, dQ/dK/dV, dQ cast).  The metric counts tensor-core work of ACTIVE
+128x128 tiles only, per query head: forward 2*128*128*(Dqk+Dv) and backward
+2*128*128*(3*Dqk+2*Dv) per tile (partial tiles count in full).  Rank 0 prints one
+JSON line.  With N > 1 (torchrun) every rank runs the same workload on its own GPU
+(independent replicas, weak scaling) and the time is the max over ranks.
+
+`--impl reference` times the fp64 CPU oracle (the reference implementation of the
+operation in this project) on a bounded sample of the same workload and prints the
+same JSON line with "impl": "reference".
+"""
+import argparse
+import ctypes
+import datetime
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from index_sparse_attention_b200 import inputs as I  # noqa: E402
+
+METRIC = "effective TFLOP/s fwd+bwd (active blocks only), % of B200 bf16 tensor peak"
+DEFAULT_WORKLOAD = "long_causal_blocksparse_h16_s32768_d256"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def tile_flops(w):
+    """(forward, backward) tensor-core FLOP of one active 128x128 tile for one query head."""
+    return 2 * 128 * 128 * (w.Dqk + w.Dv), 2 * 128 * 128 * (3 * w.Dqk + 2 * w.Dv)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return json.load(open(p)), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def bwd_source_sha():
+    h = hashlib.sha256()
+    for f in ("bwd.cu", "sa_device.cuh"):
+        h.update(open(os.path.join(ROOT, "index_sparse_attention_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch of the backward main kernel from a committed ncu summary,
+    or None when absent or taken on a different kernel source."""
+    p = os.path.join(ROOT, "profiles", "bwd_main_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("source_sha") != bwd_source_sha() or d.get("workload") != workload:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi (read-only) while timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu, self.proc, self.lines = gpu_index, None, []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(self.NAMES, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# -----------------------------------------------------------------------------------
+# CPU oracle: the cpu_baseline leg and the reference arm
+# -----------------------------------------------------------------------------------
+def active_tiles_per_row(w, inp):
+    """Active key tiles of each (b, KV head, query tile), from the mask or indices."""
+    Mt, Nt = -(-w.Sq // 128), -(-w.Sk // 128)
+    if w.mode == "block":
+        r = 128 // w.bs
+        m = np.zeros((w.B, w.HK, Mt * r, Nt * r), np.uint8)
+        m[:, :, :inp.mask.shape[2], :inp.mask.shape[3]] = inp.mask
+        act = m.reshape(w.B, w.HK, Mt, r, Nt, r).max(axis=(3, 5))
+        if w.causal:
+            act = act * np.tril(np.ones((Mt, Nt), np.uint8))[None, None]
+        return act.sum(-1)
+    out = np.zeros((w.B, w.HK, Mt), np.int64)
+    for b in range(w.B):
+        for g in range(w.HK):
+            for mt in range(Mt):
+                rows = inp.idx[b, mt * 128:(mt + 1) * 128, g]
+                ii = np.arange(mt * 128, mt * 128 + rows.shape[0])[:, None]
+                ok = (rows >= 0) & ((rows <= ii) if w.causal else True)
+                out[b, g, mt] = len(np.unique(rows[ok] // 128))
+    return out
+
+
+class OracleSampler:
+    """Times the fp64 oracle on whole query tiles of the workload.
+
+    Per sampled query tile (all 128 rows of one (b, h, m-tile)) the oracle computes the
+    forward (O, LSE), Delta and the row side of the backward (recomputed S, dP, dS and
+    dQ).  Work credited per active tile: 2*128*128*((Dqk+Dv) + (2*Dqk+Dv)) FLOP, i.e.
+    the forward plus the S, dP and dQ contractions of the backward.
+    """
+
+    def __init__(self, w, inp, seed=0):
+        import oracle
+        self.oracle = oracle
+        self.w, self.inp = w, inp
+        self.P = oracle.Problem(inp.f32("q"), inp.f32("k"), inp.f32("v"), scale=w.scale,
+                                causal=w.causal, mode=w.mode, mask=inp.mask, bs=w.bs, idx=inp.idx)
+        self.do = inp.f32("do")
+        self.act = active_tiles_per_row(w, inp)
+        self.rng = np.random.default_rng(seed)
+        self.per_tile = 2 * 128 * 128 * ((w.Dqk + w.Dv) + (2 * w.Dqk + w.Dv))
+        self.cores = len(os.sched_getaffinity(0))
+
+    def run_tile(self):
+        w, o_ = self.w, self.oracle
+        G = w.HQ // w.HK
+        b, h = int(self.rng.integers(w.B)), int(self.rng.integers(w.HQ))
+        mt = int(self.rng.integers(-(-w.Sq // 128)))
+        i = np.arange(mt * 128, min(mt * 128 + 128, w.Sq))
+        rows = np.stack([np.full(len(i), b), np.full(len(i), h), i], 1).astype(np.int64)
+        o, lse = o_.forward_rows(self.P, rows)
+        lse_full = np.zeros((w.B, w.HQ, w.Sq))
+        dlt_full = np.zeros((w.B, w.HQ, w.Sq))
+        lse_full[b, h, i] = lse
+        dlt_full[b, h, i] = np.einsum("nd,nd->n", self.do[b, i, h].astype(np.float64), o)
+        o_.backward_rows(self.P, self.do, lse_full, dlt_full, rows)
+        return int(self.act[b, h // G, mt]) * self.per_tile
+
+    def run_for(self, seconds, max_tiles=100000):
+        flop, t0, n = 0, time.perf_counter(), 0
+        while time.perf_counter() - t0 < seconds and n < max_tiles:
+            flop += self.run_tile()
+            n += 1
+        return flop, time.perf_counter() - t0, n
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:  # under torchrun only rank 0 runs the CPU reference
+        return
+    os.environ.setdefault("OMP_NUM_THREADS", str(len(os.sched_getaffinity(0))))
+    w = I.WORKLOADS[args.workload]
+    inp = I.make_inputs(w)
+    s = OracleSampler(w, inp)
+    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        s.run_for(per_step)
+    flop, sec, tiles = 0, 0.0, 0
+    for _ in range(args.steps):
+        f, t, n = s.run_for(per_step)
+        flop, sec, tiles = flop + f, sec + t, tiles + n
+    value = flop / sec / 1e12
+    sample = (f"{tiles} whole query tiles (128 rows of one (b, h, m-tile)) drawn at random over "
+              f"{args.steps} steps of ~{per_step:.0f} s: fp64 forward + Delta + dQ-side backward "
+              f"rows; credited 2*128^2*((Dqk+Dv)+(2*Dqk+Dv)) FLOP per active tile")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": int(args.gpus), "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * sec / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, None),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": s.cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, active):
+    cfg = {"workload": w.name, "B": w.B, "HQ": w.HQ, "HK": w.HK, "Sq": w.Sq, "Sk": w.Sk,
+           "Dqk": w.Dqk, "Dv": w.Dv, "mode": w.mode, "causal": w.causal, "parallelism": "replicas"}
+    if w.mode == "block":
+        cfg.update(block=w.bs, density=w.density)
+    else:
+        cfg.update(topk=w.topk)
+    if active is not None:
+        cfg["active_tile_heads"] = active
+    in_bytes = 2 * (w.B * w.Sq * w.HQ * (w.Dqk + w.Dv) + w.B * w.Sk * w.HK * (w.Dqk + w.Dv))
+    cfg["l2"] = (f"inputs larger than L2: q, k, v, dO = {in_bytes / 2**20:.0f} MiB > 126 MiB"
+                 if in_bytes > L2_BYTES else "L2 flushed between steps (256 MiB write)")
+    return cfg
+
+
+# -----------------------------------------------------------------------------------
+# GPU arm
+# -----------------------------------------------------------------------------------
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local))
+
+    import index_sparse_attention_b200 as sa
+    from index_sparse_attention_b200 import _lib
+
+    L = _lib.load()
+    w = I.WORKLOADS[args.workload]
+    inp = I.make_inputs(w)
+    dev = torch.device("cuda", local)
+
+    def bf(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+
+    host = {"q": bf(inp.q), "k": bf(inp.k), "v": bf(inp.v), "do": bf(inp.do)}
+    if w.mode == "block":
+        host["mask"] = torch.from_numpy(inp.mask)
+    else:
+        host["idx"] = torch.from_numpy(inp.idx)
+    g = {k: v.to(dev) for k, v in host.items()}
+    flush = None
+    in_bytes = sum(t.numel() * t.element_size() for t in g.values())
+    if in_bytes <= L2_BYTES:
+        flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+
+    def lists():
+        if w.mode == "block":
+            return sa.block_mask_to_block_sparse(g["mask"], w.B, w.HK, w.Sq, w.Sk, bs=w.bs,
+                                                 causal=w.causal)
+        return sa.index_to_block_sparse(g["idx"], w.Sk, causal=w.causal)
+
+    ws = torch.empty(sa.sparse_attn_bwd_workspace_size(g["q"], g["k"], g["v"], lists()),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty((w.B, w.Sq, w.HQ, w.Dv), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.HQ, w.Sq), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(g["q"]), torch.empty_like(g["k"]), torch.empty_like(g["v"])
+
+    def step(src=None):
+        bsp = lists()
+        sa.sparse_attn_fwd(g["q"], g["k"], g["v"], bsp, w.scale, o=o, lse=lse)
+        sa.sparse_attn_bwd(g["q"], g["k"], g["v"], o, lse, g["do"], bsp, w.scale, dq=dq, dk=dk,
+                           dv=dv, workspace=ws)
+        return bsp
+
+    bsp = step()
+    torch.cuda.synchronize()
+    active = bsp.active_tiles() * (w.HQ // w.HK)  # tile x query-head units
+    fwd_f, bwd_f = tile_flops(w)
+    flop_step = active * (fwd_f + bwd_f)
+
+    for _ in range(args.warmup):
+        step()
+        if flush is not None:
+            flush.zero_()
+    torch.cuda.synchronize()
+
+    # per-step events: 6 inside the library (fwd, bwd pre/main/post) + step bounds
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    stream = torch.cuda.current_stream(dev)
+    for row in evs:
+        for e in row:
+            e.record(stream)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches_per_step = (3 if w.mode == "block" else 4) + 1 + 3 + (1 if flush is not None else 0)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for s in range(args.steps):
+            arr = (ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in evs[s]])
+            L.sparse_attn_set_timing_events(arr)
+            step()
+            if flush is not None:
+                flush.zero_()
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    L.sparse_attn_set_timing_events(None)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    per_kernel = {
+        "fwd": float(np.mean([r[0].elapsed_time(r[1]) for r in evs])),
+        "bwd_pre": float(np.mean([r[2].elapsed_time(r[3]) for r in evs])),
+        "bwd_main": float(np.mean([r[3].elapsed_time(r[4]) for r in evs])),
+        "bwd_post": float(np.mean([r[4].elapsed_time(r[5]) for r in evs])),
+    }
+    ms_step = ms / args.steps
+    value = world * flop_step / (ms_step * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers: H2D of the inputs, the whole
+    # path, D2H of every output, per step
+    pin = {k: v.pin_memory() for k, v in host.items()}
+    outs = [o, lse, dq, dk, dv]
+    pin_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    e_steps = max(1, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e_steps):
+        for k in pin:
+            g[k].copy_(pin[k], non_blocking=True)
+        step()
+        for src, dst in zip(outs, pin_out):
+            dst.copy_(src, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1) / e_steps
+    if world > 1:
+        t = torch.tensor([e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+    e2e_value = world * flop_step / (e_ms * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    clocks = clk.summary()
+    if rank == 0:
+        peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        achieved = active * bwd_f / (per_kernel["bwd_main"] * 1e-3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": workload_config(w, active),
+            "pct_of_bf16_peak": 100.0 * (value / world) / peak,
+            "pct_basis": f"bf16_tflops_sustained {peak:.1f} TFLOP/s ({peak_src})",
+            "flop_per_step": flop_step, "kernel_ms": per_kernel,
+            "roofline": {
+                "kernel": "sparse_bwd_kernel", "bound": "tensor", "achieved": achieved,
+                "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_kind": f"bf16_tflops_sustained ({'of measured' if peak_src == 'measured' else 'of fallback'}); burst {peak_burst:.1f}",
+                "traffic": profiled_traffic(w.name),
+                "algorithmic": "2*128*128*(3*Dqk+2*Dv) FLOP per active tile x query head",
+            },
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e_ms},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            os.environ.setdefault("OMP_NUM_THREADS", str(len(os.sched_getaffinity(0))))
+            s = OracleSampler(w, inp)
+            s.run_tile()  # load and warm the library
+            f, sec, n = s.run_for(args.cpu_seconds)
+            line["cpu_baseline"] = {
+                "value": f / sec / 1e12, "unit": "TFLOP/s", "cores": s.cores, "kind": "oracle",
+                "sample": (f"{n} random whole query tiles of the workload, {sec:.1f} s: fp64 "
+                           "forward + Delta + dQ-side backward rows; credited "
+                           "2*128^2*((Dqk+Dv)+(2*Dqk+Dv)) FLOP per active tile")}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(I.WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

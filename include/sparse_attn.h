@@ -159,6 +159,18 @@ size_t sparse_attn_bwd_workspace_size(const sparse_attn_params *p);
 int sparse_attn_bwd(const sparse_attn_params *p, void *workspace, size_t workspace_bytes,
                     sa_stream_t stream);
 
+/*
+ * sparse_attn_set_timing_events -- optional instrumentation (no counterpart on the
+ * pages; it serves the benchmark's per-kernel timing).  `events` points to six
+ * cudaEvent_t handles created by the caller, or is NULL to switch recording off.
+ * While set, sparse_attn_fwd records events[0] before and events[1] after its kernel,
+ * and sparse_attn_bwd records events[2] before the preprocess, events[3] before the
+ * main kernel, events[4] after it and events[5] after the postprocess, each on the
+ * call's stream.  Process-wide setting, not synchronised: set it while no other
+ * thread calls into the library.  Returns SA_OK.
+ */
+int sparse_attn_set_timing_events(void *const *events);
+
 /* Static description of an SA_* code. */
 const char *sparse_attn_error_string(int code);
 

@@ -32,6 +32,7 @@ EXPORTS = (
     "sparse_attn_fwd",
     "sparse_attn_bwd_workspace_size",
     "sparse_attn_bwd",
+    "sparse_attn_set_timing_events",
     "sparse_attn_error_string",
 )
 
@@ -81,6 +82,8 @@ def load():
     L.sparse_attn_bwd_workspace_size.restype = ctypes.c_size_t
     L.sparse_attn_bwd.argtypes = [P_p, vp, ctypes.c_size_t, vp]
     L.sparse_attn_bwd.restype = ctypes.c_int
+    L.sparse_attn_set_timing_events.argtypes = [vp]
+    L.sparse_attn_set_timing_events.restype = ctypes.c_int
     L.sparse_attn_error_string.argtypes = [ctypes.c_int]
     L.sparse_attn_error_string.restype = ctypes.c_char_p
     _lib = L

@@ -9,6 +9,11 @@
 
 using namespace sa;
 
+namespace sa {
+cudaEvent_t* g_timing_events = nullptr;
+static cudaEvent_t g_events_copy[6];
+}  // namespace sa
+
 namespace {
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -25,16 +30,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 4-D map over a [B][S][H][D] bf16 tensor with 64 x 128 (D x S) boxes, 128-byte swizzle.
-// Out-of-range rows read as zeros.
-bool make_map(CUtensorMap* m, const void* base, int D, int64_t S, int H, int B) {
+// 4-D map over a [B][S][H][D] bf16 tensor with 64 x box_rows (D x S) boxes, 128-byte
+// swizzle.  Out-of-range rows (and columns) read as zeros.
+bool make_map(CUtensorMap* m, const void* base, int D, int64_t S, int H, int B, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S),
                         static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(H) * D * 2, static_cast<cuuint64_t>(D) * 2,
                            static_cast<cuuint64_t>(S) * H * D * 2};
-  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -109,14 +114,15 @@ int fill_args(const sparse_attn_params* p, AttnArgs* a, bool backward) {
   return SA_OK;
 }
 
+// Forward: Q in 128-row boxes.  Backward: Q and dO in 64-row boxes (the backward
+// consumes query tiles in 64-row halves).  K and V: 128-row boxes.
 int fill_maps(const sparse_attn_params* p, TensorMaps* m, bool backward) {
-  if (!make_map(&m->q, p->q, p->Dqk, p->Sq, p->HQ, p->B)) return SA_ERR_CUDA;
-  if (!make_map(&m->k, p->k, p->Dqk, p->Sk, p->HK, p->B)) return SA_ERR_CUDA;
-  if (!make_map(&m->v, p->v, p->Dv, p->Sk, p->HK, p->B)) return SA_ERR_CUDA;
-  if (backward) {
-    if (!make_map(&m->o, p->o, p->Dv, p->Sq, p->HQ, p->B)) return SA_ERR_CUDA;
-    if (!make_map(&m->dout, p->dout, p->Dv, p->Sq, p->HQ, p->B)) return SA_ERR_CUDA;
-  }
+  const int qrows = backward ? 64 : 128;
+  if (!make_map(&m->q, p->q, p->Dqk, p->Sq, p->HQ, p->B, qrows)) return SA_ERR_CUDA;
+  if (!make_map(&m->k, p->k, p->Dqk, p->Sk, p->HK, p->B, 128)) return SA_ERR_CUDA;
+  if (!make_map(&m->v, p->v, p->Dv, p->Sk, p->HK, p->B, 128)) return SA_ERR_CUDA;
+  if (backward && !make_map(&m->dout, p->dout, p->Dv, p->Sq, p->HQ, p->B, qrows))
+    return SA_ERR_CUDA;
   return SA_OK;
 }
 
@@ -135,6 +141,16 @@ extern "C" const char* sparse_attn_error_string(int code) {
     case SA_ERR_WORKSPACE: return "workspace missing or too small";
     default: return "unknown error code";
   }
+}
+
+extern "C" int sparse_attn_set_timing_events(void* const* events) {
+  if (!events) {
+    g_timing_events = nullptr;
+    return SA_OK;
+  }
+  for (int k = 0; k < 6; ++k) g_events_copy[k] = static_cast<cudaEvent_t>(events[k]);
+  g_timing_events = g_events_copy;
+  return SA_OK;
 }
 
 extern "C" int sparse_attn_fwd(const sparse_attn_params* p, sa_stream_t stream) {

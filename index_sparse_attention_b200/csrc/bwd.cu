@@ -1,6 +1,534 @@
-// bwd.cu -- placeholder until the backward kernels land.
+// bwd.cu -- sparse attention backward on sm_100a: dQ, dK, dV.
+//
+// Operation (MagiAttention PR #334, Summary and section 1): recompute P from the
+// saved LSE, then dV += P^T dO, dP = dO V^T, dS = P * (dP - Delta), dQ += dS K,
+// dK += dS^T Q, with Delta = rowsum(dO * O) from a preprocess kernel and a
+// postprocess that multiplies the fp32 dQ accumulator by softmax_scale and casts
+// (section 3: fp32 accumulation, then dtype conversion and softmax_scale scaling).
+//
+// B200 design.  The pages' two loop orders put either dQ or dK/dV in tensor memory.
+// Here the key tile is stationary (the transposed, key-to-query lists of MagiAttention
+// PR #331 "CSR Tile Mapping"): one CTA owns 128 keys of one (batch, KV head) and walks
+// every query tile that attends to them, for every query head of the GQA group, so
+// dK and dV accumulate in TMEM across the whole group and are stored once, with no
+// atomics.  Query tiles are consumed in 64-row halves so that K, V, a double-buffered
+// Q/dO half-tile and the dS^T staging tile fit in shared memory for every head dim.
+// For each 64-query half:
+//   S^T  = K Q^T      (M=128 keys, N=64)            -> TMEM  [SS]
+//   dP^T = V dO^T     (M=128 keys, N=64)            -> TMEM  [SS]
+//   elementwise warps: P^T = exp2(S^T*scale*log2e - LSE*log2e), dS^T = P^T (dP^T - Delta),
+//     element mask on partial tiles; bf16 P^T and dS^T written back into TMEM (A
+//     operands of the next two MMAs) and dS^T into shared memory (operand of dQ^T)
+//   dV  += P^T dO     (M=128 keys, N=Dv chunk)      TMEM A operand   [TS]
+//   dK  += dS^T Q     (M=128 keys, N=Dqk chunk)     TMEM A operand   [TS]
+//   dQ^T = K^T dS^T   (M=128 head-dim window, N=64) both MN-major    [SS]
+//   the same warps drain dQ^T from TMEM and add it (fp32 reductions, coalesced along
+//   the head dim) into the dQ accumulator.
+// When Dqk + Dv does not leave room in the 512 TMEM columns (192/128 and 256/256),
+// the head dim of dK/dV/dQ is split over two CTAs, each recomputing S^T and dP^T.
+// Every mbarrier wait is bounded (see sa_device.cuh).
 #include "sa_device.cuh"
 #include "sa_kernels.h"
+
 namespace sa {
-int launch_bwd(const AttnArgs&, const TensorMaps&, cudaStream_t) { return SA_ERR_UNSUPPORTED; }
+
+// ------------------------------------------------------------------------------------
+// preprocess: Delta = rowsum(dO * O) (fp32) and a zeroed dQ accumulator
+// ------------------------------------------------------------------------------------
+__global__ void bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
+                               const __nv_bfloat16* __restrict__ dout, float* __restrict__ delta,
+                               float* __restrict__ dq_acc, int64_t rows, int64_t Sq, int HQ,
+                               int Dv, int Dqk) {
+  const int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  // row = (b * Sq + i) * HQ + h  (the order of o / dout)
+  const uint4* po = reinterpret_cast<const uint4*>(o + row * Dv);
+  const uint4* pd = reinterpret_cast<const uint4*>(dout + row * Dv);
+  float acc = 0.f;
+  for (int c = lane; c < Dv / 8; c += 32) {
+    const uint4 a = __ldg(po + c), d = __ldg(pd + c);
+    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&d);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = __bfloat1622float2(a2[e]), y = __bfloat1622float2(d2[e]);
+      acc = fmaf(x.x, y.x, acc);
+      acc = fmaf(x.y, y.y, acc);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+  const int64_t bi = row / HQ;
+  const int h = static_cast<int>(row % HQ);
+  const int64_t b = bi / Sq, i = bi % Sq;
+  if (lane == 0) delta[(b * HQ + h) * Sq + i] = acc;
+  float4* z = reinterpret_cast<float4*>(dq_acc + row * Dqk);
+  for (int c = lane; c < Dqk / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// ------------------------------------------------------------------------------------
+// postprocess: dQ = bf16(softmax_scale * dQ_acc)
+// ------------------------------------------------------------------------------------
+__global__ void bwd_post_kernel(const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dq,
+                                int64_t n4, float scale) {
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n4;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(dq_acc) + e);
+    uint2 out;
+    out.x = pack_bf16x2(v.x * scale, v.y * scale);
+    out.y = pack_bf16x2(v.z * scale, v.w * scale);
+    reinterpret_cast<uint2*>(dq)[e] = out;
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// main kernel
+// ------------------------------------------------------------------------------------
+// DQK, DV: the head dims the kernel is built for (64-wide inputs run through the
+// 128 instance with zero-filled loads); NSPLIT: CTAs sharing one key tile, each owning
+// one head-dim chunk of dK / dV / dQ.
+template <int DQK, int DV, int NSPLIT>
+struct BwdCfg {
+  static constexpr int kBM = 64;                     // queries per inner step
+  static constexpr int kKPanel = 128 * 128;          // [128 rows x 64 cols] bf16 panel
+  static constexpr int kQPanel = kBM * 128;          // [64 rows x 64 cols] bf16 panel
+  static constexpr int kKBytes = 128 * DQK * 2;
+  static constexpr int kVBytes = 128 * DV * 2;
+  static constexpr int kQBytes = kBM * DQK * 2;
+  static constexpr int kOBytes = kBM * DV * 2;
+  static constexpr int kStages = (DQK + DV >= 512) ? 1 : 2;
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kKOff + kKBytes;
+  static constexpr int kQOff = kVOff + kVBytes;                    // per stage: Q then dO
+  static constexpr int kStageBytes = kQBytes + kOBytes;
+  static constexpr int kDSOff = kQOff + kStages * kStageBytes;     // dS^T [128 keys][64 q]
+  static constexpr int kLOff = kDSOff + 128 * kBM * 2;             // per stage: lse2[64], delta[64]
+  static constexpr int kBarOff = kLOff + kStages * 2 * kBM * 4;
+  static constexpr int kSmem = kBarOff + 256 + 1024;
+  static constexpr int kThreads = 192;
+  // head-dim chunks of this CTA: dK [kc0, kc0 + kcn), dV [vc0, vc0 + vcn)
+  static constexpr int kDKMax = NSPLIT == 1 ? DQK : (DQK == 192 ? 128 : DQK / 2);
+  static constexpr int kDVMax = DV / NSPLIT;
+  // TMEM columns
+  static constexpr uint32_t kColS = 0;
+  static constexpr uint32_t kColDP = 64;
+  static constexpr uint32_t kColDQ = 128;
+  static constexpr uint32_t kColDK = 192;
+  static constexpr uint32_t kColDV = kColDK + kDKMax;
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(kColDV + kDVMax <= kTmemCols, "tensor memory budget");
+  static_assert(kSmem <= 227 * 1024, "shared memory budget");
+};
+
+enum : int { kBKV = 0, kBQF = 1, kBQE = 3, kBLF = 5, kBSF = 7, kBPF = 8, kBDQF = 9, kBDQE = 10,
+             kBFin = 11, kBDrainB = 12, kNumBarsB = 13 };
+
+template <int DQK, int DV, int NSPLIT>
+__global__ void __launch_bounds__(192, 1)
+    sparse_bwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_do, const AttnArgs a) {
+  using C = BwdCfg<DQK, DV, NSPLIT>;
+  constexpr int BM = C::kBM;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::kBarOff;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * kNumBarsB);
+  volatile int* abort_flag =
+      reinterpret_cast<volatile int*>(smem + C::kBarOff + 8 * kNumBarsB + 4);
+  auto BAR = [&](int k) { return bar0 + 8u * static_cast<uint32_t>(k); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = static_cast<int>(blockIdx.x) % NSPLIT;
+  const int nt = static_cast<int>(blockIdx.x) / NSPLIT;
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int G = a.HQ / a.HK;
+  const int64_t bg = static_cast<int64_t>(b) * a.HK + g;
+  const int64_t trow = bg * a.Tn + nt;
+  const int n_full = __ldg(a.tcnt + 2 * trow);
+  const int n_mt = n_full + __ldg(a.tcnt + 2 * trow + 1);
+  const int32_t* tlist = a.tidx + trow * a.Tm;
+  const int n_iter = G * n_mt * 2;  // (query head, query tile, 64-row half)
+
+  // head-dim chunks owned by this CTA
+  int kc0, kcn, vc0, vcn, qw0;  // qw0: first head-dim row of the 128-wide dQ^T window
+  if (NSPLIT == 1) {
+    kc0 = 0; kcn = DQK; vc0 = 0; vcn = DV; qw0 = 0;
+  } else if (DQK == 192) {
+    kc0 = split == 0 ? 0 : 128; kcn = split == 0 ? 128 : 64;
+    vc0 = split * 64; vcn = 64;
+    qw0 = split == 0 ? 0 : 64;
+  } else {
+    kc0 = split * (DQK / 2); kcn = DQK / 2; vc0 = split * (DV / 2); vcn = DV / 2;
+    qw0 = split * (DQK / 2);
+  }
+  const int dqk_real = a.Dqk, dv_real = a.Dv;  // 64 when run through the 128 instance
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(kBKV), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR(kBQF + s), 1);
+      mbar_init(BAR(kBQE + s), 1);
+      mbar_init(BAR(kBLF + s), 32);
+    }
+    mbar_init(BAR(kBSF), 1);
+    mbar_init(BAR(kBPF), 128);
+    mbar_init(BAR(kBDQF), 1);
+    mbar_init(BAR(kBDQE), 128);
+    mbar_init(BAR(kBFin), 1);
+    mbar_init(BAR(kBDrainB), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // iteration -> (query head, query tile, half)
+  auto decode = [&](int it, int& h, int& m0, bool& partial) {
+    const int per_head = 2 * n_mt;
+    const int hh = it / per_head;
+    const int rest = it - hh * per_head;
+    const int k = rest >> 1;
+    h = g * G + hh;
+    m0 = __ldg(tlist + k) * 128 + (rest & 1) * BM;
+    partial = k >= n_full;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (n_iter > 0) {
+      if (lane == 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        prefetch_tensormap(&tm_do);
+        mbar_arrive_expect_tx(BAR(kBKV), C::kKBytes + C::kVBytes);
+        for (int c = 0; c < DQK / 64; ++c)
+          tma_load_4d(sbase + C::kKOff + c * C::kKPanel, &tm_k, BAR(kBKV), c * 64, nt * 128, g, b);
+        for (int c = 0; c < DV / 64; ++c)
+          tma_load_4d(sbase + C::kVOff + c * C::kKPanel, &tm_v, BAR(kBKV), c * 64, nt * 128, g, b);
+      }
+      float* lbuf = reinterpret_cast<float*>(smem + C::kLOff);
+      for (int it = 0; it < n_iter; ++it) {
+        int h, m0;
+        bool partial;
+        decode(it, h, m0, partial);
+        const int st = it % C::kStages, u = it / C::kStages;
+        const bool w_ok = mbar_wait(BAR(kBQE + st), (u & 1) ^ 1, abort_flag, a.status);
+        if (!__all_sync(0xFFFFFFFFu, w_ok)) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(BAR(kBQF + st), C::kQBytes + C::kOBytes);
+          const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
+          for (int c = 0; c < DQK / 64; ++c)
+            tma_load_4d(qs + c * C::kQPanel, &tm_q, BAR(kBQF + st), c * 64, m0, h, b);
+          for (int c = 0; c < DV / 64; ++c)
+            tma_load_4d(qs + C::kQBytes + c * C::kQPanel, &tm_do, BAR(kBQF + st), c * 64, m0, h, b);
+        }
+        // LSE (in log2 units) and Delta of the 64 queries; +inf / 0 past Sq
+        float* ls = lbuf + st * 2 * BM;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int q = lane + 32 * k;
+          const int64_t i = m0 + q;
+          float l2 = INFINITY, dl = 0.f;
+          if (i < a.Sq) {
+            const int64_t li = (static_cast<int64_t>(b) * a.HQ + h) * a.Sq + i;
+            l2 = __ldg(a.lse + li) * 1.4426950408889634f;
+            dl = __ldg(a.delta + li);
+          }
+          ls[q] = l2;
+          ls[BM + q] = dl;
+        }
+        mbar_arrive(BAR(kBLF + st));
+      }
+      if (lane == 0 && *abort_flag) {
+        mbar_wait_limited(BAR(kBKV), 0);
+        for (int it = max(0, n_iter - 2); it < n_iter; ++it)
+          mbar_wait_limited(BAR(kBQF + it % C::kStages), (it / C::kStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_iter > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(128, BM, 0, 0);      // S^T, dP^T
+      constexpr uint32_t idesc_dq = idesc_bf16(128, BM, 1, 1);     // dQ^T = K^T dS^T
+      const uint32_t idesc_dv = idesc_bf16(128, vcn, 0, 1);        // dV += P^T dO
+      const uint32_t idesc_dk = idesc_bf16(128, kcn, 0, 1);        // dK += dS^T Q
+      const uint32_t kbase = sbase + C::kKOff, vbase = sbase + C::kVOff;
+      const uint32_t dsb = sbase + C::kDSOff;
+      bool ok = mbar_wait(BAR(kBKV), 0, abort_flag, a.status);
+      for (int it = 0; ok && it < n_iter; ++it) {
+        const int st = it % C::kStages, u = it / C::kStages;
+        if (!mbar_wait(BAR(kBQF + st), u & 1, abort_flag, a.status)) break;
+        tc_fence_after();
+        const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
+        const uint32_t os = qs + C::kQBytes;
+#pragma unroll
+        for (int kk = 0; kk < DQK / 16; ++kk) {
+          const uint32_t ka = (kk >> 2) * C::kKPanel + (kk & 3) * 32;
+          const uint32_t qb = (kk >> 2) * C::kQPanel + (kk & 3) * 32;
+          umma_ss(tmem + C::kColS, sw128_desc(kbase + ka, 16, 1024), sw128_desc(qs + qb, 16, 1024),
+                  idesc_s, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < DV / 16; ++kk) {
+          const uint32_t va = (kk >> 2) * C::kKPanel + (kk & 3) * 32;
+          const uint32_t ob = (kk >> 2) * C::kQPanel + (kk & 3) * 32;
+          umma_ss(tmem + C::kColDP, sw128_desc(vbase + va, 16, 1024), sw128_desc(os + ob, 16, 1024),
+                  idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(BAR(kBSF));
+        if (!mbar_wait(BAR(kBPF), it & 1, abort_flag, a.status)) break;
+        tc_fence_after();
+        // dV += P^T dO  and  dK += dS^T Q (K = 64 queries: four k-steps of 16)
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          umma_ts(tmem + C::kColDV, tmem + C::kColS + kk * 8,
+                  sw128_desc(os + (vc0 / 64) * C::kQPanel + kk * 2048, C::kQPanel, 1024), idesc_dv,
+                  (it > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          umma_ts(tmem + C::kColDK, tmem + C::kColDP + kk * 8,
+                  sw128_desc(qs + (kc0 / 64) * C::kQPanel + kk * 2048, C::kQPanel, 1024), idesc_dk,
+                  (it > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(BAR(kBQE + st));
+        // dQ^T = K^T dS^T over the 128 keys, once the previous dQ^T has been drained
+        if (!mbar_wait(BAR(kBDQE), (it & 1) ^ 1, abort_flag, a.status)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          umma_ss(tmem + C::kColDQ,
+                  sw128_desc(kbase + (qw0 / 64) * C::kKPanel + kk * 2048, C::kKPanel, 1024),
+                  sw128_desc(dsb + kk * 2048, C::kKPanel, 1024), idesc_dq, kk > 0 ? 1u : 0u);
+        umma_commit(BAR(kBDQF));
+      }
+      umma_commit(BAR(kBFin));
+    }
+  } else {
+    // ------------------------------------------------------- elementwise + dQ drain
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;           // key row of the tile = TMEM lane
+    const int64_t j = static_cast<int64_t>(nt) * 128 + r;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const float* lbuf = reinterpret_cast<const float*>(smem + C::kLOff);
+    uint8_t* dsrow = smem + C::kDSOff + r * 128;
+    // head-dim rows of the dQ^T window drained by this thread
+    const int dq_d = qw0 + r;
+    const bool dq_mine = (NSPLIT == 1 || DQK != 192) ? (r < 128 && dq_d < dqk_real)
+                                                      : (dq_d >= kc0 && dq_d < kc0 + kcn);
+    bool ok = true;
+    for (int it = 0; it < n_iter; ++it) {
+      int h, m0;
+      bool partial;
+      decode(it, h, m0, partial);
+      const int st = it % C::kStages, u = it / C::kStages;
+      bool w_ok = mbar_wait(BAR(kBLF + st), u & 1, abort_flag, a.status);
+      w_ok = w_ok && mbar_wait(BAR(kBSF), it & 1, abort_flag, a.status);
+      if (!__all_sync(0xFFFFFFFFu, w_ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float* ls = lbuf + st * 2 * BM;
+      // partial-tile mask data for this key row
+      int64_t lim_lo = 0;  // queries i >= lim_lo are allowed by causality (i >= j)
+      bool key_ok = j < a.Sk;
+      uint8_t m64[2] = {1, 1};
+      if (partial) {
+        if (a.causal) lim_lo = j;
+        if (a.mode == SA_MODE_BLOCK && a.bs == 64 && key_ok) {
+          // the two 64-query blocks of this 128-row query tile are m0/64 (the half)
+          const uint8_t* mcol = a.mask + bg * a.Mb * static_cast<int64_t>(a.Nb) + j / 64;
+          const int64_t mb = m0 / 64;
+          m64[0] = mb < a.Mb ? __ldg(mcol + mb * a.Nb) : 0;
+        }
+      }
+#pragma unroll
+      for (int cc = 0; cc < BM / 32; ++cc) {
+        uint32_t s_u[32], p_u[32];
+        tmem_ld32(tl + C::kColS + cc * 32, s_u);
+        tmem_ld32(tl + C::kColDP + cc * 32, p_u);
+        tmem_wait_ld();
+        uint32_t wbits = 0xFFFFFFFFu;
+        if (partial && a.mode == SA_MODE_INDEX) {
+          // bit j of row i for the 32 queries of this chunk (one word per query)
+          wbits = 0u;
+          const int64_t wcol = j >> 5;
+          for (int e = 0; e < 32; ++e) {
+            const int64_t i = m0 + cc * 32 + e;
+            uint32_t wv = 0u;
+            if (i < a.Sq && key_ok) wv = __ldg(a.bitmap + (bg * a.Sq + i) * a.W + wcol);
+            wbits |= ((wv >> (j & 31)) & 1u) << e;
+          }
+        }
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float pv[2], dv2[2];
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const int q = cc * 32 + 2 * e + t;
+            const int64_t i = m0 + q;
+            bool allowed = true;
+            if (partial) {
+              allowed = key_ok && i >= lim_lo && m64[0] != 0 && ((wbits >> (2 * e + t)) & 1u);
+            }
+            const float s = __uint_as_float(s_u[2 * e + t]);
+            const float p = allowed ? ex2(fmaf(s, a.scale_log2, -ls[q])) : 0.f;
+            pv[t] = p;
+            dv2[t] = p * (__uint_as_float(p_u[2 * e + t]) - ls[BM + q]);
+          }
+          pk[e] = pack_bf16x2(pv[0], pv[1]);
+          dk[e] = pack_bf16x2(dv2[0], dv2[1]);
+        }
+        tmem_st16(tl + C::kColS + cc * 16, pk);
+        tmem_st16(tl + C::kColDP + cc * 16, dk);
+        // dS^T row into shared memory, 128-byte swizzled: 16-byte chunk c of row r
+        // lives at chunk c ^ (r % 8)
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const int c = cc * 4 + c4;
+          *reinterpret_cast<uint4*>(dsrow + ((c ^ (r & 7)) << 4)) =
+              make_uint4(dk[4 * c4], dk[4 * c4 + 1], dk[4 * c4 + 2], dk[4 * c4 + 3]);
+        }
+      }
+      tmem_wait_st();
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(BAR(kBPF));
+      // drain dQ^T of this step: lane = head-dim row, 64 query columns
+      w_ok = mbar_wait(BAR(kBDQF), it & 1, abort_flag, a.status);
+      if (!__all_sync(0xFFFFFFFFu, w_ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t q_u[BM];
+      tmem_ld32(tl + C::kColDQ, q_u);
+      tmem_ld32(tl + C::kColDQ + 32, q_u + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(BAR(kBDQE));
+      if (dq_mine) {
+        float* dst = a.dq_acc + ((static_cast<int64_t>(b) * a.Sq + m0) * a.HQ + h) *
+                                    static_cast<int64_t>(dqk_real) + dq_d;
+        const int64_t stride = static_cast<int64_t>(a.HQ) * dqk_real;
+        const int nq = static_cast<int>(min64(BM, a.Sq - m0));
+#pragma unroll
+        for (int q = 0; q < BM; ++q)
+          if (q < nq) atomicAdd(dst + q * stride, __uint_as_float(q_u[q]));
+      }
+    }
+    // ----------------------------------------------------------- dK / dV epilogue
+    bool have = n_iter > 0 && ok;
+    if (have) {
+      const bool w_ok = mbar_wait(BAR(kBFin), 0, abort_flag, a.status);
+      have = __all_sync(0xFFFFFFFFu, w_ok);
+      tc_fence_after();
+    }
+    const bool row_ok = j < a.Sk;
+    __nv_bfloat16* dkrow = reinterpret_cast<__nv_bfloat16*>(a.dk) +
+                           ((static_cast<int64_t>(b) * a.Sk + j) * a.HK + g) * dqk_real;
+    __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(a.dv) +
+                           ((static_cast<int64_t>(b) * a.Sk + j) * a.HK + g) * dv_real;
+    for (int pass = 0; pass < 2; ++pass) {
+      const int n = pass == 0 ? kcn : vcn;
+      const int d0 = pass == 0 ? kc0 : vc0;
+      const int dreal = pass == 0 ? dqk_real : dv_real;
+      const uint32_t col = pass == 0 ? C::kColDK : C::kColDV;
+      const float sc = pass == 0 ? a.scale : 1.f;
+      __nv_bfloat16* out = pass == 0 ? dkrow : dvrow;
+      for (int c = 0; c < n; c += 32) {
+        uint32_t v[32];
+        if (have) {
+          tmem_ld32(tl + col + c, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        }
+        if (row_ok && d0 + c < dreal) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
+          uint4* dst = reinterpret_cast<uint4*>(out + d0 + c);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
+    }
+  }
+
+  if (warp == 1 && lane == 0 && *abort_flag) {
+    umma_commit(BAR(kBDrainB));
+    mbar_wait_limited(BAR(kBDrainB), 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int DQK, int DV, int NSPLIT>
+static int launch_bwd_main(const AttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mk,
+                           const CUtensorMap& mv, const CUtensorMap& mdo, cudaStream_t st) {
+  using C = BwdCfg<DQK, DV, NSPLIT>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(sparse_bwd_kernel<DQK, DV, NSPLIT>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) != cudaSuccess)
+      return SA_ERR_CUDA;
+    attr_set = true;
+  }
+  dim3 grid(a.Tn * NSPLIT, a.HK, a.B);
+  record_event(3, st);
+  sparse_bwd_kernel<DQK, DV, NSPLIT><<<grid, C::kThreads, C::kSmem, st>>>(mq, mk, mv, mdo, a);
+  record_event(4, st);
+  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+int launch_bwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
+  const int64_t rows = static_cast<int64_t>(a.B) * a.Sq * a.HQ;
+  {
+    const int warps = 8;
+    const int64_t blocks = (rows + warps - 1) / warps;
+    record_event(2, st);
+    bwd_pre_kernel<<<static_cast<unsigned>(blocks), warps * 32, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.delta,
+        a.dq_acc, rows, a.Sq, a.HQ, a.Dv, a.Dqk);
+    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  }
+  int rc;
+  if (a.Dqk == 64 && a.Dv == 64)
+    rc = launch_bwd_main<128, 128, 1>(a, m.q, m.k, m.v, m.dout, st);
+  else if (a.Dqk == 128 && a.Dv == 128)
+    rc = launch_bwd_main<128, 128, 1>(a, m.q, m.k, m.v, m.dout, st);
+  else if (a.Dqk == 192 && a.Dv == 128)
+    rc = launch_bwd_main<192, 128, 2>(a, m.q, m.k, m.v, m.dout, st);
+  else if (a.Dqk == 256 && a.Dv == 256)
+    rc = launch_bwd_main<256, 256, 2>(a, m.q, m.k, m.v, m.dout, st);
+  else
+    return SA_ERR_UNSUPPORTED;
+  if (rc) return rc;
+  const int64_t n4 = rows * a.Dqk / 4;
+  bwd_post_kernel<<<static_cast<unsigned>(min64((n4 + 255) / 256, 148 * 16)), 256, 0, st>>>(
+      a.dq_acc, static_cast<__nv_bfloat16*>(a.dq), n4, a.scale);
+  record_event(5, st);
+  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
 }  // namespace sa

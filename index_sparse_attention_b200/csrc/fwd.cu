@@ -347,7 +347,9 @@ static int launch_fwd_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st)
     attr_set = true;
   }
   dim3 grid(a.Tm, a.HQ, a.B);
+  record_event(0, st);
   sparse_fwd_kernel<DQK, DV><<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.v, a);
+  record_event(1, st);
   return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 

@@ -35,8 +35,15 @@ struct AttnArgs {
 };
 
 struct TensorMaps {
-  CUtensorMap q, k, v, o, dout;
+  CUtensorMap q, k, v, dout;
 };
+
+// Caller-owned events recorded around the launches (see sparse_attn_set_timing_events);
+// nullptr when instrumentation is off.
+extern cudaEvent_t* g_timing_events;
+inline void record_event(int k, cudaStream_t st) {
+  if (g_timing_events) cudaEventRecord(g_timing_events[k], st);
+}
 
 int launch_fwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st);
 int launch_bwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st);
