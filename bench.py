@@ -193,12 +193,19 @@ class OracleSampler:
         return flop, time.perf_counter() - t0, n
 
 
+def get_workload(args):
+    w = I.WORKLOADS[args.workload]
+    if args.seq:
+        w = I.scaled(w, Sq=args.seq, Sk=args.seq, name=f"{w.name}@S{args.seq}")
+    return w
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:  # under torchrun only rank 0 runs the CPU reference
         return
     os.environ.setdefault("OMP_NUM_THREADS", str(len(os.sched_getaffinity(0))))
-    w = I.WORKLOADS[args.workload]
+    w = get_workload(args)
     inp = I.make_inputs(w)
     s = OracleSampler(w, inp)
     per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
@@ -262,7 +269,7 @@ def run_gpu(args):
     from index_sparse_attention_b200 import _lib
 
     L = _lib.load()
-    w = I.WORKLOADS[args.workload]
+    w = get_workload(args)
     inp = I.make_inputs(w)
     dev = torch.device("cuda", local)
 
@@ -428,6 +435,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seq", type=int, default=0,
+                    help="override Sq = Sk (smaller profiling captures of the same kernels)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":

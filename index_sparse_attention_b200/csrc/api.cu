@@ -46,6 +46,22 @@ bool make_map(CUtensorMap* m, const void* base, int D, int64_t S, int H, int B, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D map over the fp32 dQ accumulator [B][Sq][HQ][D] with 64 x 32 (D x S) boxes, no
+// swizzle: the target of the backward's bulk reduce-adds.
+bool make_map_f32(CUtensorMap* m, const void* base, int D, int64_t S, int H, int B) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S),
+                        static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(H) * D * 4, static_cast<cuuint64_t>(D) * 4,
+                           static_cast<cuuint64_t>(S) * H * D * 4};
+  cuuint32_t box[4] = {64, 32, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool dims_supported(int dqk, int dv) {
@@ -184,5 +200,6 @@ extern "C" int sparse_attn_bwd(const sparse_attn_params* p, void* workspace,
   TensorMaps m;
   rc = fill_maps(p, &m, true);
   if (rc) return rc;
+  if (!make_map_f32(&m.dq_acc, a.dq_acc, p->Dqk, p->Sq, p->HQ, p->B)) return SA_ERR_CUDA;
   return launch_bwd(a, m, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -98,38 +98,44 @@ struct BwdCfg {
   static constexpr int kQBytes = kBM * DQK * 2;
   static constexpr int kOBytes = kBM * DV * 2;
   static constexpr int kStages = (DQK + DV >= 512) ? 1 : 2;
+  static constexpr int kDSBytes = 128 * kBM * 2;     // dS^T [128 keys][64 q] bf16 (16 KB)
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kKOff + kKBytes;
   static constexpr int kQOff = kVOff + kVBytes;                    // per stage: Q then dO
   static constexpr int kStageBytes = kQBytes + kOBytes;
-  static constexpr int kDSOff = kQOff + kStages * kStageBytes;     // dS^T [128 keys][64 q]
-  static constexpr int kLOff = kDSOff + 128 * kBM * 2;             // per stage: lse2[64], delta[64]
-  static constexpr int kBarOff = kLOff + kStages * 2 * kBM * 4;
+  static constexpr int kDSOff = kQOff + kStages * kStageBytes;     // two dS^T buffers
+  static constexpr int kLOff = kDSOff + 2 * kDSBytes;              // per stage: lse2[64], delta[64]
+  static constexpr int kBMOff = kLOff + kStages * 2 * kBM * 4;     // per stage: bitmap words [64][4]
+  static constexpr int kBarOff = kBMOff + kStages * kBM * 4 * 4;
   static constexpr int kSmem = kBarOff + 256 + 1024;
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 320;
   // head-dim chunks of this CTA: dK [kc0, kc0 + kcn), dV [vc0, vc0 + vcn)
   static constexpr int kDKMax = NSPLIT == 1 ? DQK : (DQK == 192 ? 128 : DQK / 2);
   static constexpr int kDVMax = DV / NSPLIT;
-  // TMEM columns
-  static constexpr uint32_t kColS = 0;
-  static constexpr uint32_t kColDP = 64;
-  static constexpr uint32_t kColDQ = 128;
-  static constexpr uint32_t kColDK = 192;
+  // TMEM columns: S^T / P^T x2, dP^T / dS^T / dQ^T x2, dK, dV
+  static constexpr uint32_t kColS = 0;     // + 64 * buffer
+  static constexpr uint32_t kColDP = 128;  // + 64 * buffer
+  static constexpr uint32_t kColDK = 256;
   static constexpr uint32_t kColDV = kColDK + kDKMax;
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kColDV + kDVMax <= kTmemCols, "tensor memory budget");
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
 
-enum : int { kBKV = 0, kBQF = 1, kBQE = 3, kBLF = 5, kBSF = 7, kBPF = 8, kBDQF = 9, kBDQE = 10,
-             kBFin = 11, kBDrainB = 12, kNumBarsB = 13 };
+enum : int {
+  kBKV = 0, kBQF = 1, kBQE = 3, kBLF = 5, kBSF = 7, kBPF = 9, kBDQF = 11, kBDQE = 13, kBDSE = 15,
+  kBFin = 17, kBDrainB = 18, kNumBarsB = 19
+};
 
+// Warp roles: 0 producer, 1 MMA, 2-5 elementwise (one key row per thread), 6-9 dQ drain
+// (one head-dim row of the dQ^T window per thread).
 template <int DQK, int DV, int NSPLIT>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     sparse_bwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v,
-                      const __grid_constant__ CUtensorMap tm_do, const AttnArgs a) {
+                      const __grid_constant__ CUtensorMap tm_do,
+                      const __grid_constant__ CUtensorMap tm_dq, const AttnArgs a) {
   using C = BwdCfg<DQK, DV, NSPLIT>;
   constexpr int BM = C::kBM;
   extern __shared__ uint8_t smem_raw[];
@@ -174,11 +180,12 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(BAR(kBQF + s), 1);
       mbar_init(BAR(kBQE + s), 1);
       mbar_init(BAR(kBLF + s), 32);
+      mbar_init(BAR(kBSF + s), 1);
+      mbar_init(BAR(kBPF + s), 128);
+      mbar_init(BAR(kBDQF + s), 1);
+      mbar_init(BAR(kBDQE + s), 128);
+      mbar_init(BAR(kBDSE + s), 128);
     }
-    mbar_init(BAR(kBSF), 1);
-    mbar_init(BAR(kBPF), 128);
-    mbar_init(BAR(kBDQF), 1);
-    mbar_init(BAR(kBDQE), 128);
     mbar_init(BAR(kBFin), 1);
     mbar_init(BAR(kBDrainB), 1);
     *abort_flag = 0;
@@ -212,6 +219,7 @@ __global__ void __launch_bounds__(192, 1)
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
         prefetch_tensormap(&tm_do);
+        prefetch_tensormap(&tm_dq);
         mbar_arrive_expect_tx(BAR(kBKV), C::kKBytes + C::kVBytes);
         for (int c = 0; c < DQK / 64; ++c)
           tma_load_4d(sbase + C::kKOff + c * C::kKPanel, &tm_k, BAR(kBKV), c * 64, nt * 128, g, b);
@@ -219,6 +227,7 @@ __global__ void __launch_bounds__(192, 1)
           tma_load_4d(sbase + C::kVOff + c * C::kKPanel, &tm_v, BAR(kBKV), c * 64, nt * 128, g, b);
       }
       float* lbuf = reinterpret_cast<float*>(smem + C::kLOff);
+      uint32_t* bmbuf = reinterpret_cast<uint32_t*>(smem + C::kBMOff);
       for (int it = 0; it < n_iter; ++it) {
         int h, m0;
         bool partial;
@@ -249,6 +258,15 @@ __global__ void __launch_bounds__(192, 1)
           ls[q] = l2;
           ls[BM + q] = dl;
         }
+        if (partial && a.mode == SA_MODE_INDEX) {
+          // presence words of this key tile for the 64 queries: [q][4]
+          uint32_t* bw = bmbuf + st * BM * 4;
+          for (int e = lane; e < BM * 4; e += 32) {
+            const int q = e >> 2, w = nt * 4 + (e & 3);
+            const int64_t i = m0 + q;
+            bw[e] = (i < a.Sq && w < a.W) ? __ldg(a.bitmap + (bg * a.Sq + i) * a.W + w) : 0u;
+          }
+        }
         mbar_arrive(BAR(kBLF + st));
       }
       if (lane == 0 && *abort_flag) {
@@ -265,11 +283,14 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t idesc_dv = idesc_bf16(128, vcn, 0, 1);        // dV += P^T dO
       const uint32_t idesc_dk = idesc_bf16(128, kcn, 0, 1);        // dK += dS^T Q
       const uint32_t kbase = sbase + C::kKOff, vbase = sbase + C::kVOff;
-      const uint32_t dsb = sbase + C::kDSOff;
       bool ok = mbar_wait(BAR(kBKV), 0, abort_flag, a.status);
-      for (int it = 0; ok && it < n_iter; ++it) {
-        const int st = it % C::kStages, u = it / C::kStages;
-        if (!mbar_wait(BAR(kBQF + st), u & 1, abort_flag, a.status)) break;
+      // S^T(j) and dP^T(j) into TMEM buffer j & 1
+      auto issue_sdp = [&](int j) -> bool {
+        const int st = j % C::kStages, u = j / C::kStages, bj = j & 1;
+        if (!mbar_wait(BAR(kBQF + st), u & 1, abort_flag, a.status)) return false;
+        // the dQ^T of step j-2 lives in this buffer until it has been drained
+        if (j >= 2 && !mbar_wait(BAR(kBDQE + bj), ((j - 2) >> 1) & 1, abort_flag, a.status))
+          return false;
         tc_fence_after();
         const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
         const uint32_t os = qs + C::kQBytes;
@@ -277,100 +298,106 @@ __global__ void __launch_bounds__(192, 1)
         for (int kk = 0; kk < DQK / 16; ++kk) {
           const uint32_t ka = (kk >> 2) * C::kKPanel + (kk & 3) * 32;
           const uint32_t qb = (kk >> 2) * C::kQPanel + (kk & 3) * 32;
-          umma_ss(tmem + C::kColS, sw128_desc(kbase + ka, 16, 1024), sw128_desc(qs + qb, 16, 1024),
-                  idesc_s, kk > 0 ? 1u : 0u);
+          umma_ss(tmem + C::kColS + 64 * bj, sw128_desc(kbase + ka, 16, 1024),
+                  sw128_desc(qs + qb, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < DV / 16; ++kk) {
           const uint32_t va = (kk >> 2) * C::kKPanel + (kk & 3) * 32;
           const uint32_t ob = (kk >> 2) * C::kQPanel + (kk & 3) * 32;
-          umma_ss(tmem + C::kColDP, sw128_desc(vbase + va, 16, 1024), sw128_desc(os + ob, 16, 1024),
-                  idesc_s, kk > 0 ? 1u : 0u);
+          umma_ss(tmem + C::kColDP + 64 * bj, sw128_desc(vbase + va, 16, 1024),
+                  sw128_desc(os + ob, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(BAR(kBSF));
-        if (!mbar_wait(BAR(kBPF), it & 1, abort_flag, a.status)) break;
+        umma_commit(BAR(kBSF + bj));
+        return true;
+      };
+      if (ok) ok = issue_sdp(0);
+      for (int it = 0; ok && it < n_iter; ++it) {
+        const int st = it % C::kStages, bi = it & 1;
+        // with two Q/dO stages the next S^T / dP^T overlap this step's elementwise work
+        if (C::kStages >= 2 && it + 1 < n_iter && !issue_sdp(it + 1)) break;
+        if (!mbar_wait(BAR(kBPF + bi), (it >> 1) & 1, abort_flag, a.status)) break;
         tc_fence_after();
+        const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
+        const uint32_t os = qs + C::kQBytes;
         // dV += P^T dO  and  dK += dS^T Q (K = 64 queries: four k-steps of 16)
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
-          umma_ts(tmem + C::kColDV, tmem + C::kColS + kk * 8,
+          umma_ts(tmem + C::kColDV, tmem + C::kColS + 64 * bi + kk * 8,
                   sw128_desc(os + (vc0 / 64) * C::kQPanel + kk * 2048, C::kQPanel, 1024), idesc_dv,
                   (it > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
-          umma_ts(tmem + C::kColDK, tmem + C::kColDP + kk * 8,
+          umma_ts(tmem + C::kColDK, tmem + C::kColDP + 64 * bi + kk * 8,
                   sw128_desc(qs + (kc0 / 64) * C::kQPanel + kk * 2048, C::kQPanel, 1024), idesc_dk,
                   (it > 0 || kk > 0) ? 1u : 0u);
         umma_commit(BAR(kBQE + st));
-        // dQ^T = K^T dS^T over the 128 keys, once the previous dQ^T has been drained
-        if (!mbar_wait(BAR(kBDQE), (it & 1) ^ 1, abort_flag, a.status)) break;
-        tc_fence_after();
+        // dQ^T = K^T dS^T over the 128 keys, into the dP^T buffer dK has just consumed
+        const uint32_t dsb = sbase + C::kDSOff + bi * C::kDSBytes;
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ss(tmem + C::kColDQ,
+          umma_ss(tmem + C::kColDP + 64 * bi,
                   sw128_desc(kbase + (qw0 / 64) * C::kKPanel + kk * 2048, C::kKPanel, 1024),
                   sw128_desc(dsb + kk * 2048, C::kKPanel, 1024), idesc_dq, kk > 0 ? 1u : 0u);
-        umma_commit(BAR(kBDQF));
+        umma_commit(BAR(kBDQF + bi));
+        if (C::kStages == 1 && it + 1 < n_iter && !issue_sdp(it + 1)) break;
       }
       umma_commit(BAR(kBFin));
     }
-  } else {
-    // ------------------------------------------------------- elementwise + dQ drain
+  } else if (warp < 6) {
+    // ------------------------------------------------------------------ elementwise
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;           // key row of the tile = TMEM lane
     const int64_t j = static_cast<int64_t>(nt) * 128 + r;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float* lbuf = reinterpret_cast<const float*>(smem + C::kLOff);
-    uint8_t* dsrow = smem + C::kDSOff + r * 128;
-    // head-dim rows of the dQ^T window drained by this thread
-    const int dq_d = qw0 + r;
-    const bool dq_mine = (NSPLIT == 1 || DQK != 192) ? (r < 128 && dq_d < dqk_real)
-                                                      : (dq_d >= kc0 && dq_d < kc0 + kcn);
+    const uint32_t* bmbuf = reinterpret_cast<const uint32_t*>(smem + C::kBMOff);
+    const bool key_ok = j < a.Sk;
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
       int h, m0;
       bool partial;
       decode(it, h, m0, partial);
-      const int st = it % C::kStages, u = it / C::kStages;
+      const int st = it % C::kStages, u = it / C::kStages, bi = it & 1;
       bool w_ok = mbar_wait(BAR(kBLF + st), u & 1, abort_flag, a.status);
-      w_ok = w_ok && mbar_wait(BAR(kBSF), it & 1, abort_flag, a.status);
+      w_ok = w_ok && mbar_wait(BAR(kBSF + bi), (it >> 1) & 1, abort_flag, a.status);
+      // the dS^T buffer was the dQ staging area of step it-2
+      if (it >= 2) w_ok = w_ok && mbar_wait(BAR(kBDSE + bi), ((it - 2) >> 1) & 1, abort_flag, a.status);
       if (!__all_sync(0xFFFFFFFFu, w_ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const float* ls = lbuf + st * 2 * BM;
-      // partial-tile mask data for this key row
-      int64_t lim_lo = 0;  // queries i >= lim_lo are allowed by causality (i >= j)
-      bool key_ok = j < a.Sk;
-      uint8_t m64[2] = {1, 1};
+      uint8_t* dsrow = smem + C::kDSOff + bi * C::kDSBytes + r * 128;
+      // allowed-query mask of this key row over the 64 queries (partial tiles only)
+      uint64_t qmask = ~0ull;
       if (partial) {
-        if (a.causal) lim_lo = j;
+        qmask = key_ok ? ~0ull : 0ull;
+        if (a.causal) {  // i >= j
+          const int64_t lo = j - m0;
+          qmask &= lo <= 0 ? ~0ull : (lo >= 64 ? 0ull : (~0ull << lo));
+        }
         if (a.mode == SA_MODE_BLOCK && a.bs == 64 && key_ok) {
-          // the two 64-query blocks of this 128-row query tile are m0/64 (the half)
-          const uint8_t* mcol = a.mask + bg * a.Mb * static_cast<int64_t>(a.Nb) + j / 64;
           const int64_t mb = m0 / 64;
-          m64[0] = mb < a.Mb ? __ldg(mcol + mb * a.Nb) : 0;
+          const bool m = mb < a.Mb &&
+                         __ldg(a.mask + (bg * a.Mb + mb) * static_cast<int64_t>(a.Nb) + j / 64) != 0;
+          if (!m) qmask = 0ull;
+        } else if (a.mode == SA_MODE_INDEX) {
+          const uint32_t* bw = bmbuf + st * BM * 4 + (r >> 5);
+          uint64_t bits = 0ull;
+#pragma unroll 8
+          for (int q = 0; q < BM; ++q) bits |= static_cast<uint64_t>((bw[q * 4] >> lane) & 1u) << q;
+          qmask &= bits;
         }
       }
 #pragma unroll
       for (int cc = 0; cc < BM / 32; ++cc) {
         uint32_t s_u[32], p_u[32];
-        tmem_ld32(tl + C::kColS + cc * 32, s_u);
-        tmem_ld32(tl + C::kColDP + cc * 32, p_u);
+        tmem_ld32(tl + C::kColS + 64 * bi + cc * 32, s_u);
+        tmem_ld32(tl + C::kColDP + 64 * bi + cc * 32, p_u);
         tmem_wait_ld();
-        uint32_t wbits = 0xFFFFFFFFu;
-        if (partial && a.mode == SA_MODE_INDEX) {
-          // bit j of row i for the 32 queries of this chunk (one word per query)
-          wbits = 0u;
-          const int64_t wcol = j >> 5;
-          for (int e = 0; e < 32; ++e) {
-            const int64_t i = m0 + cc * 32 + e;
-            uint32_t wv = 0u;
-            if (i < a.Sq && key_ok) wv = __ldg(a.bitmap + (bg * a.Sq + i) * a.W + wcol);
-            wbits |= ((wv >> (j & 31)) & 1u) << e;
-          }
-        }
+        const uint32_t cm = static_cast<uint32_t>(qmask >> (32 * cc));
         uint32_t pk[16], dk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -378,21 +405,16 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
             const int q = cc * 32 + 2 * e + t;
-            const int64_t i = m0 + q;
-            bool allowed = true;
-            if (partial) {
-              allowed = key_ok && i >= lim_lo && m64[0] != 0 && ((wbits >> (2 * e + t)) & 1u);
-            }
             const float s = __uint_as_float(s_u[2 * e + t]);
-            const float p = allowed ? ex2(fmaf(s, a.scale_log2, -ls[q])) : 0.f;
+            const float p = ((cm >> (2 * e + t)) & 1u) ? ex2(fmaf(s, a.scale_log2, -ls[q])) : 0.f;
             pv[t] = p;
             dv2[t] = p * (__uint_as_float(p_u[2 * e + t]) - ls[BM + q]);
           }
           pk[e] = pack_bf16x2(pv[0], pv[1]);
           dk[e] = pack_bf16x2(dv2[0], dv2[1]);
         }
-        tmem_st16(tl + C::kColS + cc * 16, pk);
-        tmem_st16(tl + C::kColDP + cc * 16, dk);
+        tmem_st16(tl + C::kColS + 64 * bi + cc * 16, pk);
+        tmem_st16(tl + C::kColDP + 64 * bi + cc * 16, dk);
         // dS^T row into shared memory, 128-byte swizzled: 16-byte chunk c of row r
         // lives at chunk c ^ (r % 8)
 #pragma unroll
@@ -403,31 +425,9 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       tmem_wait_st();
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(BAR(kBPF));
-      // drain dQ^T of this step: lane = head-dim row, 64 query columns
-      w_ok = mbar_wait(BAR(kBDQF), it & 1, abort_flag, a.status);
-      if (!__all_sync(0xFFFFFFFFu, w_ok)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t q_u[BM];
-      tmem_ld32(tl + C::kColDQ, q_u);
-      tmem_ld32(tl + C::kColDQ + 32, q_u + 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(BAR(kBDQE));
-      if (dq_mine) {
-        float* dst = a.dq_acc + ((static_cast<int64_t>(b) * a.Sq + m0) * a.HQ + h) *
-                                    static_cast<int64_t>(dqk_real) + dq_d;
-        const int64_t stride = static_cast<int64_t>(a.HQ) * dqk_real;
-        const int nq = static_cast<int>(min64(BM, a.Sq - m0));
-#pragma unroll
-        for (int q = 0; q < BM; ++q)
-          if (q < nq) atomicAdd(dst + q * stride, __uint_as_float(q_u[q]));
-      }
+      mbar_arrive(BAR(kBPF + bi));
     }
     // ----------------------------------------------------------- dK / dV epilogue
     bool have = n_iter > 0 && ok;
@@ -436,7 +436,6 @@ __global__ void __launch_bounds__(192, 1)
       have = __all_sync(0xFFFFFFFFu, w_ok);
       tc_fence_after();
     }
-    const bool row_ok = j < a.Sk;
     __nv_bfloat16* dkrow = reinterpret_cast<__nv_bfloat16*>(a.dk) +
                            ((static_cast<int64_t>(b) * a.Sk + j) * a.HK + g) * dqk_real;
     __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(a.dv) +
@@ -457,7 +456,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] = 0u;
         }
-        if (row_ok && d0 + c < dreal) {
+        if (key_ok && d0 + c < dreal) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
@@ -469,6 +468,63 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
     }
+  } else {
+    // ------------------------------------------------------------------ dQ drain
+    // thread = head-dim row r of the 128-wide dQ^T window; the 64 query columns are
+    // staged as fp32 in the step's (now free) dS^T buffer, 32 queries at a time, as
+    // [64-column panel][32 q][64 d] tiles that bulk reduce-adds push into dQ_acc.
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int dtid = threadIdx.x - 192;  // 0..127 within the drain warpgroup
+    const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const int p = r >> 6;  // panel of this row within the window
+    // a panel is reduced when it lies in this CTA's dQ range and inside Dqk
+    auto panel_owned = [&](int pp) {
+      const int d0 = qw0 + 64 * pp;
+      return d0 >= kc0 && d0 + 64 <= kc0 + kcn && d0 < dqk_real;
+    };
+    const bool own0 = panel_owned(0), own1 = panel_owned(1);
+    bool ok = true;
+    for (int it = 0; it < n_iter && ok; ++it) {
+      int h, m0;
+      bool partial;
+      decode(it, h, m0, partial);
+      const int bi = it & 1;
+      const bool w_ok = mbar_wait(BAR(kBDQF + bi), (it >> 1) & 1, abort_flag, a.status);
+      if (!__all_sync(0xFFFFFFFFu, w_ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t q_u[BM];
+      tmem_ld32(tl + C::kColDP + 64 * bi, q_u);
+      tmem_ld32(tl + C::kColDP + 64 * bi + 32, q_u + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(BAR(kBDQE + bi));
+      float* stage = reinterpret_cast<float*>(smem + C::kDSOff + bi * C::kDSBytes);
+      const uint32_t stage_s = sbase + C::kDSOff + bi * C::kDSBytes;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        if (half == 1) {
+          if (dtid == 0) bulk_wait_group_read0();
+          named_bar_sync(1, 128);
+        }
+#pragma unroll
+        for (int q = 0; q < 32; ++q) stage[(p * 32 + q) * 64 + (r & 63)] = __uint_as_float(q_u[32 * half + q]);
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (dtid == 0) {
+          if (own0) tma_reduce_add_4d(&tm_dq, stage_s, qw0, m0 + 32 * half, h, b);
+          if (own1) tma_reduce_add_4d(&tm_dq, stage_s + 32 * 64 * 4, qw0 + 64, m0 + 32 * half, h, b);
+          bulk_commit_group();
+        }
+      }
+      if (dtid == 0) bulk_wait_group_read0();
+      named_bar_sync(1, 128);
+      mbar_arrive(BAR(kBDSE + bi));
+    }
+    if (dtid == 0) bulk_wait_group0();  // every reduce has landed before the CTA ends
   }
 
   if (warp == 1 && lane == 0 && *abort_flag) {
@@ -484,8 +540,7 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 template <int DQK, int DV, int NSPLIT>
-static int launch_bwd_main(const AttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mk,
-                           const CUtensorMap& mv, const CUtensorMap& mdo, cudaStream_t st) {
+static int launch_bwd_main(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
   using C = BwdCfg<DQK, DV, NSPLIT>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -496,7 +551,8 @@ static int launch_bwd_main(const AttnArgs& a, const CUtensorMap& mq, const CUten
   }
   dim3 grid(a.Tn * NSPLIT, a.HK, a.B);
   record_event(3, st);
-  sparse_bwd_kernel<DQK, DV, NSPLIT><<<grid, C::kThreads, C::kSmem, st>>>(mq, mk, mv, mdo, a);
+  sparse_bwd_kernel<DQK, DV, NSPLIT><<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.v, m.dout,
+                                                                           m.dq_acc, a);
   record_event(4, st);
   return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
@@ -514,13 +570,13 @@ int launch_bwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
   }
   int rc;
   if (a.Dqk == 64 && a.Dv == 64)
-    rc = launch_bwd_main<128, 128, 1>(a, m.q, m.k, m.v, m.dout, st);
+    rc = launch_bwd_main<128, 128, 1>(a, m, st);
   else if (a.Dqk == 128 && a.Dv == 128)
-    rc = launch_bwd_main<128, 128, 1>(a, m.q, m.k, m.v, m.dout, st);
+    rc = launch_bwd_main<128, 128, 1>(a, m, st);
   else if (a.Dqk == 192 && a.Dv == 128)
-    rc = launch_bwd_main<192, 128, 2>(a, m.q, m.k, m.v, m.dout, st);
+    rc = launch_bwd_main<192, 128, 2>(a, m, st);
   else if (a.Dqk == 256 && a.Dv == 256)
-    rc = launch_bwd_main<256, 256, 2>(a, m.q, m.k, m.v, m.dout, st);
+    rc = launch_bwd_main<256, 256, 2>(a, m, st);
   else
     return SA_ERR_UNSUPPORTED;
   if (rc) return rc;

@@ -35,7 +35,7 @@ struct AttnArgs {
 };
 
 struct TensorMaps {
-  CUtensorMap q, k, v, dout;
+  CUtensorMap q, k, v, dout, dq_acc;
 };
 
 // Caller-owned events recorded around the launches (see sparse_attn_set_timing_events);
