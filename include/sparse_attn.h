@@ -65,6 +65,7 @@ typedef struct CUstream_st *sa_stream_t; /* the same handle as cudaStream_t */
 #define SA_ERR_ALIGN (-4)       /* a base pointer is not 16-byte aligned */
 #define SA_ERR_CUDA (-5)        /* a CUDA call or kernel launch failed */
 #define SA_ERR_WORKSPACE (-7)   /* workspace missing or too small */
+#define SA_ERR_SCRATCH_LIMIT (-8) /* sparse_attn_bwd_noalloc: problem exceeds its fixed scratch */
 
 #define SA_MODE_DENSE 0
 #define SA_MODE_BLOCK 1
@@ -158,6 +159,30 @@ size_t sparse_attn_bwd_workspace_size(const sparse_attn_params *p);
  */
 int sparse_attn_bwd(const sparse_attn_params *p, void *workspace, size_t workspace_bytes,
                     sa_stream_t stream);
+
+/* Size of the fixed device scratch array used by sparse_attn_bwd_noalloc: 16 MiB. */
+#define SA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/*
+ * sparse_attn_bwd_noalloc -- the backward for callers that cannot allocate device
+ * memory.  The pages have no counterpart to this entry point.
+ * Some callers cannot call cudaMalloc or pass a workspace: code inside a host framework
+ * that owns every device allocation and hands over only inputs and outputs (a plugin
+ * or serving backend), or latency-critical loops where cudaMalloc's implicit device
+ * synchronisation is not acceptable.  This call runs the same kernels as
+ * sparse_attn_bwd (same arguments, same outputs) but takes the backward's scratch
+ * (fp32 Delta and dQ accumulator) from a file-scope device array of
+ * SA_NOALLOC_SCRATCH_BYTES bytes that every GPU loading the library holds until exit.
+ *  - Returns SA_ERR_SCRATCH_LIMIT, before enqueuing anything, when
+ *    sparse_attn_bwd_workspace_size(p) exceeds SA_NOALLOC_SCRATCH_BYTES.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make it before any stream
+ *    capture.
+ *  - All calls on a device share the array and overwrite it; calls whose GPU work
+ *    overlaps (unordered streams, several host threads) race: serialise them.
+ *  - Allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ */
+int sparse_attn_bwd_noalloc(const sparse_attn_params *p, sa_stream_t stream);
 
 /*
  * sparse_attn_set_timing_events -- optional instrumentation (no counterpart on the

@@ -15,6 +15,7 @@ from ._lib import SA_MODE_BLOCK, SA_MODE_DENSE, SA_MODE_INDEX, SA_TILE, SparseAt
 
 __all__ = ["BlockSparse", "block_mask_to_block_sparse", "index_to_block_sparse",
            "sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_bwd_workspace_size",
+           "sparse_attn_bwd_noalloc",
            "SparseAttnError", "SA_TILE"]
 
 
@@ -149,4 +150,23 @@ def sparse_attn_bwd(q, k, v, o, lse, dout, sparse, softmax_scale=None, dq=None, 
     _lib.check("sparse_attn_bwd",
                L.sparse_attn_bwd(ctypes.byref(p), _ptr(workspace), workspace.numel(),
                                  _stream(q.device)))
+    return dq, dk, dv
+
+
+def sparse_attn_bwd_noalloc(q, k, v, o, lse, dout, sparse, softmax_scale=None, dq=None, dk=None,
+                            dv=None, dev_status=None):
+    """dQ, dK, dV like sparse_attn_bwd, with the scratch taken from the library's fixed
+    device array instead of a workspace (for callers that cannot allocate device memory;
+    see include/sparse_attn.h).  Calls on one device share that array: do not overlap
+    them on the GPU."""
+    L = _lib.load()
+    Dqk = q.shape[3]
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(Dqk)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    p = _params(q, k, v, o, lse, sparse, softmax_scale, dout, dq, dk, dv, dev_status)
+    _lib.check("sparse_attn_bwd_noalloc", L.sparse_attn_bwd_noalloc(ctypes.byref(p),
+                                                                    _stream(q.device)))
     return dq, dk, dv

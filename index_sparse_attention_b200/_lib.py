@@ -18,6 +18,8 @@ SA_ERR_INDEX = -3
 SA_ERR_ALIGN = -4
 SA_ERR_CUDA = -5
 SA_ERR_WORKSPACE = -7
+SA_ERR_SCRATCH_LIMIT = -8
+SA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 SA_MODE_DENSE, SA_MODE_BLOCK, SA_MODE_INDEX = 0, 1, 2
 SA_TILE = 128
@@ -32,6 +34,7 @@ EXPORTS = (
     "sparse_attn_fwd",
     "sparse_attn_bwd_workspace_size",
     "sparse_attn_bwd",
+    "sparse_attn_bwd_noalloc",
     "sparse_attn_set_timing_events",
     "sparse_attn_error_string",
 )
@@ -82,6 +85,8 @@ def load():
     L.sparse_attn_bwd_workspace_size.restype = ctypes.c_size_t
     L.sparse_attn_bwd.argtypes = [P_p, vp, ctypes.c_size_t, vp]
     L.sparse_attn_bwd.restype = ctypes.c_int
+    L.sparse_attn_bwd_noalloc.argtypes = [P_p, vp]
+    L.sparse_attn_bwd_noalloc.restype = ctypes.c_int
     L.sparse_attn_set_timing_events.argtypes = [vp]
     L.sparse_attn_set_timing_events.restype = ctypes.c_int
     L.sparse_attn_error_string.argtypes = [ctypes.c_int]

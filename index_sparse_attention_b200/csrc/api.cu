@@ -155,6 +155,8 @@ extern "C" const char* sparse_attn_error_string(int code) {
     case SA_ERR_ALIGN: return "a tensor base pointer is not 16-byte aligned";
     case SA_ERR_CUDA: return "a CUDA call or kernel launch failed";
     case SA_ERR_WORKSPACE: return "workspace missing or too small";
+    case SA_ERR_SCRATCH_LIMIT:
+      return "problem needs more backward scratch than the fixed SA_NOALLOC_SCRATCH_BYTES array";
     default: return "unknown error code";
   }
 }

@@ -1,0 +1,66 @@
+// bwd_noalloc.cu -- sparse_attn_bwd_noalloc: the backward without a caller workspace.
+//
+// Some callers cannot call cudaMalloc (or hand this library a workspace): code that
+// runs inside a host framework which owns every device allocation and passes only
+// input and output tensors (a plugin or a serving backend), or latency-critical loops
+// where cudaMalloc's implicit device synchronisation is not acceptable.  For them this
+// entry point runs exactly the same kernels as sparse_attn_bwd, with the backward's
+// scratch (fp32 Delta and the fp32 dQ accumulator) taken from a fixed, file-scope
+// device array instead of a caller-provided buffer.
+//
+// Properties a caller must know:
+//  - The array has SA_NOALLOC_SCRATCH_BYTES bytes; every GPU that loads this library
+//    holds it until the process exits.  Problems whose scratch
+//    (sparse_attn_bwd_workspace_size) exceeds it are rejected with
+//    SA_ERR_SCRATCH_LIMIT before anything is enqueued.
+//  - The first call on each device looks up the array's device address with
+//    cudaGetSymbolAddress (with that device current).  Make that first call before
+//    any stream capture.
+//  - Every call on a device shares the one array, and each call overwrites it (the
+//    preprocess kernel writes Delta and zeroes the dQ accumulator before use).  Calls
+//    whose work overlaps on the GPU (different streams without ordering, or several
+//    host threads) race on it: serialise them.
+//  - Nothing here allocates: no cudaMalloc, cudaFree or allocating library routine.
+#include <mutex>
+
+#include "sa_device.cuh"
+#include "sa_kernels.h"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// In host code this name is only a host-side stand-in for the device array: its
+// device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_bwd_scratch[SA_NOALLOC_SCRATCH_BYTES];
+
+void* g_scratch_ptr[kMaxDevices];
+cudaError_t g_scratch_rc[kMaxDevices];
+std::once_flag g_scratch_once[kMaxDevices];
+
+// Device address of the scratch array on the current device (looked up once per device).
+void* scratch_address(int device, cudaError_t* rc) {
+  std::call_once(g_scratch_once[device], [device] {
+    void* p = nullptr;
+    g_scratch_rc[device] = cudaGetSymbolAddress(&p, g_bwd_scratch);
+    g_scratch_ptr[device] = g_scratch_rc[device] == cudaSuccess ? p : nullptr;
+  });
+  *rc = g_scratch_rc[device];
+  return g_scratch_ptr[device];
+}
+
+}  // namespace
+
+extern "C" int sparse_attn_bwd_noalloc(const sparse_attn_params* p, sa_stream_t stream) {
+  if (!p) return SA_ERR_INVALID;
+  const size_t need = sparse_attn_bwd_workspace_size(p);
+  if (need == 0) return SA_ERR_INVALID;
+  if (need > static_cast<size_t>(SA_NOALLOC_SCRATCH_BYTES)) return SA_ERR_SCRATCH_LIMIT;
+  int device = -1;
+  if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= kMaxDevices)
+    return SA_ERR_CUDA;
+  cudaError_t rc;
+  void* scratch = scratch_address(device, &rc);
+  if (rc != cudaSuccess || scratch == nullptr) return SA_ERR_CUDA;
+  return sparse_attn_bwd(p, scratch, static_cast<size_t>(SA_NOALLOC_SCRATCH_BYTES), stream);
+}
