@@ -2,6 +2,8 @@
 // launches of the forward and backward kernels.  No device memory is allocated here.
 #include <cudaTypedefs.h>
 
+#include <cstdio>
+#include <cstdlib>
 #include <mutex>
 
 #include "sa_device.cuh"
@@ -10,6 +12,13 @@
 using namespace sa;
 
 namespace sa {
+int cuda_error(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return SA_OK;
+  if (std::getenv("SA_DEBUG"))
+    std::fprintf(stderr, "sparse_attn: %s: %s (%s)\n", what, cudaGetErrorName(e),
+                 cudaGetErrorString(e));
+  return SA_ERR_CUDA;
+}
 cudaEvent_t* g_timing_events = nullptr;
 static cudaEvent_t g_events_copy[6];
 }  // namespace sa

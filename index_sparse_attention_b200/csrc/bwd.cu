@@ -30,6 +30,9 @@
 #include "sa_device.cuh"
 #include "sa_kernels.h"
 
+#include <cstdio>
+#include <cstdlib>
+
 namespace sa {
 
 // ------------------------------------------------------------------------------------
@@ -104,11 +107,15 @@ struct BwdCfg {
   static constexpr int kQOff = kVOff + kVBytes;                    // per stage: Q then dO
   static constexpr int kStageBytes = kQBytes + kOBytes;
   static constexpr int kDSOff = kQOff + kStages * kStageBytes;     // two dS^T buffers
-  static constexpr int kLOff = kDSOff + 2 * kDSBytes;              // per stage: lse2[64], delta[64]
+  // fp32 dQ staging tile [2 panels][32 q][64 d]: a buffer of its own when shared memory
+  // allows (two Q/dO stages), otherwise the step's dS^T buffer once dQ^T has read it
+  static constexpr bool kOwnStage = kStages == 2;
+  static constexpr int kDQOff = kDSOff + 2 * kDSBytes;
+  static constexpr int kLOff = kDQOff + (kOwnStage ? 128 * 32 * 4 : 0);  // lse2[64], delta[64]
   static constexpr int kBMOff = kLOff + kStages * 2 * kBM * 4;     // per stage: bitmap words [64][4]
   static constexpr int kBarOff = kBMOff + kStages * kBM * 4 * 4;
   static constexpr int kSmem = kBarOff + 256 + 1024;
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 448;
   // head-dim chunks of this CTA: dK [kc0, kc0 + kcn), dV [vc0, vc0 + vcn)
   static constexpr int kDKMax = NSPLIT == 1 ? DQK : (DQK == 192 ? 128 : DQK / 2);
   static constexpr int kDVMax = DV / NSPLIT;
@@ -127,10 +134,13 @@ enum : int {
   kBFin = 17, kBDrainB = 18, kNumBarsB = 19
 };
 
-// Warp roles: 0 producer, 1 MMA, 2-5 elementwise (one key row per thread), 6-9 dQ drain
+// Warp roles: 0 producer, 1 MMA, 2-9 elementwise (one key row and 32 of the 64 query
+// columns per thread: warps 2-5 columns 0-31, warps 6-9 columns 32-63), 10-13 dQ drain
 // (one head-dim row of the dQ^T window per thread).
+// Bf16 P^T / dS^T of query columns [32h, 32h+32) are packed into TMEM columns
+// [32h, 32h+16) of the S^T / dP^T buffer, inside the range that half itself read.
 template <int DQK, int DV, int NSPLIT>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
     sparse_bwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v,
@@ -181,7 +191,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(BAR(kBQE + s), 1);
       mbar_init(BAR(kBLF + s), 32);
       mbar_init(BAR(kBSF + s), 1);
-      mbar_init(BAR(kBPF + s), 128);
+      mbar_init(BAR(kBPF + s), 256);
       mbar_init(BAR(kBDQF + s), 1);
       mbar_init(BAR(kBDQE + s), 128);
       mbar_init(BAR(kBDSE + s), 128);
@@ -198,7 +208,8 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  // broadcast from lane 0 so that the compiler can treat it as warp-uniform
+  const uint32_t tmem = __shfl_sync(0xFFFFFFFFu, *tmem_slot, 0);
 
   // iteration -> (query head, query tile, half)
   auto decode = [&](int it, int& h, int& m0, bool& partial) {
@@ -214,7 +225,7 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
     if (n_iter > 0) {
-      if (lane == 0) {
+      if (elect_one()) {
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
@@ -232,10 +243,10 @@ __global__ void __launch_bounds__(320, 1)
         int h, m0;
         bool partial;
         decode(it, h, m0, partial);
+        m0 = __shfl_sync(0xFFFFFFFFu, m0, 0);  // warp-uniform TMA coordinate
         const int st = it % C::kStages, u = it / C::kStages;
-        const bool w_ok = mbar_wait(BAR(kBQE + st), (u & 1) ^ 1, abort_flag, a.status);
-        if (!__all_sync(0xFFFFFFFFu, w_ok)) break;
-        if (lane == 0) {
+        if (!warp_wait(BAR(kBQE + st), (u & 1) ^ 1, abort_flag, a.status)) break;
+        if (elect_one()) {
           mbar_arrive_expect_tx(BAR(kBQF + st), C::kQBytes + C::kOBytes);
           const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
           for (int c = 0; c < DQK / 64; ++c)
@@ -277,38 +288,47 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_iter > 0) {
+    // The whole warp runs this loop (converged, warp-uniform operands); one elected
+    // lane issues each batch of tcgen05 instructions.
+    if (n_iter > 0) {
       constexpr uint32_t idesc_s = idesc_bf16(128, BM, 0, 0);      // S^T, dP^T
       constexpr uint32_t idesc_dq = idesc_bf16(128, BM, 1, 1);     // dQ^T = K^T dS^T
       const uint32_t idesc_dv = idesc_bf16(128, vcn, 0, 1);        // dV += P^T dO
       const uint32_t idesc_dk = idesc_bf16(128, kcn, 0, 1);        // dK += dS^T Q
       const uint32_t kbase = sbase + C::kKOff, vbase = sbase + C::kVOff;
-      bool ok = mbar_wait(BAR(kBKV), 0, abort_flag, a.status);
+      // descriptors of panel bases; a k-step adds its byte offset / 16 to the
+      // start-address field (no carry: shared addresses stay below 2^18)
+      const uint64_t kd = sw128_desc(kbase, 16, 1024), vd = sw128_desc(vbase, 16, 1024);
+      const uint64_t kwd = sw128_desc(kbase + (qw0 / 64) * C::kKPanel, C::kKPanel, 1024);
+      bool ok = warp_wait(BAR(kBKV), 0, abort_flag, a.status);
       // S^T(j) and dP^T(j) into TMEM buffer j & 1
       auto issue_sdp = [&](int j) -> bool {
         const int st = j % C::kStages, u = j / C::kStages, bj = j & 1;
-        if (!mbar_wait(BAR(kBQF + st), u & 1, abort_flag, a.status)) return false;
+        if (!warp_wait(BAR(kBQF + st), u & 1, abort_flag, a.status)) return false;
         // the dQ^T of step j-2 lives in this buffer until it has been drained
-        if (j >= 2 && !mbar_wait(BAR(kBDQE + bj), ((j - 2) >> 1) & 1, abort_flag, a.status))
+        if (j >= 2 && !warp_wait(BAR(kBDQE + bj), ((j - 2) >> 1) & 1, abort_flag, a.status))
           return false;
         tc_fence_after();
         const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
-        const uint32_t os = qs + C::kQBytes;
+        const uint64_t qd = sw128_desc(qs, 16, 1024), od = sw128_desc(qs + C::kQBytes, 16, 1024);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < DQK / 16; ++kk) {
-          const uint32_t ka = (kk >> 2) * C::kKPanel + (kk & 3) * 32;
-          const uint32_t qb = (kk >> 2) * C::kQPanel + (kk & 3) * 32;
-          umma_ss(tmem + C::kColS + 64 * bj, sw128_desc(kbase + ka, 16, 1024),
-                  sw128_desc(qs + qb, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-        }
+          for (int kk = 0; kk < DQK / 16; ++kk) {
+            const uint32_t ka = (kk >> 2) * C::kKPanel + (kk & 3) * 32;
+            const uint32_t qb = (kk >> 2) * C::kQPanel + (kk & 3) * 32;
+            umma_ss(tmem + C::kColS + 64 * bj, kd + (ka >> 4), qd + (qb >> 4), idesc_s,
+                    kk > 0 ? 1u : 0u);
+          }
 #pragma unroll
-        for (int kk = 0; kk < DV / 16; ++kk) {
-          const uint32_t va = (kk >> 2) * C::kKPanel + (kk & 3) * 32;
-          const uint32_t ob = (kk >> 2) * C::kQPanel + (kk & 3) * 32;
-          umma_ss(tmem + C::kColDP + 64 * bj, sw128_desc(vbase + va, 16, 1024),
-                  sw128_desc(os + ob, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < DV / 16; ++kk) {
+            const uint32_t va = (kk >> 2) * C::kKPanel + (kk & 3) * 32;
+            const uint32_t ob = (kk >> 2) * C::kQPanel + (kk & 3) * 32;
+            umma_ss(tmem + C::kColDP + 64 * bj, vd + (va >> 4), od + (ob >> 4), idesc_s,
+                    kk > 0 ? 1u : 0u);
+          }
+          umma_commit(BAR(kBSF + bj));
         }
-        umma_commit(BAR(kBSF + bj));
+        __syncwarp();
         return true;
       };
       if (ok) ok = issue_sdp(0);
@@ -316,37 +336,40 @@ __global__ void __launch_bounds__(320, 1)
         const int st = it % C::kStages, bi = it & 1;
         // with two Q/dO stages the next S^T / dP^T overlap this step's elementwise work
         if (C::kStages >= 2 && it + 1 < n_iter && !issue_sdp(it + 1)) break;
-        if (!mbar_wait(BAR(kBPF + bi), (it >> 1) & 1, abort_flag, a.status)) break;
+        if (!warp_wait(BAR(kBPF + bi), (it >> 1) & 1, abort_flag, a.status)) break;
         tc_fence_after();
         const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
-        const uint32_t os = qs + C::kQBytes;
-        // dV += P^T dO  and  dK += dS^T Q (K = 64 queries: four k-steps of 16)
+        const uint64_t qmn = sw128_desc(qs + (kc0 / 64) * C::kQPanel, C::kQPanel, 1024);
+        const uint64_t omn = sw128_desc(qs + C::kQBytes + (vc0 / 64) * C::kQPanel, C::kQPanel, 1024);
+        const uint64_t dsd = sw128_desc(sbase + C::kDSOff + bi * C::kDSBytes, C::kKPanel, 1024);
+        if (elect_one()) {
+          // dV += P^T dO  and  dK += dS^T Q (K = 64 queries: four k-steps of 16)
 #pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)
-          umma_ts(tmem + C::kColDV, tmem + C::kColS + 64 * bi + kk * 8,
-                  sw128_desc(os + (vc0 / 64) * C::kQPanel + kk * 2048, C::kQPanel, 1024), idesc_dv,
-                  (it > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BM / 16; ++kk)
+            umma_ts(tmem + C::kColDV, tmem + C::kColS + 64 * bi + (kk >> 1) * 32 + (kk & 1) * 8,
+                    omn + ((kk * 2048) >> 4), idesc_dv, (it > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)
-          umma_ts(tmem + C::kColDK, tmem + C::kColDP + 64 * bi + kk * 8,
-                  sw128_desc(qs + (kc0 / 64) * C::kQPanel + kk * 2048, C::kQPanel, 1024), idesc_dk,
-                  (it > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(BAR(kBQE + st));
-        // dQ^T = K^T dS^T over the 128 keys, into the dP^T buffer dK has just consumed
-        const uint32_t dsb = sbase + C::kDSOff + bi * C::kDSBytes;
+          for (int kk = 0; kk < BM / 16; ++kk)
+            umma_ts(tmem + C::kColDK, tmem + C::kColDP + 64 * bi + (kk >> 1) * 32 + (kk & 1) * 8,
+                    qmn + ((kk * 2048) >> 4), idesc_dk, (it > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(BAR(kBQE + st));
+          // dQ^T = K^T dS^T over the 128 keys, into the dP^T buffer dK has just consumed
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ss(tmem + C::kColDP + 64 * bi,
-                  sw128_desc(kbase + (qw0 / 64) * C::kKPanel + kk * 2048, C::kKPanel, 1024),
-                  sw128_desc(dsb + kk * 2048, C::kKPanel, 1024), idesc_dq, kk > 0 ? 1u : 0u);
-        umma_commit(BAR(kBDQF + bi));
+          for (int kk = 0; kk < 128 / 16; ++kk)
+            umma_ss(tmem + C::kColDP + 64 * bi, kwd + ((kk * 2048) >> 4), dsd + ((kk * 2048) >> 4),
+                    idesc_dq, kk > 0 ? 1u : 0u);
+          umma_commit(BAR(kBDQF + bi));
+        }
+        __syncwarp();
         if (C::kStages == 1 && it + 1 < n_iter && !issue_sdp(it + 1)) break;
       }
-      umma_commit(BAR(kBFin));
+      if (elect_one()) umma_commit(BAR(kBFin));
+      __syncwarp();
     }
-  } else if (warp < 6) {
+  } else if (warp < 10) {
     // ------------------------------------------------------------------ elementwise
     const int quarter = warp & 3;
+    const int hc = (warp - 2) >> 2;              // which 32 of the 64 query columns
     const int r = quarter * 32 + lane;           // key row of the tile = TMEM lane
     const int64_t j = static_cast<int64_t>(nt) * 128 + r;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -361,68 +384,72 @@ __global__ void __launch_bounds__(320, 1)
       const int st = it % C::kStages, u = it / C::kStages, bi = it & 1;
       bool w_ok = mbar_wait(BAR(kBLF + st), u & 1, abort_flag, a.status);
       w_ok = w_ok && mbar_wait(BAR(kBSF + bi), (it >> 1) & 1, abort_flag, a.status);
-      // the dS^T buffer was the dQ staging area of step it-2
-      if (it >= 2) w_ok = w_ok && mbar_wait(BAR(kBDSE + bi), ((it - 2) >> 1) & 1, abort_flag, a.status);
+      // the dS^T buffer is free once dQ^T of step it-2 has read it (and, without a
+      // staging buffer of its own, once the drain of step it-2 has used it)
+      if (it >= 2) {
+        if (C::kOwnStage)
+          w_ok = w_ok && mbar_wait(BAR(kBDQF + bi), ((it - 2) >> 1) & 1, abort_flag, a.status);
+        else
+          w_ok = w_ok && mbar_wait(BAR(kBDSE + bi), ((it - 2) >> 1) & 1, abort_flag, a.status);
+      }
       if (!__all_sync(0xFFFFFFFFu, w_ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float* ls = lbuf + st * 2 * BM;
+      const float* ls = lbuf + st * 2 * BM + 32 * hc;
       uint8_t* dsrow = smem + C::kDSOff + bi * C::kDSBytes + r * 128;
-      // allowed-query mask of this key row over the 64 queries (partial tiles only)
-      uint64_t qmask = ~0ull;
+      const uint32_t cs = C::kColS + 64 * bi + 32 * hc, cd = C::kColDP + 64 * bi + 32 * hc;
+      uint32_t s_u[32], p_u[32];
+      tmem_ld32(tl + cs, s_u);
+      tmem_ld32(tl + cd, p_u);
+      // allowed-query mask of this key row over this half's 32 queries (partial tiles)
+      uint32_t cm = 0xFFFFFFFFu;
       if (partial) {
-        qmask = key_ok ? ~0ull : 0ull;
+        const int64_t q0 = m0 + 32 * hc;
+        cm = key_ok ? 0xFFFFFFFFu : 0u;
         if (a.causal) {  // i >= j
-          const int64_t lo = j - m0;
-          qmask &= lo <= 0 ? ~0ull : (lo >= 64 ? 0ull : (~0ull << lo));
+          const int64_t lo = j - q0;
+          cm &= lo <= 0 ? 0xFFFFFFFFu : (lo >= 32 ? 0u : (0xFFFFFFFFu << lo));
         }
         if (a.mode == SA_MODE_BLOCK && a.bs == 64 && key_ok) {
           const int64_t mb = m0 / 64;
           const bool m = mb < a.Mb &&
                          __ldg(a.mask + (bg * a.Mb + mb) * static_cast<int64_t>(a.Nb) + j / 64) != 0;
-          if (!m) qmask = 0ull;
+          if (!m) cm = 0u;
         } else if (a.mode == SA_MODE_INDEX) {
-          const uint32_t* bw = bmbuf + st * BM * 4 + (r >> 5);
-          uint64_t bits = 0ull;
+          const uint32_t* bw = bmbuf + st * BM * 4 + (32 * hc) * 4 + (r >> 5);
+          uint32_t bits = 0u;
 #pragma unroll 8
-          for (int q = 0; q < BM; ++q) bits |= static_cast<uint64_t>((bw[q * 4] >> lane) & 1u) << q;
-          qmask &= bits;
+          for (int q = 0; q < 32; ++q) bits |= ((bw[q * 4] >> lane) & 1u) << q;
+          cm &= bits;
         }
       }
+      tmem_wait_ld();
+      uint32_t pk[16], dk[16];
 #pragma unroll
-      for (int cc = 0; cc < BM / 32; ++cc) {
-        uint32_t s_u[32], p_u[32];
-        tmem_ld32(tl + C::kColS + 64 * bi + cc * 32, s_u);
-        tmem_ld32(tl + C::kColDP + 64 * bi + cc * 32, p_u);
-        tmem_wait_ld();
-        const uint32_t cm = static_cast<uint32_t>(qmask >> (32 * cc));
-        uint32_t pk[16], dk[16];
+      for (int e = 0; e < 16; ++e) {
+        float pv[2], dv2[2];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float pv[2], dv2[2];
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const int q = cc * 32 + 2 * e + t;
-            const float s = __uint_as_float(s_u[2 * e + t]);
-            const float p = ((cm >> (2 * e + t)) & 1u) ? ex2(fmaf(s, a.scale_log2, -ls[q])) : 0.f;
-            pv[t] = p;
-            dv2[t] = p * (__uint_as_float(p_u[2 * e + t]) - ls[BM + q]);
-          }
-          pk[e] = pack_bf16x2(pv[0], pv[1]);
-          dk[e] = pack_bf16x2(dv2[0], dv2[1]);
+        for (int t = 0; t < 2; ++t) {
+          const int q = 2 * e + t;
+          const float sv = __uint_as_float(s_u[q]);
+          const float p = ((cm >> q) & 1u) ? ex2(fmaf(sv, a.scale_log2, -ls[q])) : 0.f;
+          pv[t] = p;
+          dv2[t] = p * (__uint_as_float(p_u[q]) - ls[BM + q]);
         }
-        tmem_st16(tl + C::kColS + 64 * bi + cc * 16, pk);
-        tmem_st16(tl + C::kColDP + 64 * bi + cc * 16, dk);
-        // dS^T row into shared memory, 128-byte swizzled: 16-byte chunk c of row r
-        // lives at chunk c ^ (r % 8)
+        pk[e] = pack_bf16x2(pv[0], pv[1]);
+        dk[e] = pack_bf16x2(dv2[0], dv2[1]);
+      }
+      tmem_st16(tl + cs, pk);
+      tmem_st16(tl + cd, dk);
+      // dS^T row into shared memory, 128-byte swizzled: 16-byte chunk c of row r
+      // lives at chunk c ^ (r % 8)
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const int c = cc * 4 + c4;
-          *reinterpret_cast<uint4*>(dsrow + ((c ^ (r & 7)) << 4)) =
-              make_uint4(dk[4 * c4], dk[4 * c4 + 1], dk[4 * c4 + 2], dk[4 * c4 + 3]);
-        }
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const int c = hc * 4 + c4;
+        *reinterpret_cast<uint4*>(dsrow + ((c ^ (r & 7)) << 4)) =
+            make_uint4(dk[4 * c4], dk[4 * c4 + 1], dk[4 * c4 + 2], dk[4 * c4 + 3]);
       }
       tmem_wait_st();
       fence_proxy_async_smem();
@@ -440,6 +467,7 @@ __global__ void __launch_bounds__(320, 1)
                            ((static_cast<int64_t>(b) * a.Sk + j) * a.HK + g) * dqk_real;
     __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(a.dv) +
                            ((static_cast<int64_t>(b) * a.Sk + j) * a.HK + g) * dv_real;
+    // the two halves of the elementwise warps store alternating 32-column chunks
     for (int pass = 0; pass < 2; ++pass) {
       const int n = pass == 0 ? kcn : vcn;
       const int d0 = pass == 0 ? kc0 : vc0;
@@ -447,7 +475,7 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t col = pass == 0 ? C::kColDK : C::kColDV;
       const float sc = pass == 0 ? a.scale : 1.f;
       __nv_bfloat16* out = pass == 0 ? dkrow : dvrow;
-      for (int c = 0; c < n; c += 32) {
+      for (int c = 32 * hc; c < n; c += 64) {
         uint32_t v[32];
         if (have) {
           tmem_ld32(tl + col + c, v);
@@ -475,7 +503,7 @@ __global__ void __launch_bounds__(320, 1)
     // [64-column panel][32 q][64 d] tiles that bulk reduce-adds push into dQ_acc.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const int dtid = threadIdx.x - 192;  // 0..127 within the drain warpgroup
+    const int dtid = threadIdx.x - 320;  // 0..127 within the drain warpgroup
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const int p = r >> 6;  // panel of this row within the window
     // a panel is reduced when it lies in this CTA's dQ range and inside Dqk
@@ -502,11 +530,14 @@ __global__ void __launch_bounds__(320, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(BAR(kBDQE + bi));
-      float* stage = reinterpret_cast<float*>(smem + C::kDSOff + bi * C::kDSBytes);
-      const uint32_t stage_s = sbase + C::kDSOff + bi * C::kDSBytes;
+      const int soff = C::kOwnStage ? C::kDQOff : C::kDSOff + bi * C::kDSBytes;
+      float* stage = reinterpret_cast<float*>(smem + soff);
+      const uint32_t stage_s = sbase + soff;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        if (half == 1) {
+        if (half == 1 || C::kOwnStage) {
+          // the previous reduce (this step's first half, or the last step's second
+          // half in the own staging buffer) must have read the tile
           if (dtid == 0) bulk_wait_group_read0();
           named_bar_sync(1, 128);
         }
@@ -520,16 +551,21 @@ __global__ void __launch_bounds__(320, 1)
           bulk_commit_group();
         }
       }
-      if (dtid == 0) bulk_wait_group_read0();
-      named_bar_sync(1, 128);
-      mbar_arrive(BAR(kBDSE + bi));
+      if (!C::kOwnStage) {
+        if (dtid == 0) bulk_wait_group_read0();
+        named_bar_sync(1, 128);
+        mbar_arrive(BAR(kBDSE + bi));
+      }
     }
     if (dtid == 0) bulk_wait_group0();  // every reduce has landed before the CTA ends
   }
 
-  if (warp == 1 && lane == 0 && *abort_flag) {
-    umma_commit(BAR(kBDrainB));
-    mbar_wait_limited(BAR(kBDrainB), 0);
+  if (warp == 1 && *abort_flag) {
+    if (elect_one()) {
+      umma_commit(BAR(kBDrainB));
+      mbar_wait_limited(BAR(kBDrainB), 0);
+    }
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -544,17 +580,34 @@ static int launch_bwd_main(const AttnArgs& a, const TensorMaps& m, cudaStream_t 
   using C = BwdCfg<DQK, DV, NSPLIT>;
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(sparse_bwd_kernel<DQK, DV, NSPLIT>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) != cudaSuccess)
-      return SA_ERR_CUDA;
+    const int rc = cuda_error(cudaFuncSetAttribute(sparse_bwd_kernel<DQK, DV, NSPLIT>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   C::kSmem),
+                              "backward smem attribute");
+    if (rc) return rc;
     attr_set = true;
+    if (std::getenv("SA_DEBUG")) {
+      cudaFuncAttributes fa;
+      const cudaError_t qe = cudaFuncGetAttributes(&fa, sparse_bwd_kernel<DQK, DV, NSPLIT>);
+      int occ = -1;
+      const cudaError_t oe = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+          &occ, sparse_bwd_kernel<DQK, DV, NSPLIT>, C::kThreads, C::kSmem);
+      std::fprintf(stderr, "sparse_attn: attribute query %s, occupancy query %s -> %d\n",
+                   cudaGetErrorName(qe), cudaGetErrorName(oe), occ);
+      if (qe == cudaSuccess)
+        std::fprintf(stderr,
+                     "sparse_attn: backward kernel regs %d, max threads %d, static smem %zu, "
+                     "local %zu, max dyn smem %d, launch %d threads x %d B smem\n",
+                     fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes, fa.localSizeBytes,
+                     fa.maxDynamicSharedSizeBytes, C::kThreads, C::kSmem);
+    }
   }
   dim3 grid(a.Tn * NSPLIT, a.HK, a.B);
   record_event(3, st);
   sparse_bwd_kernel<DQK, DV, NSPLIT><<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.v, m.dout,
                                                                            m.dq_acc, a);
   record_event(4, st);
-  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+  return check_launch("backward main kernel launch");
 }
 
 int launch_bwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
@@ -566,7 +619,7 @@ int launch_bwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
     bwd_pre_kernel<<<static_cast<unsigned>(blocks), warps * 32, 0, st>>>(
         static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.delta,
         a.dq_acc, rows, a.Sq, a.HQ, a.Dv, a.Dqk);
-    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+    if (check_launch("backward preprocess launch")) return SA_ERR_CUDA;
   }
   int rc;
   if (a.Dqk == 64 && a.Dv == 64)
@@ -584,7 +637,7 @@ int launch_bwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
   bwd_post_kernel<<<static_cast<unsigned>(min64((n4 + 255) / 256, 148 * 16)), 256, 0, st>>>(
       a.dq_acc, static_cast<__nv_bfloat16*>(a.dq), n4, a.scale);
   record_event(5, st);
-  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+  return check_launch("backward postprocess launch");
 }
 
 }  // namespace sa

@@ -100,33 +100,44 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  // broadcast from lane 0 so that the compiler can treat it as warp-uniform
+  const uint32_t tmem = __shfl_sync(0xFFFFFFFFu, *tmem_slot, 0);
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
-    if (lane == 0 && n_iter > 0) {
-      prefetch_tensormap(&tm_q);
-      prefetch_tensormap(&tm_k);
-      prefetch_tensormap(&tm_v);
-      mbar_arrive_expect_tx(BAR(kBQ), C::kQBytes);
-      for (int c = 0; c < DQK / 64; ++c)
-        tma_load_4d(sbase + C::kQOff + c * C::kPanel, &tm_q, BAR(kBQ), c * 64, mt * 128, h, b);
-      for (int it = 0; it < n_iter; ++it) {
-        const int nt = __ldg(list + it);
-        const int ks = it % C::kKStages, ku = it / C::kKStages;
-        if (!mbar_wait(BAR(kBKE + ks), (ku & 1) ^ 1, abort_flag, a.status)) break;
-        mbar_arrive_expect_tx(BAR(kBKF + ks), C::kKBytes);
+    // converged warp; one elected lane issues the copies
+    if (n_iter > 0) {
+      if (elect_one()) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        mbar_arrive_expect_tx(BAR(kBQ), C::kQBytes);
         for (int c = 0; c < DQK / 64; ++c)
-          tma_load_4d(sbase + C::kKOff + ks * C::kKBytes + c * C::kPanel, &tm_k, BAR(kBKF + ks),
-                      c * 64, nt * 128, g, b);
-        const int vs = it % C::kVStages, vu = it / C::kVStages;
-        if (!mbar_wait(BAR(kBVE + vs), (vu & 1) ^ 1, abort_flag, a.status)) break;
-        mbar_arrive_expect_tx(BAR(kBVF + vs), C::kVBytes);
-        for (int c = 0; c < DV / 64; ++c)
-          tma_load_4d(sbase + C::kVOff + vs * C::kVBytes + c * C::kPanel, &tm_v, BAR(kBVF + vs),
-                      c * 64, nt * 128, g, b);
+          tma_load_4d(sbase + C::kQOff + c * C::kPanel, &tm_q, BAR(kBQ), c * 64, mt * 128, h, b);
       }
-      if (*abort_flag) {
+      __syncwarp();
+      for (int it = 0; it < n_iter; ++it) {
+        const int nt = __shfl_sync(0xFFFFFFFFu, __ldg(list + it), 0);
+        const int ks = it % C::kKStages, ku = it / C::kKStages;
+        if (!warp_wait(BAR(kBKE + ks), (ku & 1) ^ 1, abort_flag, a.status)) break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(BAR(kBKF + ks), C::kKBytes);
+          for (int c = 0; c < DQK / 64; ++c)
+            tma_load_4d(sbase + C::kKOff + ks * C::kKBytes + c * C::kPanel, &tm_k, BAR(kBKF + ks),
+                        c * 64, nt * 128, g, b);
+        }
+        __syncwarp();
+        const int vs = it % C::kVStages, vu = it / C::kVStages;
+        if (!warp_wait(BAR(kBVE + vs), (vu & 1) ^ 1, abort_flag, a.status)) break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(BAR(kBVF + vs), C::kVBytes);
+          for (int c = 0; c < DV / 64; ++c)
+            tma_load_4d(sbase + C::kVOff + vs * C::kVBytes + c * C::kPanel, &tm_v, BAR(kBVF + vs),
+                        c * 64, nt * 128, g, b);
+        }
+        __syncwarp();
+      }
+      if (*abort_flag && lane == 0) {
         // Let the loads already issued land before the CTA may leave (time-limited).
         mbar_wait_limited(BAR(kBQ), 0);
         for (int it = max(0, n_iter - 2); it < n_iter; ++it) {
@@ -137,48 +148,58 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_iter > 0) {
+    // The whole warp runs this loop (converged, warp-uniform operands); one elected
+    // lane issues each batch of tcgen05 instructions.
+    if (n_iter > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(128, DV, 0, 1);
-      bool ok = mbar_wait(BAR(kBQ), 0, abort_flag, a.status);
+      const uint64_t qdesc = sw128_desc(sbase + C::kQOff, 16, 1024);
+      bool ok = warp_wait(BAR(kBQ), 0, abort_flag, a.status);
       auto issue_s = [&](int it) -> bool {
         const int ks = it % C::kKStages, ku = it / C::kKStages;
-        if (!mbar_wait(BAR(kBKF + ks), ku & 1, abort_flag, a.status)) return false;
+        if (!warp_wait(BAR(kBKF + ks), ku & 1, abort_flag, a.status)) return false;
         tc_fence_after();
-        const uint32_t qa = sbase + C::kQOff;
-        const uint32_t kb = sbase + C::kKOff + ks * C::kKBytes;
+        const uint64_t kdesc = sw128_desc(sbase + C::kKOff + ks * C::kKBytes, 16, 1024);
         const uint32_t d = tmem + static_cast<uint32_t>((it & 1) * 128);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < DQK / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kPanel + (kk & 3) * 32;
-          umma_ss(d, sw128_desc(qa + off, 16, 1024), sw128_desc(kb + off, 16, 1024), idesc_qk,
-                  kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < DQK / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * C::kPanel + (kk & 3) * 32) >> 4;
+            umma_ss(d, qdesc + off, kdesc + off, idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(BAR(kBSF + (it & 1)));
+          umma_commit(BAR(kBKE + ks));
         }
-        umma_commit(BAR(kBSF + (it & 1)));
-        umma_commit(BAR(kBKE + ks));
+        __syncwarp();
         return true;
       };
       if (ok) ok = issue_s(0);
       for (int it = 0; ok && it < n_iter; ++it) {
         if (it + 1 < n_iter && !issue_s(it + 1)) break;
         const int vs = it % C::kVStages, vu = it / C::kVStages;
-        if (!mbar_wait(BAR(kBPF + (it & 1)), (it >> 1) & 1, abort_flag, a.status)) break;
-        if (!mbar_wait(BAR(kBVF + vs), vu & 1, abort_flag, a.status)) break;
+        if (!warp_wait(BAR(kBPF + (it & 1)), (it >> 1) & 1, abort_flag, a.status)) break;
+        if (!warp_wait(BAR(kBVF + vs), vu & 1, abort_flag, a.status)) break;
         tc_fence_after();
-        const uint32_t vb = sbase + C::kVOff + vs * C::kVBytes;
+        const uint64_t vdesc = sw128_desc(sbase + C::kVOff + vs * C::kVBytes, C::kPanel, 1024);
         const uint32_t pa = tmem + static_cast<uint32_t>((it & 1) * 128);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ts(tmem + C::kOCol, pa + kk * 8, sw128_desc(vb + kk * 2048, C::kPanel, 1024),
-                  idesc_pv, (it > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(BAR(kBOD));
-        umma_commit(BAR(kBVE + vs));
-        if (it == n_iter - 1) umma_commit(BAR(kBOFin));  // the final O is complete
+          for (int kk = 0; kk < 128 / 16; ++kk)
+            umma_ts(tmem + C::kOCol, pa + kk * 8, vdesc + ((kk * 2048) >> 4), idesc_pv,
+                    (it > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(BAR(kBOD));
+          umma_commit(BAR(kBVE + vs));
+          if (it == n_iter - 1) umma_commit(BAR(kBOFin));  // the final O is complete
+        }
+        __syncwarp();
       }
       if (*abort_flag) {
         // Drain: wait (time-limited) for the MMAs issued so far before TMEM is released.
-        umma_commit(BAR(kBDrain));
-        mbar_wait_limited(BAR(kBDrain), 0);
+        if (elect_one()) {
+          umma_commit(BAR(kBDrain));
+          mbar_wait_limited(BAR(kBDrain), 0);
+        }
+        __syncwarp();
       }
     }
   } else {
@@ -341,16 +362,18 @@ static int launch_fwd_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st)
   using C = FwdCfg<DQK, DV>;
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(sparse_fwd_kernel<DQK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmem) != cudaSuccess)
-      return SA_ERR_CUDA;
+    const int rc = cuda_error(cudaFuncSetAttribute(sparse_fwd_kernel<DQK, DV>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   C::kSmem),
+                              "forward smem attribute");
+    if (rc) return rc;
     attr_set = true;
   }
   dim3 grid(a.Tm, a.HQ, a.B);
   record_event(0, st);
   sparse_fwd_kernel<DQK, DV><<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.v, a);
   record_event(1, st);
-  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+  return check_launch("forward kernel launch");
 }
 
 int launch_fwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {

@@ -97,6 +97,23 @@ __device__ __forceinline__ bool mbar_wait_limited(uint32_t bar, uint32_t parity)
   return true;
 }
 
+// Warp-collective form: every lane waits; the result is the same on every lane.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          int32_t* status) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort, status));
+}
+
+// Picks one active lane of a converged warp (true on that lane only).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // ---------------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library)
 // ---------------------------------------------------------------------------------

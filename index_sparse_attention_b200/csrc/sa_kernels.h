@@ -45,6 +45,11 @@ inline void record_event(int k, cudaStream_t st) {
   if (g_timing_events) cudaEventRecord(g_timing_events[k], st);
 }
 
+// Turns a CUDA error into SA_ERR_CUDA; with SA_DEBUG set in the environment it also
+// prints which call failed and why.
+int cuda_error(cudaError_t e, const char* what);
+inline int check_launch(const char* what) { return cuda_error(cudaGetLastError(), what); }
+
 int launch_fwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st);
 int launch_bwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st);
 
