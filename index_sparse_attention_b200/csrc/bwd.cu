@@ -100,7 +100,12 @@ struct BwdCfg {
   static constexpr int kVBytes = 128 * DV * 2;
   static constexpr int kQBytes = kBM * DQK * 2;
   static constexpr int kOBytes = kBM * DV * 2;
-  static constexpr int kStages = (DQK + DV >= 512) ? 1 : 2;
+  // Q/dO stages: three at D=128, two at (192,128); one at (256,256), split in two
+  // halves with their own barriers: the panels this CTA's dK/dV chunk needs (held until
+  // dK/dV are done) and the other panels (free once S^T/dP^T are done, so the next
+  // step's copy of them overlaps the elementwise work)
+  static constexpr int kStages = (DQK + DV >= 512) ? 1 : (DQK == 128 ? 3 : 2);
+  static constexpr bool kSplitStage = kStages == 1;
   static constexpr int kDSBytes = 128 * kBM * 2;     // dS^T [128 keys][64 q] bf16 (16 KB)
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kKOff + kKBytes;
@@ -109,7 +114,7 @@ struct BwdCfg {
   static constexpr int kDSOff = kQOff + kStages * kStageBytes;     // two dS^T buffers
   // fp32 dQ staging tile [2 panels][32 q][64 d]: a buffer of its own when shared memory
   // allows (two Q/dO stages), otherwise the step's dS^T buffer once dQ^T has read it
-  static constexpr bool kOwnStage = kStages == 2;
+  static constexpr bool kOwnStage = kStages >= 2;
   static constexpr int kDQOff = kDSOff + 2 * kDSBytes;
   static constexpr int kLOff = kDQOff + (kOwnStage ? 128 * 32 * 4 : 0);  // lse2[64], delta[64]
   static constexpr int kBMOff = kLOff + kStages * 2 * kBM * 4;     // per stage: bitmap words [64][4]
@@ -130,9 +135,10 @@ struct BwdCfg {
 };
 
 enum : int {
-  kBKV = 0, kBQF = 1, kBQE = 3, kBLF = 5, kBSF = 7, kBPF = 9, kBDQF = 11, kBDQE = 13, kBDSE = 15,
-  kBFin = 17, kBDrainB = 18, kNumBarsB = 19
+  kBKV = 0, kBQF = 1, kBQE = 4, kBLF = 7, kBSF = 10, kBPF = 12, kBDQF = 14, kBDQE = 16, kBDSE = 18,
+  kBFin = 20, kBDrainB = 21, kNumBarsB = 22
 };
+// With a split stage, QF/QE slot 0 guards the own panels and slot 1 the other panels.
 
 // Warp roles: 0 producer, 1 MMA, 2-9 elementwise (one key row and 32 of the 64 query
 // columns per thread: warps 2-5 columns 0-31, warps 6-9 columns 32-63), 10-13 dQ drain
@@ -186,10 +192,12 @@ __global__ void __launch_bounds__(448, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(kBKV), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < 3; ++s) {
       mbar_init(BAR(kBQF + s), 1);
       mbar_init(BAR(kBQE + s), 1);
       mbar_init(BAR(kBLF + s), 32);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(kBSF + s), 1);
       mbar_init(BAR(kBPF + s), 256);
       mbar_init(BAR(kBDQF + s), 1);
@@ -245,14 +253,39 @@ __global__ void __launch_bounds__(448, 1)
         decode(it, h, m0, partial);
         m0 = __shfl_sync(0xFFFFFFFFu, m0, 0);  // warp-uniform TMA coordinate
         const int st = it % C::kStages, u = it / C::kStages;
-        if (!warp_wait(BAR(kBQE + st), (u & 1) ^ 1, abort_flag, a.status)) break;
-        if (elect_one()) {
-          mbar_arrive_expect_tx(BAR(kBQF + st), C::kQBytes + C::kOBytes);
-          const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
-          for (int c = 0; c < DQK / 64; ++c)
-            tma_load_4d(qs + c * C::kQPanel, &tm_q, BAR(kBQF + st), c * 64, m0, h, b);
-          for (int c = 0; c < DV / 64; ++c)
-            tma_load_4d(qs + C::kQBytes + c * C::kQPanel, &tm_do, BAR(kBQF + st), c * 64, m0, h, b);
+        const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
+        if (C::kSplitStage) {
+          // other panels first (free early), then the panels of this CTA's chunk
+          const int po = 2 * (1 - split);
+          if (!warp_wait(BAR(kBQE + 1), (u & 1) ^ 1, abort_flag, a.status)) break;
+          if (elect_one()) {
+            mbar_arrive_expect_tx(BAR(kBQF + 1), (C::kQBytes + C::kOBytes) / 2);
+            for (int c = po; c < po + 2; ++c) {
+              tma_load_4d(qs + c * C::kQPanel, &tm_q, BAR(kBQF + 1), c * 64, m0, h, b);
+              tma_load_4d(qs + C::kQBytes + c * C::kQPanel, &tm_do, BAR(kBQF + 1), c * 64, m0, h, b);
+            }
+          }
+          __syncwarp();
+          const int pw = 2 * split;
+          if (!warp_wait(BAR(kBQE), (u & 1) ^ 1, abort_flag, a.status)) break;
+          if (elect_one()) {
+            mbar_arrive_expect_tx(BAR(kBQF), (C::kQBytes + C::kOBytes) / 2);
+            for (int c = pw; c < pw + 2; ++c) {
+              tma_load_4d(qs + c * C::kQPanel, &tm_q, BAR(kBQF), c * 64, m0, h, b);
+              tma_load_4d(qs + C::kQBytes + c * C::kQPanel, &tm_do, BAR(kBQF), c * 64, m0, h, b);
+            }
+          }
+          __syncwarp();
+        } else {
+          if (!warp_wait(BAR(kBQE + st), (u & 1) ^ 1, abort_flag, a.status)) break;
+          if (elect_one()) {
+            mbar_arrive_expect_tx(BAR(kBQF + st), C::kQBytes + C::kOBytes);
+            for (int c = 0; c < DQK / 64; ++c)
+              tma_load_4d(qs + c * C::kQPanel, &tm_q, BAR(kBQF + st), c * 64, m0, h, b);
+            for (int c = 0; c < DV / 64; ++c)
+              tma_load_4d(qs + C::kQBytes + c * C::kQPanel, &tm_do, BAR(kBQF + st), c * 64, m0, h, b);
+          }
+          __syncwarp();
         }
         // LSE (in log2 units) and Delta of the 64 queries; +inf / 0 past Sq
         float* ls = lbuf + st * 2 * BM;
@@ -282,8 +315,10 @@ __global__ void __launch_bounds__(448, 1)
       }
       if (lane == 0 && *abort_flag) {
         mbar_wait_limited(BAR(kBKV), 0);
-        for (int it = max(0, n_iter - 2); it < n_iter; ++it)
+        for (int it = max(0, n_iter - C::kStages); it < n_iter; ++it) {
           mbar_wait_limited(BAR(kBQF + it % C::kStages), (it / C::kStages) & 1);
+          if (C::kSplitStage) mbar_wait_limited(BAR(kBQF + 1), it & 1);
+        }
       }
     }
   } else if (warp == 1) {
@@ -301,41 +336,54 @@ __global__ void __launch_bounds__(448, 1)
       const uint64_t kd = sw128_desc(kbase, 16, 1024), vd = sw128_desc(vbase, 16, 1024);
       const uint64_t kwd = sw128_desc(kbase + (qw0 / 64) * C::kKPanel, C::kKPanel, 1024);
       bool ok = warp_wait(BAR(kBKV), 0, abort_flag, a.status);
-      // S^T(j) and dP^T(j) into TMEM buffer j & 1
-      auto issue_sdp = [&](int j) -> bool {
+      // S^T(j) and dP^T(j) into TMEM buffer j & 1.  part: 0 all panels, 1 the panels
+      // outside this CTA's chunk (issued first, accumulate from zero), 2 the rest.
+      auto issue_sdp = [&](int j, int part) -> bool {
         const int st = j % C::kStages, u = j / C::kStages, bj = j & 1;
-        if (!warp_wait(BAR(kBQF + st), u & 1, abort_flag, a.status)) return false;
+        const int fslot = part == 1 ? kBQF + 1 : kBQF + st;
+        if (!warp_wait(BAR(fslot), u & 1, abort_flag, a.status)) return false;
         // the dQ^T of step j-2 lives in this buffer until it has been drained
-        if (j >= 2 && !warp_wait(BAR(kBDQE + bj), ((j - 2) >> 1) & 1, abort_flag, a.status))
+        if (part != 2 && j >= 2 &&
+            !warp_wait(BAR(kBDQE + bj), ((j - 2) >> 1) & 1, abort_flag, a.status))
           return false;
         tc_fence_after();
         const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
         const uint64_t qd = sw128_desc(qs, 16, 1024), od = sw128_desc(qs + C::kQBytes, 16, 1024);
+        // panel range [p0, p1) of the contraction issued now
+        const int p0 = part == 0 ? 0 : (part == 1 ? 2 * (1 - split) : 2 * split);
+        const int pn = part == 0 ? DQK / 64 : 2;
         if (elect_one()) {
+          for (int pi = 0; pi < pn; ++pi) {
+            const int p = p0 + pi;
 #pragma unroll
-          for (int kk = 0; kk < DQK / 16; ++kk) {
-            const uint32_t ka = (kk >> 2) * C::kKPanel + (kk & 3) * 32;
-            const uint32_t qb = (kk >> 2) * C::kQPanel + (kk & 3) * 32;
-            umma_ss(tmem + C::kColS + 64 * bj, kd + (ka >> 4), qd + (qb >> 4), idesc_s,
-                    kk > 0 ? 1u : 0u);
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const uint32_t ka = p * C::kKPanel + k4 * 32, qb = p * C::kQPanel + k4 * 32;
+              const uint32_t acc = (part != 2 && pi == 0 && k4 == 0) ? 0u : 1u;
+              umma_ss(tmem + C::kColS + 64 * bj, kd + (ka >> 4), qd + (qb >> 4), idesc_s, acc);
+            }
           }
+          const int pvn = part == 0 ? DV / 64 : 2;
+          for (int pi = 0; pi < pvn; ++pi) {
+            const int p = p0 + pi;
 #pragma unroll
-          for (int kk = 0; kk < DV / 16; ++kk) {
-            const uint32_t va = (kk >> 2) * C::kKPanel + (kk & 3) * 32;
-            const uint32_t ob = (kk >> 2) * C::kQPanel + (kk & 3) * 32;
-            umma_ss(tmem + C::kColDP + 64 * bj, vd + (va >> 4), od + (ob >> 4), idesc_s,
-                    kk > 0 ? 1u : 0u);
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const uint32_t va = p * C::kKPanel + k4 * 32, ob = p * C::kQPanel + k4 * 32;
+              const uint32_t acc = (part != 2 && pi == 0 && k4 == 0) ? 0u : 1u;
+              umma_ss(tmem + C::kColDP + 64 * bj, vd + (va >> 4), od + (ob >> 4), idesc_s, acc);
+            }
           }
-          umma_commit(BAR(kBSF + bj));
+          if (part != 1) umma_commit(BAR(kBSF + bj));
+          if (part == 2) umma_commit(BAR(kBQE + 1));  // other panels free once this is done
         }
         __syncwarp();
         return true;
       };
-      if (ok) ok = issue_sdp(0);
+      if (ok) ok = C::kSplitStage ? (issue_sdp(0, 1) && issue_sdp(0, 2)) : issue_sdp(0, 0);
       for (int it = 0; ok && it < n_iter; ++it) {
         const int st = it % C::kStages, bi = it & 1;
-        // with two Q/dO stages the next S^T / dP^T overlap this step's elementwise work
-        if (C::kStages >= 2 && it + 1 < n_iter && !issue_sdp(it + 1)) break;
+        // the next S^T / dP^T (with a split stage: its first half) overlap this step's
+        // elementwise work
+        if (it + 1 < n_iter && !issue_sdp(it + 1, C::kSplitStage ? 1 : 0)) break;
         if (!warp_wait(BAR(kBPF + bi), (it >> 1) & 1, abort_flag, a.status)) break;
         tc_fence_after();
         const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
@@ -361,7 +409,7 @@ __global__ void __launch_bounds__(448, 1)
           umma_commit(BAR(kBDQF + bi));
         }
         __syncwarp();
-        if (C::kStages == 1 && it + 1 < n_iter && !issue_sdp(it + 1)) break;
+        if (C::kSplitStage && it + 1 < n_iter && !issue_sdp(it + 1, 2)) break;
       }
       if (elect_one()) umma_commit(BAR(kBFin));
       __syncwarp();
@@ -427,19 +475,43 @@ __global__ void __launch_bounds__(448, 1)
       }
       tmem_wait_ld();
       uint32_t pk[16], dk[16];
+      const float4* ls4 = reinterpret_cast<const float4*>(ls);         // lse2[q] (log2 units)
+      const float4* dl4 = reinterpret_cast<const float4*>(ls + BM);    // Delta[q]
+      const float sc = a.scale_log2;
+      if (!partial) {
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        float pv[2], dv2[2];
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 l = ls4[e4], d = dl4[e4];
+          const float lv[4] = {l.x, l.y, l.z, l.w}, dv4[4] = {d.x, d.y, d.z, d.w};
+          float pv[4], dsv[4];
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const int q = 2 * e + t;
-          const float sv = __uint_as_float(s_u[q]);
-          const float p = ((cm >> q) & 1u) ? ex2(fmaf(sv, a.scale_log2, -ls[q])) : 0.f;
-          pv[t] = p;
-          dv2[t] = p * (__uint_as_float(p_u[q]) - ls[BM + q]);
+          for (int t = 0; t < 4; ++t) {
+            const int q = 4 * e4 + t;
+            pv[t] = ex2(fmaf(__uint_as_float(s_u[q]), sc, -lv[t]));
+            dsv[t] = pv[t] * (__uint_as_float(p_u[q]) - dv4[t]);
+          }
+          pk[2 * e4] = pack_bf16x2(pv[0], pv[1]);
+          pk[2 * e4 + 1] = pack_bf16x2(pv[2], pv[3]);
+          dk[2 * e4] = pack_bf16x2(dsv[0], dsv[1]);
+          dk[2 * e4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
         }
-        pk[e] = pack_bf16x2(pv[0], pv[1]);
-        dk[e] = pack_bf16x2(dv2[0], dv2[1]);
+      } else {
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 l = ls4[e4], d = dl4[e4];
+          const float lv[4] = {l.x, l.y, l.z, l.w}, dv4[4] = {d.x, d.y, d.z, d.w};
+          float pv[4], dsv[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int q = 4 * e4 + t;
+            pv[t] = ((cm >> q) & 1u) ? ex2(fmaf(__uint_as_float(s_u[q]), sc, -lv[t])) : 0.f;
+            dsv[t] = pv[t] * (__uint_as_float(p_u[q]) - dv4[t]);
+          }
+          pk[2 * e4] = pack_bf16x2(pv[0], pv[1]);
+          pk[2 * e4 + 1] = pack_bf16x2(pv[2], pv[3]);
+          dk[2 * e4] = pack_bf16x2(dsv[0], dsv[1]);
+          dk[2 * e4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
+        }
       }
       tmem_st16(tl + cs, pk);
       tmem_st16(tl + cd, dk);
