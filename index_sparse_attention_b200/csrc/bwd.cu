@@ -372,8 +372,8 @@ __global__ void __launch_bounds__(448, 1)
               umma_ss(tmem + C::kColDP + 64 * bj, vd + (va >> 4), od + (ob >> 4), idesc_s, acc);
             }
           }
+          if (part == 1) umma_commit(BAR(kBQE + 1));  // other panels free once these are done
           if (part != 1) umma_commit(BAR(kBSF + bj));
-          if (part == 2) umma_commit(BAR(kBQE + 1));  // other panels free once this is done
         }
         __syncwarp();
         return true;
