@@ -38,6 +38,22 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 L2_BYTES = 126 * 1024 * 1024
 
 
+def max_over_ranks(x, device):
+    """Max of a per-rank float over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(flop_per_rank_step, ms_per_step_max, world):
+    """Whole-job TFLOP/s: the work of every rank divided by the slowest rank's step time."""
+    return world * flop_per_rank_step / (ms_per_step_max * 1e-3) / 1e12
+
+
 def tile_flops(w):
     """(forward, backward) tensor-core FLOP of one active 128x128 tile for one query head."""
     return 2 * 128 * 128 * (w.Dqk + w.Dv), 2 * 128 * 128 * (3 * w.Dqk + 2 * w.Dv)
@@ -84,7 +100,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", str(self.gpu), "-lms", "100"], stdout=subprocess.PIPE,
+                 "-i", str(self.gpu), "-lms", "20"], stdout=subprocess.PIPE,
                 stderr=subprocess.DEVNULL, text=True)
             threading.Thread(target=self._read, daemon=True).start()
             time.sleep(0.3)
@@ -208,7 +224,7 @@ def run_reference(args):
     w = get_workload(args)
     inp = I.make_inputs(w)
     s = OracleSampler(w, inp)
-    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    per_step = args.ref_seconds or max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         s.run_for(per_step)
     flop, sec, tiles = 0, 0.0, 0
@@ -344,11 +360,7 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
     per_kernel = {
         "fwd": float(np.mean([r[0].elapsed_time(r[1]) for r in evs])),
         "bwd_pre": float(np.mean([r[2].elapsed_time(r[3]) for r in evs])),
@@ -356,7 +368,7 @@ def run_gpu(args):
         "bwd_post": float(np.mean([r[4].elapsed_time(r[5]) for r in evs])),
     }
     ms_step = ms / args.steps
-    value = world * flop_step / (ms_step * 1e-3) / 1e12
+    value = whole_job_rate(flop_step, ms_step, world)
 
     # end to end through the public API with host buffers: H2D of the inputs, the whole
     # path, D2H of every output, per step
@@ -377,12 +389,8 @@ def run_gpu(args):
             dst.copy_(src, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1) / e_steps
-    if world > 1:
-        t = torch.tensor([e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
-    e2e_value = world * flop_step / (e_ms * 1e-3) / 1e12
+    e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps, dev)
+    e2e_value = whole_job_rate(flop_step, e_ms, world)
 
     peaks, peak_src = load_peaks()
     clocks = clk.summary()
@@ -429,12 +437,14 @@ def run_gpu(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(I.WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=0.0,
+                    help="CPU seconds per reference step (default: the run ends in ~2.5 min)")
     ap.add_argument("--seq", type=int, default=0,
                     help="override Sq = Sk (smaller profiling captures of the same kernels)")
     args = ap.parse_args()
