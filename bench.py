@@ -66,9 +66,17 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def bwd_kernel_name(w):
+    """The backward main kernel that the library launches for this workload's head dims."""
+    if (w.Dqk, w.Dv) == (256, 256):
+        return "sparse_bwd_pair_kernel"
+    inst = {(64, 64): "128,128,1", (128, 128): "128,128,1", (192, 128): "192,128,2"}
+    return f"sparse_bwd_kernel<{inst.get((w.Dqk, w.Dv), '?')}>"
+
+
 def bwd_source_sha():
     h = hashlib.sha256()
-    for f in ("bwd.cu", "sa_device.cuh"):
+    for f in ("bwd.cu", "bwd_pair.cu", "sa_device.cuh"):
         h.update(open(os.path.join(ROOT, "index_sparse_attention_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -407,7 +415,7 @@ def run_gpu(args):
             "pct_basis": f"bf16_tflops_sustained {peak:.1f} TFLOP/s ({peak_src})",
             "flop_per_step": flop_step, "kernel_ms": per_kernel,
             "roofline": {
-                "kernel": "sparse_bwd_kernel", "bound": "tensor", "achieved": achieved,
+                "kernel": bwd_kernel_name(w), "bound": "tensor", "achieved": achieved,
                 "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_kind": f"bf16_tflops_sustained ({'of measured' if peak_src == 'measured' else 'of fallback'}); burst {peak_burst:.1f}",
                 "traffic": profiled_traffic(w.name),

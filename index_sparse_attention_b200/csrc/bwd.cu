@@ -24,8 +24,9 @@
 //   dQ^T = K^T dS^T   (M=128 head-dim window, N=64) both MN-major    [SS]
 //   the same warps drain dQ^T from TMEM and add it (fp32 reductions, coalesced along
 //   the head dim) into the dQ accumulator.
-// When Dqk + Dv does not leave room in the 512 TMEM columns (192/128 and 256/256),
-// the head dim of dK/dV/dQ is split over two CTAs, each recomputing S^T and dP^T.
+// When Dqk + Dv does not leave room in the 512 TMEM columns (192/128), the head dim of
+// dK/dV/dQ is split over two CTAs, each recomputing S^T and dP^T.  Head dims 256/256
+// run on a 2-CTA cluster that splits the work instead (bwd_pair.cu).
 // Every mbarrier wait is bounded (see sa_device.cuh).
 #include "sa_device.cuh"
 #include "sa_kernels.h"
@@ -100,23 +101,17 @@ struct BwdCfg {
   static constexpr int kVBytes = 128 * DV * 2;
   static constexpr int kQBytes = kBM * DQK * 2;
   static constexpr int kOBytes = kBM * DV * 2;
-  // Q/dO stages: three at D=128, two at (192,128); one at (256,256), split in two
-  // halves with their own barriers: the panels this CTA's dK/dV chunk needs (held until
-  // dK/dV are done) and the other panels (free once S^T/dP^T are done, so the next
-  // step's copy of them overlaps the elementwise work)
-  static constexpr int kStages = (DQK + DV >= 512) ? 1 : (DQK == 128 ? 3 : 2);
-  static constexpr bool kSplitStage = kStages == 1;
+  // Q/dO stages: three at D=128, two at (192,128)
+  static constexpr int kStages = DQK == 128 ? 3 : 2;
   static constexpr int kDSBytes = 128 * kBM * 2;     // dS^T [128 keys][64 q] bf16 (16 KB)
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kKOff + kKBytes;
   static constexpr int kQOff = kVOff + kVBytes;                    // per stage: Q then dO
   static constexpr int kStageBytes = kQBytes + kOBytes;
   static constexpr int kDSOff = kQOff + kStages * kStageBytes;     // two dS^T buffers
-  // fp32 dQ staging tile [2 panels][32 q][64 d]: a buffer of its own when shared memory
-  // allows (two Q/dO stages), otherwise the step's dS^T buffer once dQ^T has read it
-  static constexpr bool kOwnStage = kStages >= 2;
+  // fp32 dQ staging tile [2 panels][32 q][64 d]
   static constexpr int kDQOff = kDSOff + 2 * kDSBytes;
-  static constexpr int kLOff = kDQOff + (kOwnStage ? 128 * 32 * 4 : 0);  // lse2[64], delta[64]
+  static constexpr int kLOff = kDQOff + 128 * 32 * 4;               // per stage: lse2[64], delta[64]
   static constexpr int kBMOff = kLOff + kStages * 2 * kBM * 4;     // per stage: bitmap words [64][4]
   static constexpr int kBarOff = kBMOff + kStages * kBM * 4 * 4;
   static constexpr int kSmem = kBarOff + 256 + 1024;
@@ -130,15 +125,15 @@ struct BwdCfg {
   static constexpr uint32_t kColDK = 256;
   static constexpr uint32_t kColDV = kColDK + kDKMax;
   static constexpr uint32_t kTmemCols = 512;
+  static_assert(DQK + DV < 512, "head dims 256/256 run in the 2-CTA kernel");
   static_assert(kColDV + kDVMax <= kTmemCols, "tensor memory budget");
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
 
 enum : int {
-  kBKV = 0, kBQF = 1, kBQE = 4, kBLF = 7, kBSF = 10, kBPF = 12, kBDQF = 14, kBDQE = 16, kBDSE = 18,
-  kBFin = 20, kBDrainB = 21, kNumBarsB = 22
+  kBKV = 0, kBQF = 1, kBQE = 4, kBLF = 7, kBSF = 10, kBPF = 12, kBDQF = 14, kBDQE = 16,
+  kBFin = 18, kBDrainB = 19, kNumBarsB = 20
 };
-// With a split stage, QF/QE slot 0 guards the own panels and slot 1 the other panels.
 
 // Warp roles: 0 producer, 1 MMA, 2-9 elementwise (one key row and 32 of the 64 query
 // columns per thread: warps 2-5 columns 0-31, warps 6-9 columns 32-63), 10-13 dQ drain
@@ -180,13 +175,11 @@ __global__ void __launch_bounds__(448, 1)
   int kc0, kcn, vc0, vcn, qw0;  // qw0: first head-dim row of the 128-wide dQ^T window
   if (NSPLIT == 1) {
     kc0 = 0; kcn = DQK; vc0 = 0; vcn = DV; qw0 = 0;
-  } else if (DQK == 192) {
+  } else {  // (192, 128): dK 128 + 64 columns, dV 64 + 64
+    static_assert(NSPLIT == 1 || DQK == 192, "head-dim split is built for (192, 128)");
     kc0 = split == 0 ? 0 : 128; kcn = split == 0 ? 128 : 64;
     vc0 = split * 64; vcn = 64;
     qw0 = split == 0 ? 0 : 64;
-  } else {
-    kc0 = split * (DQK / 2); kcn = DQK / 2; vc0 = split * (DV / 2); vcn = DV / 2;
-    qw0 = split * (DQK / 2);
   }
   const int dqk_real = a.Dqk, dv_real = a.Dv;  // 64 when run through the 128 instance
 
@@ -202,7 +195,6 @@ __global__ void __launch_bounds__(448, 1)
       mbar_init(BAR(kBPF + s), 256);
       mbar_init(BAR(kBDQF + s), 1);
       mbar_init(BAR(kBDQE + s), 128);
-      mbar_init(BAR(kBDSE + s), 128);
     }
     mbar_init(BAR(kBFin), 1);
     mbar_init(BAR(kBDrainB), 1);
@@ -254,39 +246,15 @@ __global__ void __launch_bounds__(448, 1)
         m0 = __shfl_sync(0xFFFFFFFFu, m0, 0);  // warp-uniform TMA coordinate
         const int st = it % C::kStages, u = it / C::kStages;
         const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
-        if (C::kSplitStage) {
-          // other panels first (free early), then the panels of this CTA's chunk
-          const int po = 2 * (1 - split);
-          if (!warp_wait(BAR(kBQE + 1), (u & 1) ^ 1, abort_flag, a.status)) break;
-          if (elect_one()) {
-            mbar_arrive_expect_tx(BAR(kBQF + 1), (C::kQBytes + C::kOBytes) / 2);
-            for (int c = po; c < po + 2; ++c) {
-              tma_load_4d(qs + c * C::kQPanel, &tm_q, BAR(kBQF + 1), c * 64, m0, h, b);
-              tma_load_4d(qs + C::kQBytes + c * C::kQPanel, &tm_do, BAR(kBQF + 1), c * 64, m0, h, b);
-            }
-          }
-          __syncwarp();
-          const int pw = 2 * split;
-          if (!warp_wait(BAR(kBQE), (u & 1) ^ 1, abort_flag, a.status)) break;
-          if (elect_one()) {
-            mbar_arrive_expect_tx(BAR(kBQF), (C::kQBytes + C::kOBytes) / 2);
-            for (int c = pw; c < pw + 2; ++c) {
-              tma_load_4d(qs + c * C::kQPanel, &tm_q, BAR(kBQF), c * 64, m0, h, b);
-              tma_load_4d(qs + C::kQBytes + c * C::kQPanel, &tm_do, BAR(kBQF), c * 64, m0, h, b);
-            }
-          }
-          __syncwarp();
-        } else {
-          if (!warp_wait(BAR(kBQE + st), (u & 1) ^ 1, abort_flag, a.status)) break;
-          if (elect_one()) {
-            mbar_arrive_expect_tx(BAR(kBQF + st), C::kQBytes + C::kOBytes);
-            for (int c = 0; c < DQK / 64; ++c)
-              tma_load_4d(qs + c * C::kQPanel, &tm_q, BAR(kBQF + st), c * 64, m0, h, b);
-            for (int c = 0; c < DV / 64; ++c)
-              tma_load_4d(qs + C::kQBytes + c * C::kQPanel, &tm_do, BAR(kBQF + st), c * 64, m0, h, b);
-          }
-          __syncwarp();
+        if (!warp_wait(BAR(kBQE + st), (u & 1) ^ 1, abort_flag, a.status)) break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(BAR(kBQF + st), C::kQBytes + C::kOBytes);
+          for (int c = 0; c < DQK / 64; ++c)
+            tma_load_4d(qs + c * C::kQPanel, &tm_q, BAR(kBQF + st), c * 64, m0, h, b);
+          for (int c = 0; c < DV / 64; ++c)
+            tma_load_4d(qs + C::kQBytes + c * C::kQPanel, &tm_do, BAR(kBQF + st), c * 64, m0, h, b);
         }
+        __syncwarp();
         // LSE (in log2 units) and Delta of the 64 queries; +inf / 0 past Sq
         float* ls = lbuf + st * 2 * BM;
 #pragma unroll
@@ -315,10 +283,8 @@ __global__ void __launch_bounds__(448, 1)
       }
       if (lane == 0 && *abort_flag) {
         mbar_wait_limited(BAR(kBKV), 0);
-        for (int it = max(0, n_iter - C::kStages); it < n_iter; ++it) {
+        for (int it = max(0, n_iter - C::kStages); it < n_iter; ++it)
           mbar_wait_limited(BAR(kBQF + it % C::kStages), (it / C::kStages) & 1);
-          if (C::kSplitStage) mbar_wait_limited(BAR(kBQF + 1), it & 1);
-        }
       }
     }
   } else if (warp == 1) {
@@ -336,54 +302,43 @@ __global__ void __launch_bounds__(448, 1)
       const uint64_t kd = sw128_desc(kbase, 16, 1024), vd = sw128_desc(vbase, 16, 1024);
       const uint64_t kwd = sw128_desc(kbase + (qw0 / 64) * C::kKPanel, C::kKPanel, 1024);
       bool ok = warp_wait(BAR(kBKV), 0, abort_flag, a.status);
-      // S^T(j) and dP^T(j) into TMEM buffer j & 1.  part: 0 all panels, 1 the panels
-      // outside this CTA's chunk (issued first, accumulate from zero), 2 the rest.
-      auto issue_sdp = [&](int j, int part) -> bool {
+      // S^T(j) and dP^T(j) into TMEM buffer j & 1
+      auto issue_sdp = [&](int j) -> bool {
         const int st = j % C::kStages, u = j / C::kStages, bj = j & 1;
-        const int fslot = part == 1 ? kBQF + 1 : kBQF + st;
-        if (!warp_wait(BAR(fslot), u & 1, abort_flag, a.status)) return false;
+        if (!warp_wait(BAR(kBQF + st), u & 1, abort_flag, a.status)) return false;
         // the dQ^T of step j-2 lives in this buffer until it has been drained
-        if (part != 2 && j >= 2 &&
-            !warp_wait(BAR(kBDQE + bj), ((j - 2) >> 1) & 1, abort_flag, a.status))
+        if (j >= 2 && !warp_wait(BAR(kBDQE + bj), ((j - 2) >> 1) & 1, abort_flag, a.status))
           return false;
         tc_fence_after();
         const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
         const uint64_t qd = sw128_desc(qs, 16, 1024), od = sw128_desc(qs + C::kQBytes, 16, 1024);
-        // panel range [p0, p1) of the contraction issued now
-        const int p0 = part == 0 ? 0 : (part == 1 ? 2 * (1 - split) : 2 * split);
-        const int pn = part == 0 ? DQK / 64 : 2;
         if (elect_one()) {
-          for (int pi = 0; pi < pn; ++pi) {
-            const int p = p0 + pi;
+          for (int p = 0; p < DQK / 64; ++p) {
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const uint32_t ka = p * C::kKPanel + k4 * 32, qb = p * C::kQPanel + k4 * 32;
-              const uint32_t acc = (part != 2 && pi == 0 && k4 == 0) ? 0u : 1u;
-              umma_ss(tmem + C::kColS + 64 * bj, kd + (ka >> 4), qd + (qb >> 4), idesc_s, acc);
+              umma_ss(tmem + C::kColS + 64 * bj, kd + (ka >> 4), qd + (qb >> 4), idesc_s,
+                      (p > 0 || k4 > 0) ? 1u : 0u);
             }
           }
-          const int pvn = part == 0 ? DV / 64 : 2;
-          for (int pi = 0; pi < pvn; ++pi) {
-            const int p = p0 + pi;
+          for (int p = 0; p < DV / 64; ++p) {
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const uint32_t va = p * C::kKPanel + k4 * 32, ob = p * C::kQPanel + k4 * 32;
-              const uint32_t acc = (part != 2 && pi == 0 && k4 == 0) ? 0u : 1u;
-              umma_ss(tmem + C::kColDP + 64 * bj, vd + (va >> 4), od + (ob >> 4), idesc_s, acc);
+              umma_ss(tmem + C::kColDP + 64 * bj, vd + (va >> 4), od + (ob >> 4), idesc_s,
+                      (p > 0 || k4 > 0) ? 1u : 0u);
             }
           }
-          if (part == 1) umma_commit(BAR(kBQE + 1));  // other panels free once these are done
-          if (part != 1) umma_commit(BAR(kBSF + bj));
+          umma_commit(BAR(kBSF + bj));
         }
         __syncwarp();
         return true;
       };
-      if (ok) ok = C::kSplitStage ? (issue_sdp(0, 1) && issue_sdp(0, 2)) : issue_sdp(0, 0);
+      if (ok) ok = issue_sdp(0);
       for (int it = 0; ok && it < n_iter; ++it) {
         const int st = it % C::kStages, bi = it & 1;
-        // the next S^T / dP^T (with a split stage: its first half) overlap this step's
-        // elementwise work
-        if (it + 1 < n_iter && !issue_sdp(it + 1, C::kSplitStage ? 1 : 0)) break;
+        // the next S^T / dP^T overlap this step's elementwise work
+        if (it + 1 < n_iter && !issue_sdp(it + 1)) break;
         if (!warp_wait(BAR(kBPF + bi), (it >> 1) & 1, abort_flag, a.status)) break;
         tc_fence_after();
         const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
@@ -409,7 +364,6 @@ __global__ void __launch_bounds__(448, 1)
           umma_commit(BAR(kBDQF + bi));
         }
         __syncwarp();
-        if (C::kSplitStage && it + 1 < n_iter && !issue_sdp(it + 1, 2)) break;
       }
       if (elect_one()) umma_commit(BAR(kBFin));
       __syncwarp();
@@ -432,14 +386,9 @@ __global__ void __launch_bounds__(448, 1)
       const int st = it % C::kStages, u = it / C::kStages, bi = it & 1;
       bool w_ok = mbar_wait(BAR(kBLF + st), u & 1, abort_flag, a.status);
       w_ok = w_ok && mbar_wait(BAR(kBSF + bi), (it >> 1) & 1, abort_flag, a.status);
-      // the dS^T buffer is free once dQ^T of step it-2 has read it (and, without a
-      // staging buffer of its own, once the drain of step it-2 has used it)
-      if (it >= 2) {
-        if (C::kOwnStage)
-          w_ok = w_ok && mbar_wait(BAR(kBDQF + bi), ((it - 2) >> 1) & 1, abort_flag, a.status);
-        else
-          w_ok = w_ok && mbar_wait(BAR(kBDSE + bi), ((it - 2) >> 1) & 1, abort_flag, a.status);
-      }
+      // the dS^T buffer is free once dQ^T of step it-2 has read it
+      if (it >= 2)
+        w_ok = w_ok && mbar_wait(BAR(kBDQF + bi), ((it - 2) >> 1) & 1, abort_flag, a.status);
       if (!__all_sync(0xFFFFFFFFu, w_ok)) {
         ok = false;
         break;
@@ -590,8 +539,9 @@ __global__ void __launch_bounds__(448, 1)
       bool partial;
       decode(it, h, m0, partial);
       const int bi = it & 1;
+      // the four drain warps leave together (they share named barrier 1 below)
       const bool w_ok = mbar_wait(BAR(kBDQF + bi), (it >> 1) & 1, abort_flag, a.status);
-      if (!__all_sync(0xFFFFFFFFu, w_ok)) {
+      if (!named_bar_and(1, 128, w_ok)) {
         ok = false;
         break;
       }
@@ -602,17 +552,14 @@ __global__ void __launch_bounds__(448, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(BAR(kBDQE + bi));
-      const int soff = C::kOwnStage ? C::kDQOff : C::kDSOff + bi * C::kDSBytes;
-      float* stage = reinterpret_cast<float*>(smem + soff);
-      const uint32_t stage_s = sbase + soff;
+      float* stage = reinterpret_cast<float*>(smem + C::kDQOff);
+      const uint32_t stage_s = sbase + C::kDQOff;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        if (half == 1 || C::kOwnStage) {
-          // the previous reduce (this step's first half, or the last step's second
-          // half in the own staging buffer) must have read the tile
-          if (dtid == 0) bulk_wait_group_read0();
-          named_bar_sync(1, 128);
-        }
+        // the previous reduce (this step's first half, or the last step's second half)
+        // must have read the staging tile
+        if (dtid == 0) bulk_wait_group_read0();
+        named_bar_sync(1, 128);
 #pragma unroll
         for (int q = 0; q < 32; ++q) stage[(p * 32 + q) * 64 + (r & 63)] = __uint_as_float(q_u[32 * half + q]);
         fence_proxy_async_smem();
@@ -622,11 +569,6 @@ __global__ void __launch_bounds__(448, 1)
           if (own1) tma_reduce_add_4d(&tm_dq, stage_s + 32 * 64 * 4, qw0 + 64, m0 + 32 * half, h, b);
           bulk_commit_group();
         }
-      }
-      if (!C::kOwnStage) {
-        if (dtid == 0) bulk_wait_group_read0();
-        named_bar_sync(1, 128);
-        mbar_arrive(BAR(kBDSE + bi));
       }
     }
     if (dtid == 0) bulk_wait_group0();  // every reduce has landed before the CTA ends
@@ -701,7 +643,7 @@ int launch_bwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
   else if (a.Dqk == 192 && a.Dv == 128)
     rc = launch_bwd_main<192, 128, 2>(a, m, st);
   else if (a.Dqk == 256 && a.Dv == 256)
-    rc = launch_bwd_main<256, 256, 2>(a, m, st);
+    rc = launch_bwd_pair(a, m, st);
   else
     return SA_ERR_UNSUPPORTED;
   if (rc) return rc;

@@ -52,5 +52,6 @@ inline int check_launch(const char* what) { return cuda_error(cudaGetLastError()
 
 int launch_fwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st);
 int launch_bwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st);
+int launch_bwd_pair(const AttnArgs& a, const TensorMaps& m, cudaStream_t st);
 
 }  // namespace sa
