@@ -7,72 +7,108 @@
 // MagiAttention PR #331 ("CSR Tile Mapping").
 //
 // Why a pair.  With 256-wide heads the fp32 dK and dV accumulators of a 128-key tile
-// need 512 TMEM columns, everything the SM has, so each CTA can hold only a 128-wide
-// head-dim half of them.  Two CTAs that each recompute S^T and dP^T for their half
-// would do those contractions twice and would leave room for only one Q/dO stage.
-// Here the two CTAs of a cluster split the work instead of duplicating it:
-//   rank 0: S^T = K Q^T (all of K resident), P^T = exp2(S^T scale log2e - LSE log2e)
-//           with the element mask, P^T -> own TMEM and (bf16, distributed shared
-//           memory) rank 1's exchange tile; dV[:, 0:128] += P^T dO, dK[:, 0:128] +=
-//           dS^T Q, dQ^T[0:128] = K^T dS^T with dS^T received from rank 1.
-//   rank 1: dP^T = V dO^T (all of V resident), dS^T = P^T (dP^T - Delta) with P^T from
-//           rank 0, dS^T -> own TMEM, own shared memory and rank 0's exchange tile;
-//           dV[:, 128:256] += P^T dO, dK[:, 128:256] += dS^T Q,
-//           dQ^T[128:256] = K^T dS^T.
-// Each rank does the same tensor-core work per step, keeps two Q/dO stages, and the
-// exchange tiles are double-buffered, so the next step's S^T / dP^T overlap the
-// current step's elementwise work on both ranks.
+// need 512 TMEM columns, everything one SM has.  Two CTAs that each recompute S^T and
+// dP^T for a head-dim half would do those contractions twice and have room for only
+// one Q/dO stage.  Here the two CTAs of a cluster split the work by role:
+//   rank 0 holds K and stages of Q: S^T = K Q^T, P^T = exp2(S^T scale log2e - LSE log2e)
+//           with the element mask (bf16, into an exchange tile), dK += dS^T Q (all 256
+//           columns), dQ^T[0:128] = K[:, 0:128]^T dS^T;
+//   rank 1 holds V in TMEM, K[:, 128:256] and stages of dO: dP^T = V dO^T (V as the
+//           TMEM operand), dS^T = P^T (dP^T - Delta) (bf16, into an exchange tile),
+//           dV += P^T dO (all 256 columns), dQ^T[128:256] = K[:, 128:256]^T dS^T into
+//           the TMEM buffer the elementwise warps have just read dP^T from.
+// Each rank issues about the same tensor-core work per 64-query step, and a stage
+// holds only Q or only dO, so three stages fit on each rank.
 //
-// Per 64-query step the exchanges are single 16 KB bulk copies (cp.async.bulk,
-// shared::cta -> shared::cluster, no multicast) of a whole exchange tile, completing as
-// transaction bytes on the receiving CTA's barrier XF[b].  The receiver arms XF[b] itself
-// (one local arrival expecting the 16 KB) for step it+2 once it has consumed step it, so
-// a sender issues nothing but the copy:
-//   rank 0 stages P^T(it) in its own tile b and copies it into rank 1's tile b;
-//   rank 1 overwrites its tile b with dS^T(it) (after dV has read P^T there) and copies
-//   it into rank 0's tile b (rank 0's copy of P^T has landed by then).
-// A copy signals only its receiver, so the receiver tells the sender when a tile may be
-// reused, with a relaxed remote arrival (it carries no data: the readers have finished):
-//   XS[b] on rank 1: dS^T(it) has landed in rank 0 (rank 1's dQ drain may stage in tile b);
-//   XE[b] on rank 0: rank 1's tile b is free (its dQ drain used it as staging last).
-// A release at cluster scope is avoided throughout: it would stall the signalling thread
-// on all of its earlier memory operations.
+// Exchanges.  Per step, P^T (rank 0 -> 1) and dS^T (rank 1 -> 0) cross as one 16 KB
+// bulk copy each (cp.async.bulk shared::cta -> shared::cluster, no multicast) that
+// completes its bytes on the receiver's barrier XF; the receiver arms XF itself (one
+// local arrival expecting 16 KB) for the step that will use the tile next, so a sender
+// issues nothing but the copy.  Each rank has four exchange tiles, step it using tile
+// it % 4: on rank 0 it stages P^T, then receives dS^T, then stages the dQ drain; on
+// rank 1 it receives P^T and is overwritten by dS^T once dV has read it (rank 1 stages
+// its dQ drain in a buffer of its own).  A copy signals only its receiver, so the
+// receivers report back with relaxed remote arrivals, which order no data (the readers
+// have finished when they are sent):
+//   XS[b] on rank 1: its dS^T copy from tile b has landed in rank 0;
+//   XE[b] on rank 0: rank 1's tile b is free again (dQ^T has read it, and XS[b] came).
+// A release at cluster scope is never used on the step path: it stalls the signalling
+// thread on all of its earlier memory operations (about a microsecond on B200).
+//
+// Issue order.  The MMA warp of each rank does not follow a fixed order: it polls the
+// barriers of its MMA streams and issues whichever is ready (rank 0: dK/dQ^T of the
+// oldest step, else the next S^T; rank 1: dV, else dQ^T, else the next dP^T), and keeps
+// S^T / dP^T at most a step or two ahead, because the tensor pipe runs in order and a
+// queued batch would delay the contractions the exchange chain waits for.
+//
 // No TMA multicast and no multicast commit are used.  Every wait is bounded.
 #include "sa_device.cuh"
 #include "sa_kernels.h"
 
 #include <cstdio>
-#include <cstdlib>
 
 namespace sa {
 namespace pairbwd {
 
 constexpr int BM = 64;                      // queries per step
+constexpr int kStages = 3;                  // Q (rank 0) / dO (rank 1) stages
+constexpr int kNX = 4;                      // exchange tiles per rank
 constexpr int kKPanel = 128 * 128;          // [128 rows x 64 cols] bf16 (16 KB)
 constexpr int kQPanel = BM * 128;           // [64 rows x 64 cols] bf16 (8 KB)
-constexpr int kTile = 128 * BM * 2;         // [128 keys][64 q] bf16 exchange tile (16 KB)
-constexpr int kOffA = 0;                    // rank 0: K (4 panels); rank 1: V (4 panels)
-constexpr int kOffB = 64 * 1024;            // rank 1: K panels 2,3; rank 0: dQ staging + words
-constexpr int kOffBM = kOffB + 16 * 1024;   // rank 0: presence words [2][64][4] (index mode)
-constexpr int kOffStage = 96 * 1024;        // two stages of 48 KB
-constexpr int kStageBytes = 48 * 1024;      // rank 0: Q p0-3, dO p0-1; rank 1: dO p0-3, Q p2-3
-constexpr int kOffX = kOffStage + 2 * kStageBytes;   // two exchange tiles
-constexpr int kOffL = kOffX + 2 * kTile;              // per stage lse2[64] / delta[64]
-constexpr int kOffBar = kOffL + 2 * BM * 4;
-constexpr int kSmem = kOffBar + 256 + 1024;
+constexpr int kStageBytes = 4 * kQPanel;    // one 64 x 256 tile (32 KB)
+constexpr int kTile = 128 * BM * 2;         // exchange tile [128 keys][64 q] bf16 (16 KB)
+// rank 0: K | 3 Q stages | 4 exchange tiles | lse2 per stage
+constexpr int kOffK0 = 0;
+constexpr int kOffStage0 = 64 * 1024;
+constexpr int kOffX0 = kOffStage0 + kStages * kStageBytes;
+constexpr int kOffL0 = kOffX0 + kNX * kTile;
+// rank 1: K columns 128..255 | 3 dO stages | 4 exchange tiles | dQ staging | delta per
+// stage.  V passes through stages 1 and 2 on its way into TMEM.
+constexpr int kOffK1 = 0;
+constexpr int kOffStage1 = 32 * 1024;
+constexpr int kOffV1 = kOffStage1 + kStageBytes;
+constexpr int kOffX1 = kOffStage1 + kStages * kStageBytes;
+constexpr int kOffDQ1 = kOffX1 + kNX * kTile;
+constexpr int kOffL1 = kOffDQ1 + kTile;
+// barriers at the same offset on both ranks (a rank addresses the peer's barriers
+// through its own offsets)
+constexpr int kOffBar = kOffL0 + 1024;
+constexpr int kSmem = kOffBar + 512 + 1024;
 constexpr int kThreads = 448;
+static_assert(kOffL0 + kStages * BM * 4 <= kOffBar, "rank 0 shared-memory layout");
+static_assert(kOffL1 + kStages * BM * 4 <= kOffBar, "rank 1 shared-memory layout");
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
-// TMEM columns
-constexpr uint32_t kColBuf = 0;   // + 64 * b: S^T (rank 0) / dP^T (rank 1); packed bf16 in low cols
-constexpr uint32_t kColDQ = 128;  // dQ^T (head-dim row x 64 queries)
-constexpr uint32_t kColDV = 192;
-constexpr uint32_t kColDK = 320;
+// TMEM columns.  Rank 0: S^T buffers, dK, dQ^T.  Rank 1: dP^T buffers (each then holds
+// the step's dQ^T half), dV, V as the A operand (bf16, two per column).
+constexpr uint32_t kColS0 = 0;     // + 64 * (step % 3)
+constexpr uint32_t kColAcc0 = 192;
+constexpr uint32_t kColDQ0 = 448;
+constexpr uint32_t kColP1 = 0;     // + 64 * (step % 2)
+constexpr uint32_t kColAcc1 = 128;
+constexpr uint32_t kColV1 = 384;
 constexpr uint32_t kTmemCols = 512;
+// how many steps S^T (rank 0) / dP^T (rank 1) may run ahead of the oldest dK / dV
+constexpr int kLookS0 = 2;
+constexpr int kLookS1 = 1;
 
 enum : int {
-  kBKV = 0, kBQF = 1, kBQE = 3, kBLF = 5, kBSF = 7, kBEW = 9, kBXF = 11, kBXE = 13, kBPV = 15,
-  kBDQF = 17, kBDQE = 19, kBFin = 21, kBDrain = 22, kBXS = 23, kNumBars = 25
+  kBKV = 0,    // K / V (and rank 1's K half) loaded
+  kBVT = 1,    // rank 1: V copied into TMEM (256 threads)
+  kBQF = 2,    // [3] stage loaded
+  kBQE = 5,    // [3] stage free (commit after dK on rank 0, after dV on rank 1)
+  kBLF = 8,    // [3] per-stage LSE / Delta written (32 producer lanes)
+  kBSF = 11,   // [3] S^T / dP^T of step complete (commit), indexed by step % 3
+  kBEW = 14,   // [3] elementwise work of the step done (256 threads)
+  kBXF = 17,   // [4] exchange tile received (receiver's arrival + 16 KB)
+  kBXT = 21,   // [4] rank 0: own tile free after its dQ drain
+  kBXE = 25,   // [4] rank 0: rank 1's tile free (remote)
+  kBXS = 29,   // [4] rank 1: its dS^T copy has landed in rank 0 (remote)
+  kBPV = 33,   // [4] rank 1: dV has read P^T from the tile (commit)
+  kBDQF = 37,  // [2] dQ^T complete (commit); rank 0 uses slot 0 only
+  kBDQE = 39,  // [2] dQ^T drained from TMEM (128 threads)
+  kBFin = 41, kBDrain = 42, kNumBars = 43
 };
+static_assert(8 * kNumBars + 8 <= 512, "barrier area");
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     sparse_bwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -100,36 +136,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
   const int n_full = __ldg(a.tcnt + 2 * trow);
   const int n_mt = n_full + __ldg(a.tcnt + 2 * trow + 1);
   const int32_t* tlist = a.tidx + trow * a.Tm;
-  const int n_iter = G * n_mt * 2;
-  const int c0 = 128 * static_cast<int>(rank);  // this rank's head-dim half
+  const int n_iter = G * n_mt * 2;  // (query head, query tile, 64-row half)
+  const uint32_t off_stage = rank == 0 ? kOffStage0 : kOffStage1;
+  const uint32_t off_x = rank == 0 ? kOffX0 : kOffX1;
+  const uint32_t off_l = rank == 0 ? kOffL0 : kOffL1;
+  const uint32_t col_acc = rank == 0 ? kColAcc0 : kColAcc1;
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(kBKV), 1);
-    for (int s = 0; s < 2; ++s) {
+    mbar_init(BAR(kBVT), 256);
+    for (int s = 0; s < 3; ++s) {
       mbar_init(BAR(kBQF + s), 1);
       mbar_init(BAR(kBQE + s), 1);
       mbar_init(BAR(kBLF + s), 32);
       mbar_init(BAR(kBSF + s), 1);
       mbar_init(BAR(kBEW + s), 256);
+    }
+    for (int s = 0; s < kNX; ++s) {
       mbar_init(BAR(kBXF + s), 1);
+      mbar_init(BAR(kBXT + s), 1);
       mbar_init(BAR(kBXE + s), 1);
       mbar_init(BAR(kBXS + s), 1);
       mbar_init(BAR(kBPV + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(kBDQF + s), 1);
       mbar_init(BAR(kBDQE + s), 128);
     }
     mbar_init(BAR(kBFin), 1);
     mbar_init(BAR(kBDrain), 1);
     *abort_flag = 0;
+    // the first exchange tiles may arrive from the peer at any time
+    for (int s = 0; s < kNX && s < n_iter; ++s) mbar_arrive_expect_tx(BAR(kBXF + s), kTile);
     fence_mbar_init();
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
-  }
-  // the exchange tiles of steps 0 and 1 may arrive from the peer at any time
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < 2 && s < n_iter; ++s) mbar_arrive_expect_tx(BAR(kBXF + s), kTile);
   }
   tc_fence_before();
   __syncthreads();
@@ -159,44 +202,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         if (rank == 0) {
           mbar_arrive_expect_tx(BAR(kBKV), 4 * kKPanel);
           for (int c = 0; c < 4; ++c)
-            tma_load_4d(sbase + kOffA + c * kKPanel, &tm_k, BAR(kBKV), c * 64, nt * 128, g, b);
+            tma_load_4d(sbase + kOffK0 + c * kKPanel, &tm_k, BAR(kBKV), c * 64, nt * 128, g, b);
         } else {
           mbar_arrive_expect_tx(BAR(kBKV), 6 * kKPanel);
           for (int c = 0; c < 4; ++c)
-            tma_load_4d(sbase + kOffA + c * kKPanel, &tm_v, BAR(kBKV), c * 64, nt * 128, g, b);
+            tma_load_4d(sbase + kOffV1 + c * kKPanel, &tm_v, BAR(kBKV), c * 64, nt * 128, g, b);
           for (int c = 2; c < 4; ++c)
-            tma_load_4d(sbase + kOffB + (c - 2) * kKPanel, &tm_k, BAR(kBKV), c * 64, nt * 128, g, b);
+            tma_load_4d(sbase + kOffK1 + (c - 2) * kKPanel, &tm_k, BAR(kBKV), c * 64, nt * 128, g, b);
         }
       }
       __syncwarp();
-      float* lbuf = reinterpret_cast<float*>(smem + kOffL);
-      uint32_t* bmbuf = reinterpret_cast<uint32_t*>(smem + kOffBM);
+      float* lbuf = reinterpret_cast<float*>(smem + off_l);
+      const CUtensorMap* tm_stage = rank == 0 ? &tm_q : &tm_do;
       for (int it = 0; it < n_iter; ++it) {
         int h, m0;
         bool partial;
         decode(it, h, m0, partial);
-        m0 = __shfl_sync(0xFFFFFFFFu, m0, 0);
-        const int st = it & 1, u = it >> 1;
-        if (!warp_wait(BAR(kBQE + st), (u & 1) ^ 1, abort_flag, a.status)) break;
-        const uint32_t qs = sbase + kOffStage + st * kStageBytes;
+        m0 = __shfl_sync(0xFFFFFFFFu, m0, 0);  // warp-uniform TMA coordinate
+        const int s = it % kStages, u = it / kStages;
+        if (!warp_wait(BAR(kBQE + s), (u & 1) ^ 1, abort_flag, a.status)) break;
+        // rank 1: V occupies stages 1 and 2 until it has been copied into TMEM
+        if (rank == 1 && (it == 1 || it == 2) && !warp_wait(BAR(kBVT), 0, abort_flag, a.status))
+          break;
+        const uint32_t qs = sbase + off_stage + s * kStageBytes;
         if (elect_one()) {
-          mbar_arrive_expect_tx(BAR(kBQF + st), kStageBytes);
-          if (rank == 0) {
-            for (int c = 0; c < 4; ++c)
-              tma_load_4d(qs + c * kQPanel, &tm_q, BAR(kBQF + st), c * 64, m0, h, b);
-            for (int c = 0; c < 2; ++c)
-              tma_load_4d(qs + 32 * 1024 + c * kQPanel, &tm_do, BAR(kBQF + st), c * 64, m0, h, b);
-          } else {
-            for (int c = 0; c < 4; ++c)
-              tma_load_4d(qs + c * kQPanel, &tm_do, BAR(kBQF + st), c * 64, m0, h, b);
-            for (int c = 2; c < 4; ++c)
-              tma_load_4d(qs + 32 * 1024 + (c - 2) * kQPanel, &tm_q, BAR(kBQF + st), c * 64, m0, h,
-                          b);
-          }
+          mbar_arrive_expect_tx(BAR(kBQF + s), kStageBytes);
+          for (int c = 0; c < 4; ++c) tma_load_4d(qs + c * kQPanel, tm_stage, BAR(kBQF + s), c * 64, m0, h, b);
         }
         __syncwarp();
+        // the tile of step it + 3 is requested into L2 now, so that its own load (issued
+        // when a stage frees up) mostly hits L2
+        if (it + kStages < n_iter) {
+          int hp, mp;
+          bool pp;
+          decode(it + kStages, hp, mp, pp);
+          mp = __shfl_sync(0xFFFFFFFFu, mp, 0);
+          if (elect_one())
+            for (int c = 0; c < 4; ++c) tma_prefetch_l2_4d(tm_stage, c * 64, mp, hp, b);
+          __syncwarp();
+        }
+        // rank 1 frees a stage when dV is done, which can precede the elementwise warps'
+        // read of the step's Delta: wait for them before overwriting it
+        if (rank == 1 && it >= kStages &&
+            !warp_wait(BAR(kBEW + s), ((it - kStages) / kStages) & 1, abort_flag, a.status))
+          break;
         // rank 0: LSE in log2 units (+inf past Sq); rank 1: Delta (0 past Sq)
-        float* ls = lbuf + st * BM;
+        float* ls = lbuf + s * BM;
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           const int q = lane + 32 * k;
@@ -208,135 +259,148 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
           }
           ls[q] = v;
         }
-        if (rank == 0 && partial && a.mode == SA_MODE_INDEX) {
-          uint32_t* bw = bmbuf + st * BM * 4;
-          for (int e = lane; e < BM * 4; e += 32) {
-            const int q = e >> 2, w = nt * 4 + (e & 3);
-            const int64_t i = m0 + q;
-            bw[e] = (i < a.Sq && w < a.W) ? __ldg(a.bitmap + (bg * a.Sq + i) * a.W + w) : 0u;
-          }
-        }
-        mbar_arrive(BAR(kBLF + st));
+        mbar_arrive(BAR(kBLF + s));
       }
       if (lane == 0 && *abort_flag) {
         mbar_wait_limited(BAR(kBKV), 0);
-        for (int it = max(0, n_iter - 2); it < n_iter; ++it)
-          mbar_wait_limited(BAR(kBQF + (it & 1)), (it >> 1) & 1);
+        for (int it = max(0, n_iter - kStages); it < n_iter; ++it)
+          mbar_wait_limited(BAR(kBQF + it % kStages), (it / kStages) & 1);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
+    // The whole warp runs this loop (converged, warp-uniform decisions from lane 0);
+    // one elected lane issues each batch of tcgen05 instructions.
     if (n_iter > 0) {
       constexpr uint32_t idesc_s = idesc_bf16(128, BM, 0, 0);     // S^T / dP^T
-      constexpr uint32_t idesc_dq = idesc_bf16(128, BM, 1, 1);    // dQ^T = K^T dS^T
-      constexpr uint32_t idesc_tsn = idesc_bf16(128, 128, 0, 1);  // A in TMEM, B MN-major
-      constexpr uint32_t idesc_ssn = idesc_bf16(128, 128, 0, 1);  // A K-major smem, B MN-major
-      const uint64_t ad = sw128_desc(sbase + kOffA, 16, 1024);    // K (rank 0) / V (rank 1)
+      constexpr uint32_t idesc_acc = idesc_bf16(128, 256, 0, 1);  // dK / dV (tile K-major, stage MN-major)
+      constexpr uint32_t idesc_dq = idesc_bf16(128, BM, 1, 1);    // dQ^T (both MN-major)
+      const uint64_t kd = sw128_desc(sbase + kOffK0, 16, 1024);   // rank 0: S^T A operand
       // dQ^T A operand: this rank's 128 head-dim rows of K (MN-major)
-      const uint64_t kwd = sw128_desc(sbase + (rank == 0 ? kOffA : kOffB), kKPanel, 1024);
-      bool ok = warp_wait(BAR(kBKV), 0, abort_flag, a.status);
-      // S^T (rank 0) or dP^T (rank 1) of step j into TMEM buffer j & 1
-      auto issue_first = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!warp_wait(BAR(kBQF + st), (j >> 1) & 1, abort_flag, a.status)) return false;
-        tc_fence_after();
-        const uint64_t bd = sw128_desc(sbase + kOffStage + st * kStageBytes, 16, 1024);
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < 16; ++kk) {
-            const uint32_t off_a = (kk >> 2) * kKPanel + (kk & 3) * 32;
-            const uint32_t off_b = (kk >> 2) * kQPanel + (kk & 3) * 32;
-            umma_ss(tmem + kColBuf + 64 * st, ad + (off_a >> 4), bd + (off_b >> 4), idesc_s,
-                    kk > 0 ? 1u : 0u);
-          }
-          umma_commit(BAR(kBSF + st));
-        }
-        __syncwarp();
-        return true;
+      const uint64_t kwd = sw128_desc(sbase + (rank == 0 ? kOffK0 : kOffK1), kKPanel, 1024);
+      auto ready = [&](int k, int parity) {
+        return __shfl_sync(0xFFFFFFFFu, mbar_test(BAR(k), parity) ? 1 : 0, 0) != 0;
       };
-      if (ok) ok = issue_first(0);
-      for (int it = 0; ok && it < n_iter; ++it) {
-        const int bi = it & 1, st = it & 1, ph = (it >> 1) & 1;
-        const uint32_t qs = sbase + kOffStage + st * kStageBytes;
-        const uint32_t xt = sbase + kOffX + bi * kTile;
-        // this rank's half of the second operand: rank 0 dO panels 0,1 / Q panels 0,1;
-        // rank 1 dO panels 2,3 / Q panels 2,3
-        const uint64_t do_half = sw128_desc(qs + (rank == 0 ? 32 * 1024 : 2 * kQPanel), kQPanel, 1024);
-        const uint64_t q_half = sw128_desc(qs + (rank == 0 ? 0 : 32 * 1024), kQPanel, 1024);
-        const uint64_t xk = sw128_desc(xt, 16, 1024);        // exchange tile, K-major A
-        const uint64_t xmn = sw128_desc(xt, kKPanel, 1024);  // exchange tile, MN-major B
-        if (rank == 0) {
-          // the next S^T overlaps this step's elementwise work
-          if (it + 1 < n_iter && !issue_first(it + 1)) break;
-          // dV += P^T dO (P^T packed in TMEM by the elementwise warps)
-          if (!warp_wait(BAR(kBEW + bi), ph, abort_flag, a.status)) break;
-          tc_fence_after();
+      bool ok = warp_wait(BAR(kBKV), 0, abort_flag, a.status);
+      if (rank == 1) ok = ok && warp_wait(BAR(kBVT), 0, abort_flag, a.status);
+      int js = 0;  // next S^T (rank 0) / dP^T (rank 1)
+      int jv = 0;  // rank 1: next dV
+      int jk = 0;  // next dK + dQ^T (rank 0) / dQ^T (rank 1)
+      int jx = 0;  // rank 0: next step whose dS^T arrival is reported back to rank 1
+      uint64_t t_last = globaltimer_ns();
+      while (ok && jk < n_iter) {
+        bool prog = false;
+        // rank 0: report each dS^T arrival at once and arm the barrier for the step that
+        // uses the tile next
+        if (rank == 0 && jx < js && ready(kBXF + jx % kNX, (jx / kNX) & 1)) {
           if (elect_one()) {
+            mbar_arrive_remote_relaxed(mapa_shared(BAR(kBXS + jx % kNX), peer));
+            if (jx + kNX < n_iter) mbar_arrive_expect_tx(BAR(kBXF + jx % kNX), kTile);
+          }
+          __syncwarp();
+          ++jx;
+          prog = true;
+        }
+        // rank 1: dV += P^T dO as soon as P^T of the oldest step has arrived
+        if (rank == 1 && jv < js && ready(kBXF + jv % kNX, (jv / kNX) & 1)) {
+          tc_fence_after();
+          const int xb = jv % kNX;
+          const uint64_t xk = sw128_desc(sbase + off_x + xb * kTile, 16, 1024);
+          const uint64_t bmn = sw128_desc(sbase + off_stage + (jv % kStages) * kStageBytes, kQPanel, 1024);
+          if (elect_one()) {
+            // every reader of this phase has passed it (the elementwise warps read the
+            // tile before P^T of step jv+4 can be sent): arm the barrier for step jv+4
+            if (jv + kNX < n_iter) mbar_arrive_expect_tx(BAR(kBXF + xb), kTile);
 #pragma unroll
             for (int kk = 0; kk < BM / 16; ++kk)
-              umma_ts(tmem + kColDV, tmem + kColBuf + 64 * bi + (kk >> 1) * 32 + (kk & 1) * 8,
-                      do_half + ((kk * 2048) >> 4), idesc_tsn, (it > 0 || kk > 0) ? 1u : 0u);
+              umma_ss(tmem + col_acc, xk + ((kk * 32) >> 4), bmn + ((kk * 2048) >> 4), idesc_acc,
+                      (jv > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(BAR(kBPV + xb));            // P^T read: dS^T may replace it
+            umma_commit(BAR(kBQE + jv % kStages));  // dO stage free (dP^T read it earlier)
           }
           __syncwarp();
-          // dK += dS^T Q with dS^T copied in by rank 1 (exchange tile, K-major A)
-          if (!warp_wait(BAR(kBXF + bi), ph, abort_flag, a.status)) break;
-          if (elect_one()) {
-            mbar_arrive_remote_relaxed(mapa_shared(BAR(kBXS + bi), peer));
-            if (it + 2 < n_iter) mbar_arrive_expect_tx(BAR(kBXF + bi), kTile);
-          }
-          __syncwarp();
+          ++jv;
+          prog = true;
+        }
+        // rank 0: dK += dS^T Q and dQ^T once dS^T has arrived and the last dQ^T has been
+        // drained; rank 1: dQ^T once its elementwise warps have written dS^T
+        if (rank == 0 ? (jk < jx && (jk == 0 || ready(kBDQE, (jk - 1) & 1)))
+                      : (jk < jv && ready(kBEW + jk % kStages, (jk / kStages) & 1))) {
           tc_fence_after();
+          const uint32_t xt = sbase + off_x + (jk % kNX) * kTile;
+          const uint64_t xmn = sw128_desc(xt, kKPanel, 1024);  // exchange tile, MN-major B
+          if (rank == 0) {
+            const uint64_t xk = sw128_desc(xt, 16, 1024);      // exchange tile, K-major A
+            const uint64_t bmn = sw128_desc(sbase + off_stage + (jk % kStages) * kStageBytes, kQPanel, 1024);
+            if (elect_one()) {
+#pragma unroll
+              for (int kk = 0; kk < BM / 16; ++kk)
+                umma_ss(tmem + col_acc, xk + ((kk * 32) >> 4), bmn + ((kk * 2048) >> 4), idesc_acc,
+                        (jk > 0 || kk > 0) ? 1u : 0u);
+              umma_commit(BAR(kBQE + jk % kStages));  // Q stage free
+            }
+            __syncwarp();
+          }
+          const uint32_t dq_col = rank == 0 ? kColDQ0 : kColP1 + 64 * (jk & 1);
           if (elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < BM / 16; ++kk)
-              umma_ss(tmem + kColDK, xk + ((kk * 32) >> 4), q_half + ((kk * 2048) >> 4), idesc_ssn,
-                      (it > 0 || kk > 0) ? 1u : 0u);
-            umma_commit(BAR(kBQE + st));
+            for (int kk = 0; kk < 128 / 16; ++kk)
+              umma_ss(tmem + dq_col, kwd + ((kk * 2048) >> 4), xmn + ((kk * 2048) >> 4), idesc_dq,
+                      kk > 0 ? 1u : 0u);
+            umma_commit(BAR(kBDQF + (rank == 0 ? 0 : (jk & 1))));
           }
           __syncwarp();
+          ++jk;
+          prog = true;
+        }
+        // S^T (rank 0) / dP^T (rank 1) of the next step: stage loaded, TMEM buffer free
+        // (rank 0: read by the elementwise warps; rank 1: its dQ^T drained), not too far
+        // ahead of the dK / dV stream
+        if (js < n_iter && js <= (rank == 0 ? jk + kLookS0 : jv + kLookS1) &&
+            ready(kBQF + js % kStages, (js / kStages) & 1) &&
+            (rank == 0 ? (js < 3 || ready(kBEW + js % 3, ((js - 3) / 3) & 1))
+                       : (js < 2 || ready(kBDQE + (js & 1), ((js - 2) >> 1) & 1)))) {
+          tc_fence_after();
+          const int s = js % kStages;
+          const uint64_t bd = sw128_desc(sbase + off_stage + s * kStageBytes, 16, 1024);
+          if (elect_one()) {
+            if (rank == 0) {
+#pragma unroll
+              for (int kk = 0; kk < 16; ++kk) {
+                const uint32_t off_a = (kk >> 2) * kKPanel + (kk & 3) * 32;
+                const uint32_t off_b = (kk >> 2) * kQPanel + (kk & 3) * 32;
+                umma_ss(tmem + kColS0 + 64 * s, kd + (off_a >> 4), bd + (off_b >> 4), idesc_s,
+                        kk > 0 ? 1u : 0u);
+              }
+            } else {
+              // A = V from TMEM: 16 head-dim columns (8 TMEM columns) per k-step
+#pragma unroll
+              for (int kk = 0; kk < 16; ++kk) {
+                const uint32_t off_b = (kk >> 2) * kQPanel + (kk & 3) * 32;
+                umma_ts(tmem + kColP1 + 64 * (js & 1), tmem + kColV1 + kk * 8, bd + (off_b >> 4),
+                        idesc_s, kk > 0 ? 1u : 0u);
+              }
+            }
+            umma_commit(BAR(kBSF + s));
+          }
+          __syncwarp();
+          ++js;
+          prog = true;
+        }
+        if (prog) {
+          t_last = globaltimer_ns();
         } else {
-          // dV += P^T dO with P^T copied in by rank 0 (exchange tile, K-major A), first,
-          // so that the elementwise warps may overwrite the tile with dS^T soon
-          if (!warp_wait(BAR(kBXF + bi), ph, abort_flag, a.status)) break;
-          tc_fence_after();
-          if (elect_one()) {
-            // every reader of this phase has passed its wait (the elementwise warps read
-            // the tile before step it+2 can be sent): arm the barrier for step it+2
-            if (it + 2 < n_iter) mbar_arrive_expect_tx(BAR(kBXF + bi), kTile);
-#pragma unroll
-            for (int kk = 0; kk < BM / 16; ++kk)
-              umma_ss(tmem + kColDV, xk + ((kk * 32) >> 4), do_half + ((kk * 2048) >> 4), idesc_ssn,
-                      (it > 0 || kk > 0) ? 1u : 0u);
-            umma_commit(BAR(kBPV + bi));
+          if (__shfl_sync(0xFFFFFFFFu, *abort_flag, 0) != 0) break;
+          if (globaltimer_ns() - t_last > kWaitLimitNs) {
+            if (lane == 0) {
+              *abort_flag = 1;
+              report_status(a.status, kStatusTimeout);
+            }
+            __syncwarp();
+            break;
           }
-          __syncwarp();
-          // the next dP^T overlaps this step's elementwise work
-          if (it + 1 < n_iter && !issue_first(it + 1)) break;
-          // dK += dS^T Q (dS^T packed in TMEM by the elementwise warps)
-          if (!warp_wait(BAR(kBEW + bi), ph, abort_flag, a.status)) break;
-          tc_fence_after();
-          if (elect_one()) {
-#pragma unroll
-            for (int kk = 0; kk < BM / 16; ++kk)
-              umma_ts(tmem + kColDK, tmem + kColBuf + 64 * bi + (kk >> 1) * 32 + (kk & 1) * 8,
-                      q_half + ((kk * 2048) >> 4), idesc_tsn, (it > 0 || kk > 0) ? 1u : 0u);
-            umma_commit(BAR(kBQE + st));
-          }
-          __syncwarp();
+          __nanosleep(32);
         }
-        // dQ^T = K^T dS^T for this rank's head-dim half, once the last one was drained
-        if (it >= 1 &&
-            !warp_wait(BAR(kBDQE + ((it - 1) & 1)), ((it - 1) >> 1) & 1, abort_flag, a.status))
-          break;
-        tc_fence_after();
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk)
-            umma_ss(tmem + kColDQ, kwd + ((kk * 2048) >> 4), xmn + ((kk * 2048) >> 4), idesc_dq,
-                    kk > 0 ? 1u : 0u);
-          umma_commit(BAR(kBDQF + bi));
-        }
-        __syncwarp();
       }
       if (elect_one()) umma_commit(BAR(kBFin));
       __syncwarp();
@@ -348,33 +412,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     const int r = quarter * 32 + lane;  // key row = TMEM lane
     const int64_t j = static_cast<int64_t>(nt) * 128 + r;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const float* lbuf = reinterpret_cast<const float*>(smem + kOffL);
-    const uint32_t* bmbuf = reinterpret_cast<const uint32_t*>(smem + kOffBM);
+    const float* lbuf = reinterpret_cast<const float*>(smem + off_l);
     const bool key_ok = j < a.Sk;
     bool ok = true;
-    for (int it = 0; it < n_iter; ++it) {
+    if (rank == 1 && n_iter > 0) {
+      // V row r into TMEM (row r in lane r, head dims 2e, 2e+1 in column e): this half
+      // of the warps copies head dims [128 hc, 128 hc + 128) from the swizzled panels
+      const bool v_ok = __all_sync(0xFFFFFFFFu, mbar_wait(BAR(kBKV), 0, abort_flag, a.status));
+      if (v_ok) {
+#pragma unroll
+        for (int pl = 0; pl < 2; ++pl) {
+          const int p = 2 * hc + pl;
+          const uint8_t* prow = smem + kOffV1 + p * kKPanel + r * 128;
+          uint32_t w[32];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint4 v = *reinterpret_cast<const uint4*>(prow + ((k ^ (r & 7)) << 4));
+            w[4 * k] = v.x;
+            w[4 * k + 1] = v.y;
+            w[4 * k + 2] = v.z;
+            w[4 * k + 3] = v.w;
+          }
+          tmem_st32(tl + kColV1 + p * 32, w);
+        }
+        tmem_wait_st();
+      }
+      ok = v_ok;
+      fence_proxy_async_smem();  // the producer reloads these stages with TMA next
+      tc_fence_before();
+      mbar_arrive(BAR(kBVT));
+    }
+    for (int it = 0; ok && it < n_iter; ++it) {
       int h, m0;
       bool partial;
       decode(it, h, m0, partial);
-      const int bi = it & 1, st = it & 1, ph = (it >> 1) & 1;
-      bool w_ok = mbar_wait(BAR(kBLF + st), ph, abort_flag, a.status);
-      w_ok = w_ok && mbar_wait(BAR(kBSF + bi), ph, abort_flag, a.status);
-      if (rank == 1) {
-        w_ok = w_ok && mbar_wait(BAR(kBXF + bi), ph, abort_flag, a.status);  // P^T(it) arrived
-      } else if (it >= 2) {
-        // own tile b: dK and dQ^T of step it-2 have read dS^T
-        w_ok = w_ok && mbar_wait(BAR(kBDQF + bi), ((it - 2) >> 1) & 1, abort_flag, a.status);
+      const int s = it % kStages, ph = (it / kStages) & 1;
+      const int xb = it % kNX, phx = (it / kNX) & 1;
+      bool w_ok = mbar_wait(BAR(kBLF + s), ph, abort_flag, a.status);
+      w_ok = w_ok && mbar_wait(BAR(kBSF + s), ph, abort_flag, a.status);
+      if (rank == 0) {
+        // own tile xb: the dQ drain of step it-4 is done with it
+        if (it >= kNX)
+          w_ok = w_ok && mbar_wait(BAR(kBXT + xb), phx ^ 1, abort_flag, a.status);
+      } else {
+        w_ok = w_ok && mbar_wait(BAR(kBXF + xb), phx, abort_flag, a.status);  // P^T arrived
       }
       if (!__all_sync(0xFFFFFFFFu, w_ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float* ls = lbuf + st * BM + 32 * hc;
-      const uint32_t cbuf = kColBuf + 64 * bi + 32 * hc;
+      const float* ls = lbuf + s * BM + 32 * hc;
+      const uint32_t row_off = off_x + xb * kTile + r * 128;  // row r of own tile xb
       uint32_t s_u[32];
-      tmem_ld32(tl + cbuf, s_u);
-      const uint32_t row_off = kOffX + bi * kTile + r * 128;  // row r of exchange tile b
+      tmem_ld32(tl + (rank == 0 ? kColS0 + 64 * s : kColP1 + 64 * (it & 1)) + 32 * hc, s_u);
       uint32_t pk[16];
       if (rank == 0) {
         uint32_t cm = 0xFFFFFFFFu;
@@ -391,10 +482,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                            __ldg(a.mask + (bg * a.Mb + mb) * static_cast<int64_t>(a.Nb) + j / 64) != 0;
             if (!m) cm = 0u;
           } else if (a.mode == SA_MODE_INDEX) {
-            const uint32_t* bw = bmbuf + st * BM * 4 + (32 * hc) * 4 + (r >> 5);
+            // presence word of this key row's 32-key group for each of the 32 queries
+            // (the same address across the warp: one broadcast load per query)
+            const int w = nt * 4 + (r >> 5);
             uint32_t bits = 0u;
 #pragma unroll 8
-            for (int q = 0; q < 32; ++q) bits |= ((bw[q * 4] >> lane) & 1u) << q;
+            for (int q = 0; q < 32; ++q) {
+              const int64_t i = q0 + q;
+              const uint32_t word =
+                  (i < a.Sq && w < a.W) ? __ldg(a.bitmap + (bg * a.Sq + i) * a.W + w) : 0u;
+              bits |= ((word >> lane) & 1u) << q;
+            }
             cm &= bits;
           }
         }
@@ -414,28 +512,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
           pk[2 * e4] = pack_bf16x2(pv[0], pv[1]);
           pk[2 * e4 + 1] = pack_bf16x2(pv[2], pv[3]);
         }
-        tmem_st16(tl + cbuf, pk);
-        // P^T row (this half's 32 queries) into the own exchange tile, 128-byte swizzled:
-        // 16-byte chunk c of row r lives at chunk c ^ (r % 8)
+        // P^T row (this half's 32 queries), 128-byte swizzled: 16-byte chunk c of row r
+        // lives at chunk c ^ (r % 8)
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
           const int c = hc * 4 + c4;
           *reinterpret_cast<uint4*>(smem + row_off + ((c ^ (r & 7)) << 4)) =
               make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
         }
-        tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(BAR(kBEW + bi));
-        // one thread copies the whole tile into rank 1 once every row is in and rank 1's
-        // tile b is free (its dQ drain of step it-2 is done with it)
-        if (threadIdx.x == 64 && mbar_wait(BAR(kBEW + bi), ph, abort_flag, a.status) &&
-            (it < 2 || mbar_wait(BAR(kBXE + bi), ((it - 2) >> 1) & 1, abort_flag, a.status))) {
-          bulk_copy_to_cluster(mapa_shared(sbase + kOffX + bi * kTile, peer),
-                               sbase + kOffX + bi * kTile, kTile, mapa_shared(BAR(kBXF + bi), peer));
+        mbar_arrive(BAR(kBEW + s));
+        // one thread copies the tile into rank 1's tile xb once every row is in and that
+        // tile is free (rank 1 is done with step it-4 there)
+        if (threadIdx.x == 64 && mbar_wait(BAR(kBEW + s), ph, abort_flag, a.status) &&
+            (it < kNX || mbar_wait(BAR(kBXE + xb), phx ^ 1, abort_flag, a.status))) {
+          bulk_copy_to_cluster(mapa_shared(sbase + kOffX1 + xb * kTile, peer),
+                               sbase + kOffX0 + xb * kTile, kTile, mapa_shared(BAR(kBXF + xb), peer));
         }
       } else {
-        // P^T row from the own exchange tile (written by rank 0)
+        // P^T row (copied in by rank 0)
         uint32_t pw[16];
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
@@ -463,9 +559,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
           pk[2 * e4] = pack_bf16x2(dsv[0], dsv[1]);
           pk[2 * e4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
         }
-        tmem_st16(tl + cbuf, pk);
         // dV of this step must have read P^T before dS^T replaces it in the tile
-        const bool pv_ok = mbar_wait(BAR(kBPV + bi), ph, abort_flag, a.status);
+        const bool pv_ok = mbar_wait(BAR(kBPV + xb), phx, abort_flag, a.status);
         if (!__all_sync(0xFFFFFFFFu, pv_ok)) {
           ok = false;
           break;
@@ -476,14 +571,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
           *reinterpret_cast<uint4*>(smem + row_off + ((c ^ (r & 7)) << 4)) =
               make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
         }
-        tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(BAR(kBEW + bi));
-        // one thread copies the whole dS^T tile into rank 0 once every row is in
-        if (threadIdx.x == 64 && mbar_wait(BAR(kBEW + bi), ph, abort_flag, a.status)) {
-          bulk_copy_to_cluster(mapa_shared(sbase + kOffX + bi * kTile, peer),
-                               sbase + kOffX + bi * kTile, kTile, mapa_shared(BAR(kBXF + bi), peer));
+        mbar_arrive(BAR(kBEW + s));
+        // one thread copies the dS^T tile into rank 0's tile xb once every row is in
+        // (that tile held P^T of this step, which rank 1 has already received)
+        if (threadIdx.x == 64 && mbar_wait(BAR(kBEW + s), ph, abort_flag, a.status)) {
+          bulk_copy_to_cluster(mapa_shared(sbase + kOffX0 + xb * kTile, peer),
+                               sbase + kOffX1 + xb * kTile, kTile, mapa_shared(BAR(kBXF + xb), peer));
         }
       }
     }
@@ -494,76 +589,76 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       have = __all_sync(0xFFFFFFFFu, w_ok);
       tc_fence_after();
     }
-    __nv_bfloat16* dkrow = reinterpret_cast<__nv_bfloat16*>(a.dk) +
-                           ((static_cast<int64_t>(b) * a.Sk + j) * a.HK + g) * 256;
-    __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(a.dv) +
-                           ((static_cast<int64_t>(b) * a.Sk + j) * a.HK + g) * 256;
-    for (int pass = 0; pass < 2; ++pass) {
-      const uint32_t col = pass == 0 ? kColDK : kColDV;
-      const float sc = pass == 0 ? a.scale : 1.f;
-      __nv_bfloat16* out = pass == 0 ? dkrow : dvrow;
-      for (int c = 32 * hc; c < 128; c += 64) {
-        uint32_t v[32];
-        if (have) {
-          tmem_ld32(tl + col + c, v);
-          tmem_wait_ld();
-        } else {
+    // rank 0 stores dK (times softmax_scale), rank 1 stores dV
+    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(rank == 0 ? a.dk : a.dv) +
+                         ((static_cast<int64_t>(b) * a.Sk + j) * a.HK + g) * 256;
+    const float sc = rank == 0 ? a.scale : 1.f;
+    for (int c = 32 * hc; c < 256; c += 64) {
+      uint32_t v[32];
+      if (have) {
+        tmem_ld32(tl + col_acc + c, v);
+        tmem_wait_ld();
+      } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = 0u;
-        }
-        if (key_ok) {
-          uint32_t pq[16];
+        for (int e = 0; e < 32; ++e) v[e] = 0u;
+      }
+      if (key_ok) {
+        uint32_t pq[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pq[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
-          uint4* dst = reinterpret_cast<uint4*>(out + c0 + c);
+        for (int e = 0; e < 16; ++e)
+          pq[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
+        uint4* dst = reinterpret_cast<uint4*>(out + c);
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pq[4 * e], pq[4 * e + 1], pq[4 * e + 2], pq[4 * e + 3]);
-        }
+        for (int e = 0; e < 4; ++e)
+          dst[e] = make_uint4(pq[4 * e], pq[4 * e + 1], pq[4 * e + 2], pq[4 * e + 3]);
       }
     }
   } else {
     // ------------------------------------------------------------------ dQ drain
+    // thread = head-dim row r of this rank's half; the 64 query columns are staged as
+    // fp32 (rank 0: in the step's exchange tile, free once dQ^T has read it; rank 1: in
+    // its staging buffer), 32 queries at a time, as [64-column panel][32 q][64 d] tiles
+    // that bulk reduce-adds push into dQ_acc
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;  // head-dim row of this rank's half
+    const int r = quarter * 32 + lane;
     const int dtid = threadIdx.x - 320;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const int p = r >> 6;
+    const int c0 = 128 * static_cast<int>(rank);
     bool ok = true;
     for (int it = 0; it < n_iter && ok; ++it) {
       int h, m0;
       bool partial;
       decode(it, h, m0, partial);
-      const int bi = it & 1;
+      const int xb = it % kNX, phx = (it / kNX) & 1;
+      const int qb = rank == 0 ? 0 : (it & 1);
       // the four drain warps leave together (they share named barrier 1 below)
-      const bool w_ok = mbar_wait(BAR(kBDQF + bi), (it >> 1) & 1, abort_flag, a.status);
+      const bool w_ok = mbar_wait(BAR(kBDQF + qb), rank == 0 ? (it & 1) : ((it >> 1) & 1),
+                                  abort_flag, a.status);
       if (!named_bar_and(1, 128, w_ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t q_u[BM];
-      tmem_ld32(tl + kColDQ, q_u);
-      tmem_ld32(tl + kColDQ + 32, q_u + 32);
+      const uint32_t dq_col = rank == 0 ? kColDQ0 : kColP1 + 64 * (it & 1);
+      tmem_ld32(tl + dq_col, q_u);
+      tmem_ld32(tl + dq_col + 32, q_u + 32);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(BAR(kBDQE + bi));
-      if (rank == 1) {
-        // the outgoing copy of dS^T must have read the exchange tile before staging
-        const bool x_ok = mbar_wait(BAR(kBXS + bi), (it >> 1) & 1, abort_flag, a.status);
-        if (!named_bar_and(1, 128, x_ok)) {
-          ok = false;
-          break;
-        }
-      }
-      // staging: rank 0 has a buffer of its own, rank 1 reuses the exchange tile
-      const int soff = rank == 0 ? kOffB : kOffX + bi * kTile;
+      mbar_arrive(BAR(kBDQE + qb));
+      // rank 1: its tile xb is free once dQ^T has read it (done) and its dS^T copy has
+      // landed in rank 0; tell rank 0, which sends P^T of step it+4 into it
+      if (rank == 1 && dtid == 0 && mbar_wait(BAR(kBXS + xb), phx, abort_flag, a.status))
+        mbar_arrive_remote_relaxed(mapa_shared(BAR(kBXE + xb), peer));
+      const uint32_t soff = rank == 0 ? kOffX0 + xb * kTile : kOffDQ1;
       float* stage = reinterpret_cast<float*>(smem + soff);
       const uint32_t stage_s = sbase + soff;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        if (half == 1 || rank == 0) {
+        // the previous reduce (this step's first half; on rank 1 also the last step's
+        // second half, which used the same staging buffer) must have read the buffer
+        if (half == 1 || rank == 1) {
           if (dtid == 0) bulk_wait_group_read0();
           named_bar_sync(1, 128);
         }
@@ -578,11 +673,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
           bulk_commit_group();
         }
       }
-      if (rank == 1) {
-        // the exchange tile is free once the reduce has read it: rank 0 may refill it
-        if (dtid == 0) bulk_wait_group_read0();
-        named_bar_sync(1, 128);
-        if (dtid == 0) mbar_arrive_remote_relaxed(mapa_shared(BAR(kBXE + bi), peer));
+      // rank 0: the tile is free once the reduces have read it
+      if (rank == 0 && dtid == 0) {
+        bulk_wait_group_read0();
+        mbar_arrive(BAR(kBXT + xb));
       }
     }
     if (dtid == 0) bulk_wait_group0();
