@@ -32,6 +32,14 @@ SMALL = [
              density=0.3, name="causal_d256"),
     I.scaled(W["long_causal_blocksparse_h16_s32768_d256"], Sq=333, Sk=333, HQ=1, HK=1,
              density=0.5, name="ragged_d256"),
+    # head dims 256/256 run on the 2-CTA backward: GQA, batch > 1, 64-wide blocks,
+    # index mode, and a non-causal case with Sq != Sk
+    I.scaled(W["long_causal_blocksparse_h16_s32768_d256"], B=2, Sq=384, Sk=384, HQ=4, HK=2,
+             bs=64, density=0.5, name="bs64_gqa_b2_d256"),
+    I.scaled(W["long_causal_blocksparse_h16_s32768_d256"], mode="index", Sq=520, Sk=520, HQ=4,
+             HK=2, topk=150, name="index_gqa_d256"),
+    I.scaled(W["long_causal_blocksparse_h16_s32768_d256"], Sq=200, Sk=450, HQ=2, HK=1,
+             causal=False, density=1.0, name="noncausal_sq_ne_sk_d256"),
 ]
 FULL = [W[k] for k in ("blocksparse_mha_s256_d64", "dense_full_b2_h16_s4096_d128",
                        "dense_causal_b2_h16_s4096_d128", "gqa_blocksparse_b2_hq32_hk8_s8192_d128",
