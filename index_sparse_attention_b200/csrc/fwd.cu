@@ -7,9 +7,11 @@
 // un-normalised P = exp(s - max), accumulate P V, final O = acc / sum.
 //
 // B200 design (one CTA per 128-query tile of one (batch, query head)):
-//   warp 0     TMA producer: Q once, then the K and V tiles of the ACTIVE key tiles
-//              only (the forward list), 128-byte swizzled, double-buffered when
-//              shared memory allows.
+//   warp 0     TMA producer: Q once, then the K tiles of the ACTIVE key tiles only
+//              (the forward list), 128-byte swizzled, double-buffered when shared
+//              memory allows;
+//   warp 6     TMA producer of the V tiles, so that a K load (which S waits for)
+//              never queues behind a V load that waits for the previous P V.
 //   warp 1     allocates 512 TMEM columns and issues the tcgen05 MMAs from one
 //              thread: S = Q K^T into one of two TMEM S buffers (so the next S is
 //              computed while the softmax works on the current one), and
@@ -41,7 +43,7 @@ struct FwdCfg {
   static constexpr int kVOff = kKOff + kKStages * kKBytes;
   static constexpr int kBarOff = kVOff + kVStages * kVBytes;
   static constexpr int kSmem = kBarOff + 256 + 1024;  // barriers + alignment slack
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 224;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kOCol = 256;
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
@@ -53,7 +55,7 @@ enum : int { kBQ = 0, kBKF = 1, kBKE = 3, kBVF = 5, kBVE = 7, kBSF = 9, kBPF = 1
              kBDrain = 14, kBOFin = 15, kNumBars = 16 };
 
 template <int DQK, int DV>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(224, 1)
     sparse_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
@@ -116,6 +118,8 @@ __global__ void __launch_bounds__(192, 1)
           tma_load_4d(sbase + C::kQOff + c * C::kPanel, &tm_q, BAR(kBQ), c * 64, mt * 128, h, b);
       }
       __syncwarp();
+      // K tiles: each one as soon as S of the tile that last used its buffer is done (V
+      // tiles have a producer warp of their own, so a K load never waits behind P V)
       for (int it = 0; it < n_iter; ++it) {
         const int nt = __shfl_sync(0xFFFFFFFFu, __ldg(list + it), 0);
         const int ks = it % C::kKStages, ku = it / C::kKStages;
@@ -127,6 +131,19 @@ __global__ void __launch_bounds__(192, 1)
                         c * 64, nt * 128, g, b);
         }
         __syncwarp();
+      }
+      if (*abort_flag && lane == 0) {
+        // Let the loads already issued land before the CTA may leave (time-limited).
+        mbar_wait_limited(BAR(kBQ), 0);
+        for (int it = max(0, n_iter - 2); it < n_iter; ++it)
+          mbar_wait_limited(BAR(kBKF + it % C::kKStages), (it / C::kKStages) & 1);
+      }
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------------ V producer
+    if (n_iter > 0) {
+      for (int it = 0; it < n_iter; ++it) {
+        const int nt = __shfl_sync(0xFFFFFFFFu, __ldg(list + it), 0);
         const int vs = it % C::kVStages, vu = it / C::kVStages;
         if (!warp_wait(BAR(kBVE + vs), (vu & 1) ^ 1, abort_flag, a.status)) break;
         if (elect_one()) {
@@ -138,12 +155,8 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
       }
       if (*abort_flag && lane == 0) {
-        // Let the loads already issued land before the CTA may leave (time-limited).
-        mbar_wait_limited(BAR(kBQ), 0);
-        for (int it = max(0, n_iter - 2); it < n_iter; ++it) {
-          mbar_wait_limited(BAR(kBKF + it % C::kKStages), (it / C::kKStages) & 1);
+        for (int it = max(0, n_iter - 2); it < n_iter; ++it)
           mbar_wait_limited(BAR(kBVF + it % C::kVStages), (it / C::kVStages) & 1);
-        }
       }
     }
   } else if (warp == 1) {
