@@ -230,17 +230,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
           for (int c = 0; c < 4; ++c) tma_load_4d(qs + c * kQPanel, tm_stage, BAR(kBQF + s), c * 64, m0, h, b);
         }
         __syncwarp();
-        // the tile of step it + 3 is requested into L2 now, so that its own load (issued
-        // when a stage frees up) mostly hits L2
-        if (it + kStages < n_iter) {
-          int hp, mp;
-          bool pp;
-          decode(it + kStages, hp, mp, pp);
-          mp = __shfl_sync(0xFFFFFFFFu, mp, 0);
-          if (elect_one())
-            for (int c = 0; c < 4; ++c) tma_prefetch_l2_4d(tm_stage, c * 64, mp, hp, b);
-          __syncwarp();
-        }
         // rank 1 frees a stage when dV is done, which can precede the elementwise warps'
         // read of the step's Delta: wait for them before overwriting it
         if (rank == 1 && it >= kStages &&
