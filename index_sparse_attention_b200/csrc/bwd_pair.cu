@@ -10,7 +10,8 @@
 // need 512 TMEM columns, everything one SM has.  Two CTAs that each recompute S^T and
 // dP^T for a head-dim half would do those contractions twice and have room for only
 // one Q/dO stage.  Here the two CTAs of a cluster split the work by role:
-//   rank 0 holds K and stages of Q: S^T = K Q^T, P^T = exp2(S^T scale log2e - LSE log2e)
+//   rank 0 holds K in TMEM (and K[:, 0:128] in shared memory) and stages of Q:
+//           S^T = K Q^T (K as the TMEM operand), P^T = exp2(S^T scale log2e - LSE log2e)
 //           with the element mask (bf16, into an exchange tile), dK += dS^T Q (all 256
 //           columns), dQ^T[0:128] = K[:, 0:128]^T dS^T;
 //   rank 1 holds V in TMEM, K[:, 128:256] and stages of dO: dP^T = V dO^T (V as the
@@ -18,7 +19,12 @@
 //           dV += P^T dO (all 256 columns), dQ^T[128:256] = K[:, 128:256]^T dS^T into
 //           the TMEM buffer the elementwise warps have just read dP^T from.
 // Each rank issues about the same tensor-core work per 64-query step, and a stage
-// holds only Q or only dO, so three stages fit on each rank.
+// holds only Q or only dO.  Both contractions over the full head dim read their
+// stationary operand from TMEM: with 256-wide heads a shared-memory operand would cost
+// 64 KB of shared-memory reads per step, the resource that bounds this kernel (the
+// tensor core reads at most 128 B/clk of operands from it, and the TMA loads, the
+// exchanges and the dQ staging share the same bandwidth).  Rank 0 keeps four Q stages
+// (its stages are held from the load to dK, across both exchanges), rank 1 three.
 //
 // Exchanges.  Per step, P^T (rank 0 -> 1) and dS^T (rank 1 -> 0) cross as one 16 KB
 // bulk copy each (cp.async.bulk shared::cta -> shared::cluster, no multicast) that
@@ -51,23 +57,26 @@ namespace sa {
 namespace pairbwd {
 
 constexpr int BM = 64;                      // queries per step
-constexpr int kStages = 3;                  // Q (rank 0) / dO (rank 1) stages
+constexpr int kStages0 = 4;                 // Q stages (rank 0)
+constexpr int kStages1 = 3;                 // dO stages (rank 1)
+constexpr int kMaxStages = 4;
 constexpr int kNX = 4;                      // exchange tiles per rank
 constexpr int kKPanel = 128 * 128;          // [128 rows x 64 cols] bf16 (16 KB)
 constexpr int kQPanel = BM * 128;           // [64 rows x 64 cols] bf16 (8 KB)
 constexpr int kStageBytes = 4 * kQPanel;    // one 64 x 256 tile (32 KB)
 constexpr int kTile = 128 * BM * 2;         // exchange tile [128 keys][64 q] bf16 (16 KB)
-// rank 0: K | 3 Q stages | 4 exchange tiles | lse2 per stage
+// rank 0: K columns 0..127 | 4 Q stages | 4 exchange tiles | lse2 per stage.  K columns
+// 128..255 pass through exchange tiles 0 and 1 on their way into TMEM.
 constexpr int kOffK0 = 0;
-constexpr int kOffStage0 = 64 * 1024;
-constexpr int kOffX0 = kOffStage0 + kStages * kStageBytes;
+constexpr int kOffStage0 = 32 * 1024;
+constexpr int kOffX0 = kOffStage0 + kStages0 * kStageBytes;
 constexpr int kOffL0 = kOffX0 + kNX * kTile;
 // rank 1: K columns 128..255 | 3 dO stages | 4 exchange tiles | dQ staging | delta per
 // stage.  V passes through stages 1 and 2 on its way into TMEM.
 constexpr int kOffK1 = 0;
 constexpr int kOffStage1 = 32 * 1024;
 constexpr int kOffV1 = kOffStage1 + kStageBytes;
-constexpr int kOffX1 = kOffStage1 + kStages * kStageBytes;
+constexpr int kOffX1 = kOffStage1 + kStages1 * kStageBytes;
 constexpr int kOffDQ1 = kOffX1 + kNX * kTile;
 constexpr int kOffL1 = kOffDQ1 + kTile;
 // barriers at the same offset on both ranks (a rank addresses the peer's barriers
@@ -75,12 +84,14 @@ constexpr int kOffL1 = kOffDQ1 + kTile;
 constexpr int kOffBar = kOffL0 + 1024;
 constexpr int kSmem = kOffBar + 512 + 1024;
 constexpr int kThreads = 448;
-static_assert(kOffL0 + kStages * BM * 4 <= kOffBar, "rank 0 shared-memory layout");
-static_assert(kOffL1 + kStages * BM * 4 <= kOffBar, "rank 1 shared-memory layout");
+static_assert(kOffL0 + kStages0 * BM * 4 <= kOffBar, "rank 0 shared-memory layout");
+static_assert(kOffL1 + kStages1 * BM * 4 <= kOffBar, "rank 1 shared-memory layout");
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
-// TMEM columns.  Rank 0: S^T buffers, dK, dQ^T.  Rank 1: dP^T buffers (each then holds
-// the step's dQ^T half), dV, V as the A operand (bf16, two per column).
-constexpr uint32_t kColS0 = 0;     // + 64 * (step % 3)
+// TMEM columns.  Rank 0: K as the A operand (bf16, two per column), one S^T buffer (the
+// elementwise warps release it as soon as they have loaded it), dK, dQ^T.  Rank 1: dP^T
+// buffers (each then holds the step's dQ^T half), dV, V as the A operand.
+constexpr uint32_t kColK0 = 0;
+constexpr uint32_t kColS0 = 128;
 constexpr uint32_t kColAcc0 = 192;
 constexpr uint32_t kColDQ0 = 448;
 constexpr uint32_t kColP1 = 0;     // + 64 * (step % 2)
@@ -88,25 +99,26 @@ constexpr uint32_t kColAcc1 = 128;
 constexpr uint32_t kColV1 = 384;
 constexpr uint32_t kTmemCols = 512;
 // how many steps S^T (rank 0) / dP^T (rank 1) may run ahead of the oldest dK / dV
-constexpr int kLookS0 = 2;
+constexpr int kLookS0 = 3;
 constexpr int kLookS1 = 1;
 
 enum : int {
   kBKV = 0,    // K / V (and rank 1's K half) loaded
-  kBVT = 1,    // rank 1: V copied into TMEM (256 threads)
-  kBQF = 2,    // [3] stage loaded
-  kBQE = 5,    // [3] stage free (commit after dK on rank 0, after dV on rank 1)
-  kBLF = 8,    // [3] per-stage LSE / Delta written (32 producer lanes)
-  kBSF = 11,   // [3] S^T / dP^T of step complete (commit), indexed by step % 3
-  kBEW = 14,   // [3] elementwise work of the step done (256 threads)
-  kBXF = 17,   // [4] exchange tile received (receiver's arrival + 16 KB)
-  kBXT = 21,   // [4] rank 0: own tile free after its dQ drain
-  kBXE = 25,   // [4] rank 0: rank 1's tile free (remote)
-  kBXS = 29,   // [4] rank 1: its dS^T copy has landed in rank 0 (remote)
-  kBPV = 33,   // [4] rank 1: dV has read P^T from the tile (commit)
-  kBDQF = 37,  // [2] dQ^T complete (commit); rank 0 uses slot 0 only
-  kBDQE = 39,  // [2] dQ^T drained from TMEM (128 threads)
-  kBFin = 41, kBDrain = 42, kNumBars = 43
+  kBVT = 1,    // K (rank 0) / V (rank 1) copied into TMEM (256 threads)
+  kBQF = 2,    // [4] stage loaded
+  kBQE = 6,    // [4] stage free (commit after dK on rank 0, after dV on rank 1)
+  kBLF = 10,   // [4] per-stage LSE / Delta written (32 producer lanes)
+  kBSF = 14,   // [4] S^T / dP^T of step complete (commit), indexed by step % stages
+  kBEW = 18,   // [4] elementwise work of the step done (256 threads)
+  kBXF = 22,   // [4] exchange tile received (receiver's arrival + 16 KB)
+  kBXT = 26,   // [4] rank 0: own tile free after its dQ drain
+  kBXE = 30,   // [4] rank 0: rank 1's tile free (remote)
+  kBXS = 34,   // [4] rank 1: its dS^T copy has landed in rank 0 (remote)
+  kBPV = 38,   // [4] rank 1: dV has read P^T from the tile (commit)
+  kBDQF = 42,  // [2] dQ^T complete (commit); rank 0 uses slot 0 only
+  kBDQE = 44,  // [2] dQ^T drained from TMEM (128 threads)
+  kBSR = 46,   // rank 0: the elementwise warps have loaded S^T (256 threads)
+  kBFin = 47, kBDrain = 48, kNumBars = 49
 };
 static_assert(8 * kNumBars + 8 <= 512, "barrier area");
 
@@ -141,11 +153,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
   const uint32_t off_x = rank == 0 ? kOffX0 : kOffX1;
   const uint32_t off_l = rank == 0 ? kOffL0 : kOffL1;
   const uint32_t col_acc = rank == 0 ? kColAcc0 : kColAcc1;
+  const int ns = rank == 0 ? kStages0 : kStages1;  // Q / dO stages of this rank
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(kBKV), 1);
     mbar_init(BAR(kBVT), 256);
-    for (int s = 0; s < 3; ++s) {
+    for (int s = 0; s < kMaxStages; ++s) {
       mbar_init(BAR(kBQF + s), 1);
       mbar_init(BAR(kBQE + s), 1);
       mbar_init(BAR(kBLF + s), 32);
@@ -163,6 +176,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       mbar_init(BAR(kBDQF + s), 1);
       mbar_init(BAR(kBDQE + s), 128);
     }
+    mbar_init(BAR(kBSR), 256);
     mbar_init(BAR(kBFin), 1);
     mbar_init(BAR(kBDrain), 1);
     *abort_flag = 0;
@@ -200,9 +214,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         prefetch_tensormap(&tm_do);
         prefetch_tensormap(&tm_dq);
         if (rank == 0) {
+          // K columns 0..127 stay in shared memory (the dQ^T operand); 128..255 land in
+          // exchange tiles 0 and 1 until the elementwise warps have copied K into TMEM
           mbar_arrive_expect_tx(BAR(kBKV), 4 * kKPanel);
           for (int c = 0; c < 4; ++c)
-            tma_load_4d(sbase + kOffK0 + c * kKPanel, &tm_k, BAR(kBKV), c * 64, nt * 128, g, b);
+            tma_load_4d(sbase + (c < 2 ? kOffK0 + c * kKPanel : kOffX0 + (c - 2) * kKPanel), &tm_k,
+                        BAR(kBKV), c * 64, nt * 128, g, b);
         } else {
           mbar_arrive_expect_tx(BAR(kBKV), 6 * kKPanel);
           for (int c = 0; c < 4; ++c)
@@ -219,7 +236,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         bool partial;
         decode(it, h, m0, partial);
         m0 = __shfl_sync(0xFFFFFFFFu, m0, 0);  // warp-uniform TMA coordinate
-        const int s = it % kStages, u = it / kStages;
+        const int s = it % ns, u = it / ns;
         if (!warp_wait(BAR(kBQE + s), (u & 1) ^ 1, abort_flag, a.status)) break;
         // rank 1: V occupies stages 1 and 2 until it has been copied into TMEM
         if (rank == 1 && (it == 1 || it == 2) && !warp_wait(BAR(kBVT), 0, abort_flag, a.status))
@@ -232,8 +249,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         __syncwarp();
         // rank 1 frees a stage when dV is done, which can precede the elementwise warps'
         // read of the step's Delta: wait for them before overwriting it
-        if (rank == 1 && it >= kStages &&
-            !warp_wait(BAR(kBEW + s), ((it - kStages) / kStages) & 1, abort_flag, a.status))
+        if (rank == 1 && it >= ns &&
+            !warp_wait(BAR(kBEW + s), ((it - ns) / ns) & 1, abort_flag, a.status))
           break;
         // rank 0: LSE in log2 units (+inf past Sq); rank 1: Delta (0 past Sq)
         float* ls = lbuf + s * BM;
@@ -252,8 +269,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       }
       if (lane == 0 && *abort_flag) {
         mbar_wait_limited(BAR(kBKV), 0);
-        for (int it = max(0, n_iter - kStages); it < n_iter; ++it)
-          mbar_wait_limited(BAR(kBQF + it % kStages), (it / kStages) & 1);
+        for (int it = max(0, n_iter - ns); it < n_iter; ++it)
+          mbar_wait_limited(BAR(kBQF + it % ns), (it / ns) & 1);
       }
     }
   } else if (warp == 1) {
@@ -264,14 +281,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       constexpr uint32_t idesc_s = idesc_bf16(128, BM, 0, 0);     // S^T / dP^T
       constexpr uint32_t idesc_acc = idesc_bf16(128, 256, 0, 1);  // dK / dV (tile K-major, stage MN-major)
       constexpr uint32_t idesc_dq = idesc_bf16(128, BM, 1, 1);    // dQ^T (both MN-major)
-      const uint64_t kd = sw128_desc(sbase + kOffK0, 16, 1024);   // rank 0: S^T A operand
       // dQ^T A operand: this rank's 128 head-dim rows of K (MN-major)
       const uint64_t kwd = sw128_desc(sbase + (rank == 0 ? kOffK0 : kOffK1), kKPanel, 1024);
       auto ready = [&](int k, int parity) {
         return __shfl_sync(0xFFFFFFFFu, mbar_test(BAR(k), parity) ? 1 : 0, 0) != 0;
       };
       bool ok = warp_wait(BAR(kBKV), 0, abort_flag, a.status);
-      if (rank == 1) ok = ok && warp_wait(BAR(kBVT), 0, abort_flag, a.status);
+      ok = ok && warp_wait(BAR(kBVT), 0, abort_flag, a.status);
       int js = 0;  // next S^T (rank 0) / dP^T (rank 1)
       int jv = 0;  // rank 1: next dV
       int jk = 0;  // next dK + dQ^T (rank 0) / dQ^T (rank 1)
@@ -295,7 +311,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
           tc_fence_after();
           const int xb = jv % kNX;
           const uint64_t xk = sw128_desc(sbase + off_x + xb * kTile, 16, 1024);
-          const uint64_t bmn = sw128_desc(sbase + off_stage + (jv % kStages) * kStageBytes, kQPanel, 1024);
+          const uint64_t bmn = sw128_desc(sbase + off_stage + (jv % ns) * kStageBytes, kQPanel, 1024);
           if (elect_one()) {
             // every reader of this phase has passed it (the elementwise warps read the
             // tile before P^T of step jv+4 can be sent): arm the barrier for step jv+4
@@ -305,7 +321,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
               umma_ss(tmem + col_acc, xk + ((kk * 32) >> 4), bmn + ((kk * 2048) >> 4), idesc_acc,
                       (jv > 0 || kk > 0) ? 1u : 0u);
             umma_commit(BAR(kBPV + xb));            // P^T read: dS^T may replace it
-            umma_commit(BAR(kBQE + jv % kStages));  // dO stage free (dP^T read it earlier)
+            umma_commit(BAR(kBQE + jv % ns));  // dO stage free (dP^T read it earlier)
           }
           __syncwarp();
           ++jv;
@@ -314,19 +330,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         // rank 0: dK += dS^T Q and dQ^T once dS^T has arrived and the last dQ^T has been
         // drained; rank 1: dQ^T once its elementwise warps have written dS^T
         if (rank == 0 ? (jk < jx && (jk == 0 || ready(kBDQE, (jk - 1) & 1)))
-                      : (jk < jv && ready(kBEW + jk % kStages, (jk / kStages) & 1))) {
+                      : (jk < jv && ready(kBEW + jk % ns, (jk / ns) & 1))) {
           tc_fence_after();
           const uint32_t xt = sbase + off_x + (jk % kNX) * kTile;
           const uint64_t xmn = sw128_desc(xt, kKPanel, 1024);  // exchange tile, MN-major B
           if (rank == 0) {
             const uint64_t xk = sw128_desc(xt, 16, 1024);      // exchange tile, K-major A
-            const uint64_t bmn = sw128_desc(sbase + off_stage + (jk % kStages) * kStageBytes, kQPanel, 1024);
+            const uint64_t bmn = sw128_desc(sbase + off_stage + (jk % ns) * kStageBytes, kQPanel, 1024);
             if (elect_one()) {
 #pragma unroll
               for (int kk = 0; kk < BM / 16; ++kk)
                 umma_ss(tmem + col_acc, xk + ((kk * 32) >> 4), bmn + ((kk * 2048) >> 4), idesc_acc,
                         (jk > 0 || kk > 0) ? 1u : 0u);
-              umma_commit(BAR(kBQE + jk % kStages));  // Q stage free
+              umma_commit(BAR(kBQE + jk % ns));  // Q stage free
             }
             __syncwarp();
           }
@@ -343,32 +359,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
           prog = true;
         }
         // S^T (rank 0) / dP^T (rank 1) of the next step: stage loaded, TMEM buffer free
-        // (rank 0: read by the elementwise warps; rank 1: its dQ^T drained), not too far
+        // (rank 0: loaded by the elementwise warps; rank 1: its dQ^T drained), not too far
         // ahead of the dK / dV stream
         if (js < n_iter && js <= (rank == 0 ? jk + kLookS0 : jv + kLookS1) &&
-            ready(kBQF + js % kStages, (js / kStages) & 1) &&
-            (rank == 0 ? (js < 3 || ready(kBEW + js % 3, ((js - 3) / 3) & 1))
+            ready(kBQF + js % ns, (js / ns) & 1) &&
+            (rank == 0 ? (js == 0 || ready(kBSR, (js - 1) & 1))
                        : (js < 2 || ready(kBDQE + (js & 1), ((js - 2) >> 1) & 1)))) {
           tc_fence_after();
-          const int s = js % kStages;
+          const int s = js % ns;
           const uint64_t bd = sw128_desc(sbase + off_stage + s * kStageBytes, 16, 1024);
+          // A = K (rank 0) / V (rank 1) from TMEM: 16 head-dim columns (8 TMEM columns)
+          // per k-step
+          const uint32_t d_col = rank == 0 ? kColS0 : kColP1 + 64 * (js & 1);
+          const uint32_t a_col = rank == 0 ? kColK0 : kColV1;
           if (elect_one()) {
-            if (rank == 0) {
 #pragma unroll
-              for (int kk = 0; kk < 16; ++kk) {
-                const uint32_t off_a = (kk >> 2) * kKPanel + (kk & 3) * 32;
-                const uint32_t off_b = (kk >> 2) * kQPanel + (kk & 3) * 32;
-                umma_ss(tmem + kColS0 + 64 * s, kd + (off_a >> 4), bd + (off_b >> 4), idesc_s,
-                        kk > 0 ? 1u : 0u);
-              }
-            } else {
-              // A = V from TMEM: 16 head-dim columns (8 TMEM columns) per k-step
-#pragma unroll
-              for (int kk = 0; kk < 16; ++kk) {
-                const uint32_t off_b = (kk >> 2) * kQPanel + (kk & 3) * 32;
-                umma_ts(tmem + kColP1 + 64 * (js & 1), tmem + kColV1 + kk * 8, bd + (off_b >> 4),
-                        idesc_s, kk > 0 ? 1u : 0u);
-              }
+            for (int kk = 0; kk < 16; ++kk) {
+              const uint32_t off_b = (kk >> 2) * kQPanel + (kk & 3) * 32;
+              umma_ts(tmem + d_col, tmem + a_col + kk * 8, bd + (off_b >> 4), idesc_s,
+                      kk > 0 ? 1u : 0u);
             }
             umma_commit(BAR(kBSF + s));
           }
@@ -404,15 +413,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     const float* lbuf = reinterpret_cast<const float*>(smem + off_l);
     const bool key_ok = j < a.Sk;
     bool ok = true;
-    if (rank == 1 && n_iter > 0) {
-      // V row r into TMEM (row r in lane r, head dims 2e, 2e+1 in column e): this half
-      // of the warps copies head dims [128 hc, 128 hc + 128) from the swizzled panels
+    if (n_iter > 0) {
+      // K (rank 0) / V (rank 1) row r into TMEM (row r in lane r, head dims 2e, 2e+1 in
+      // column e): this half of the warps copies head dims [128 hc, 128 hc + 128) from
+      // the swizzled panels
       const bool v_ok = __all_sync(0xFFFFFFFFu, mbar_wait(BAR(kBKV), 0, abort_flag, a.status));
       if (v_ok) {
 #pragma unroll
         for (int pl = 0; pl < 2; ++pl) {
           const int p = 2 * hc + pl;
-          const uint8_t* prow = smem + kOffV1 + p * kKPanel + r * 128;
+          const uint32_t panel = rank == 1 ? kOffV1 + p * kKPanel
+                                           : (p < 2 ? kOffK0 + p * kKPanel : kOffX0 + (p - 2) * kKPanel);
+          const uint8_t* prow = smem + panel + r * 128;
           uint32_t w[32];
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
@@ -422,12 +434,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
             w[4 * k + 2] = v.z;
             w[4 * k + 3] = v.w;
           }
-          tmem_st32(tl + kColV1 + p * 32, w);
+          tmem_st32(tl + (rank == 1 ? kColV1 : kColK0) + p * 32, w);
         }
         tmem_wait_st();
       }
       ok = v_ok;
-      fence_proxy_async_smem();  // the producer reloads these stages with TMA next
+      // rank 1: the producer reloads these stages with TMA next; rank 0: the exchange
+      // tiles are written by bulk copies later
+      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(BAR(kBVT));
     }
@@ -435,7 +449,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       int h, m0;
       bool partial;
       decode(it, h, m0, partial);
-      const int s = it % kStages, ph = (it / kStages) & 1;
+      const int s = it % ns, ph = (it / ns) & 1;
       const int xb = it % kNX, phx = (it / kNX) & 1;
       bool w_ok = mbar_wait(BAR(kBLF + s), ph, abort_flag, a.status);
       w_ok = w_ok && mbar_wait(BAR(kBSF + s), ph, abort_flag, a.status);
@@ -454,7 +468,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       const float* ls = lbuf + s * BM + 32 * hc;
       const uint32_t row_off = off_x + xb * kTile + r * 128;  // row r of own tile xb
       uint32_t s_u[32];
-      tmem_ld32(tl + (rank == 0 ? kColS0 + 64 * s : kColP1 + 64 * (it & 1)) + 32 * hc, s_u);
+      tmem_ld32(tl + (rank == 0 ? kColS0 : kColP1 + 64 * (it & 1)) + 32 * hc, s_u);
       uint32_t pk[16];
       if (rank == 0) {
         uint32_t cm = 0xFFFFFFFFu;
@@ -486,6 +500,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
           }
         }
         tmem_wait_ld();
+        // S^T is in registers: the buffer may take the next step's S^T
+        tc_fence_before();
+        mbar_arrive(BAR(kBSR));
         const float4* ls4 = reinterpret_cast<const float4*>(ls);
         const float sc = a.scale_log2;
 #pragma unroll
