@@ -231,6 +231,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       __syncwarp();
       float* lbuf = reinterpret_cast<float*>(smem + off_l);
       const CUtensorMap* tm_stage = rank == 0 ? &tm_q : &tm_do;
+      // rank 0: LSE in log2 units (+inf past Sq); rank 1: Delta (0 past Sq).  The values
+      // of step it+1 are loaded while step it's stage is being waited for and loaded, so
+      // that their latency stays off the issue path of the stage loads.
+      auto load_rows = [&](int it_, float (&v)[2]) {
+        int h_, m0_;
+        bool partial_;
+        decode(it_, h_, m0_, partial_);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int64_t i = m0_ + lane + 32 * k;
+          v[k] = rank == 0 ? INFINITY : 0.f;
+          if (i < a.Sq) {
+            const int64_t li = (static_cast<int64_t>(b) * a.HQ + h_) * a.Sq + i;
+            v[k] = rank == 0 ? __ldg(a.lse + li) * 1.4426950408889634f : __ldg(a.delta + li);
+          }
+        }
+      };
+      float rows[2];
+      load_rows(0, rows);
       for (int it = 0; it < n_iter; ++it) {
         int h, m0;
         bool partial;
@@ -252,20 +271,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         if (rank == 1 && it >= ns &&
             !warp_wait(BAR(kBEW + s), ((it - ns) / ns) & 1, abort_flag, a.status))
           break;
-        // rank 0: LSE in log2 units (+inf past Sq); rank 1: Delta (0 past Sq)
         float* ls = lbuf + s * BM;
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int q = lane + 32 * k;
-          const int64_t i = m0 + q;
-          float v = rank == 0 ? INFINITY : 0.f;
-          if (i < a.Sq) {
-            const int64_t li = (static_cast<int64_t>(b) * a.HQ + h) * a.Sq + i;
-            v = rank == 0 ? __ldg(a.lse + li) * 1.4426950408889634f : __ldg(a.delta + li);
-          }
-          ls[q] = v;
-        }
+        ls[lane] = rows[0];
+        ls[lane + 32] = rows[1];
         mbar_arrive(BAR(kBLF + s));
+        if (it + 1 < n_iter) load_rows(it + 1, rows);
       }
       if (lane == 0 && *abort_flag) {
         mbar_wait_limited(BAR(kBKV), 0);
