@@ -183,6 +183,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     // the first exchange tiles may arrive from the peer at any time
     for (int s = 0; s < kNX && s < n_iter; ++s) mbar_arrive_expect_tx(BAR(kBXF + s), kTile);
     fence_mbar_init();
+    // K / V do not depend on the tile list: start their loads before the TMEM
+    // allocation and the cluster handshake
+    if (n_iter > 0) {
+      if (rank == 0) {
+        // K columns 0..127 stay in shared memory (the dQ^T operand); 128..255 land in
+        // exchange tiles 0 and 1 until the elementwise warps have copied K into TMEM
+        mbar_arrive_expect_tx(BAR(kBKV), 4 * kKPanel);
+        for (int c = 0; c < 4; ++c)
+          tma_load_4d(sbase + (c < 2 ? kOffK0 + c * kKPanel : kOffX0 + (c - 2) * kKPanel), &tm_k,
+                      BAR(kBKV), c * 64, nt * 128, g, b);
+      } else {
+        mbar_arrive_expect_tx(BAR(kBKV), 6 * kKPanel);
+        for (int c = 0; c < 4; ++c)
+          tma_load_4d(sbase + kOffV1 + c * kKPanel, &tm_v, BAR(kBKV), c * 64, nt * 128, g, b);
+        for (int c = 2; c < 4; ++c)
+          tma_load_4d(sbase + kOffK1 + (c - 2) * kKPanel, &tm_k, BAR(kBKV), c * 64, nt * 128, g, b);
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -208,25 +226,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     // ------------------------------------------------------------------ producer
     if (n_iter > 0) {
       if (elect_one()) {
-        prefetch_tensormap(&tm_q);
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_v);
-        prefetch_tensormap(&tm_do);
+        prefetch_tensormap(rank == 0 ? &tm_q : &tm_do);
         prefetch_tensormap(&tm_dq);
-        if (rank == 0) {
-          // K columns 0..127 stay in shared memory (the dQ^T operand); 128..255 land in
-          // exchange tiles 0 and 1 until the elementwise warps have copied K into TMEM
-          mbar_arrive_expect_tx(BAR(kBKV), 4 * kKPanel);
-          for (int c = 0; c < 4; ++c)
-            tma_load_4d(sbase + (c < 2 ? kOffK0 + c * kKPanel : kOffX0 + (c - 2) * kKPanel), &tm_k,
-                        BAR(kBKV), c * 64, nt * 128, g, b);
-        } else {
-          mbar_arrive_expect_tx(BAR(kBKV), 6 * kKPanel);
-          for (int c = 0; c < 4; ++c)
-            tma_load_4d(sbase + kOffV1 + c * kKPanel, &tm_v, BAR(kBKV), c * 64, nt * 128, g, b);
-          for (int c = 2; c < 4; ++c)
-            tma_load_4d(sbase + kOffK1 + (c - 2) * kKPanel, &tm_k, BAR(kBKV), c * 64, nt * 128, g, b);
-        }
       }
       __syncwarp();
       float* lbuf = reinterpret_cast<float*>(smem + off_l);
