@@ -270,9 +270,15 @@ __global__ void __launch_bounds__(224, 1)
             if (!((wd[c >> 5] >> (c & 31)) & 1u)) x[c] = -INFINITY;
         }
       }
-      float mx = x[0];
+      // row max with eight independent chains (a single chain of 127 dependent fmaxf
+      // is latency bound: one softmax warp per SM sub-partition has nothing to hide it)
+      float mx8[8];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+      for (int k = 0; k < 8; ++k) mx8[k] = x[k];
+#pragma unroll
+      for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_tile = mx * a.scale_log2;
       // Lazy rescale: only when this row's max grows by more than 2^8; the decision is
       // taken per warp so that the warp-collective TMEM accesses stay converged.
@@ -305,7 +311,7 @@ __global__ void __launch_bounds__(224, 1)
       }
       const float m_eff = (m_run == -INFINITY) ? 0.f : m_run;
       const float sc = a.scale_log2;
-      float psum = 0.f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
 #pragma unroll
       for (int c0 = 0; c0 < 128; c0 += 32) {
         uint32_t pk[16];
@@ -313,12 +319,12 @@ __global__ void __launch_bounds__(224, 1)
         for (int e = 0; e < 16; ++e) {
           const float p0 = ex2(fmaf(x[c0 + 2 * e], sc, -m_eff));
           const float p1 = ex2(fmaf(x[c0 + 2 * e + 1], sc, -m_eff));
-          psum += p0 + p1;
+          ps[e & 3] += p0 + p1;
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tl + sb * 128 + c0 / 2, pk);
       }
-      l_run += psum;
+      l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(kBPF + sb));
