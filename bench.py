@@ -442,6 +442,97 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
+# -----------------------------------------------------------------------------------
+# Top-k selector (the producer of index mode's indices), measured on its own
+# -----------------------------------------------------------------------------------
+TOPK_METRIC = "top-k selector time per packed sequence (ms)"
+# the pages' standalone medians of their TileLang selector (hardware not stated), per
+# pack length: context only
+TOPK_PAGE_MS = {16384: 2.660752, 32768: 5.570000, 65536: 12.461776, 131072: 30.375248}
+
+
+def run_topk(args):
+    import torch
+
+    import index_sparse_attention_b200 as sa
+    from index_sparse_attention_b200 import _lib
+
+    L = _lib.load()
+    n, k = args.pack, args.k
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    host = I.topk_scores(n, n, seed=6000)
+    starts, ends = I.packed_causal_ranges(n)
+    scores = torch.from_numpy(host).to(dev)
+    st, en = torch.from_numpy(starts).to(dev), torch.from_numpy(ends).to(dev)
+    idx = torch.empty((n, k), dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    for _ in range(args.warmup):
+        sa.topk_select(scores, k, st, en, out_idx=idx, dev_status=status)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            sa.topk_select(scores, k, st, en, out_idx=idx, dev_status=status)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    assert int(status.item()) == 0
+    # end to end: pinned scores in, indices out, every step
+    pin_s = torch.from_numpy(host).pin_memory()
+    pin_i = torch.empty((n, k), dtype=torch.int32, pin_memory=True)
+    e_steps = max(1, min(args.steps, 5))
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e_steps):
+        scores.copy_(pin_s, non_blocking=True)
+        sa.topk_select(scores, k, st, en, out_idx=idx, dev_status=status)
+        pin_i.copy_(idx, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1) / e_steps
+    peaks, src = load_peaks()
+    read_bytes = 4 * int((ends.astype(np.int64) - starts).sum())
+    bytes_step = read_bytes + 4 * n * k
+    achieved = bytes_step / (ms * 1e-3) / 1e9
+    line = {
+        "metric": TOPK_METRIC, "value": ms, "unit": "ms", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"topk_pack{n}_k{k}", "rows": n, "cols": n, "k": k,
+                   "ranges": "one packed causal segment: row i selects from [0, i+1)",
+                   "scores": "standard normal fp32 (seed 6000)",
+                   "l2": f"inputs larger than L2: scores {4 * n * n / 2**20:.0f} MiB"},
+        "pages_context_ms": TOPK_PAGE_MS.get(n),
+        "roofline": {"kernel": "topk_kernel", "bound": "hbm", "achieved": achieved,
+                     "peak": float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])), "unit": "GB/s",
+                     "frac": achieved / float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
+                     "traffic": None,
+                     "algorithmic": "4 B per valid score read once + 4 B per output index"},
+        "e2e": {"value": e_ms, "unit": "ms", "h2d_bytes_per_step": 4 * n * n,
+                "d2h_bytes_per_step": 4 * n * k},
+        "gpu_launches": args.steps, "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline:
+        from oracle import topk as T
+        rng = np.random.default_rng(0)
+        t0, rows_done, work = time.perf_counter(), 0, 0
+        while time.perf_counter() - t0 < args.cpu_seconds:
+            r = int(rng.integers(n))
+            T.topk_select(host, k, starts, ends, rows=[r])
+            rows_done += 1
+            work += int(ends[r] - starts[r])
+        sec = time.perf_counter() - t0
+        total = int((ends.astype(np.int64) - starts).sum())
+        line["cpu_baseline"] = {
+            "value": 1e3 * sec * total / max(1, work), "unit": "ms", "cores": 1, "kind": "oracle",
+            "sample": f"{rows_done} random rows ({work} valid scores) in {sec:.1f} s, one numpy sort "
+                      "per row, scaled to the whole pack by its number of valid scores"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -455,8 +546,15 @@ def main():
                     help="CPU seconds per reference step (default: the run ends in ~2.5 min)")
     ap.add_argument("--seq", type=int, default=0,
                     help="override Sq = Sk (smaller profiling captures of the same kernels)")
+    ap.add_argument("--op", default="attention", choices=["attention", "topk"],
+                    help="topk: time the top-k selector alone on one packed sequence")
+    ap.add_argument("--pack", type=int, default=16384, help="--op topk: packed sequence length")
+    ap.add_argument("--k", type=int, default=2048, help="--op topk: k")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.op == "topk":
+        run_topk(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

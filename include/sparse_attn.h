@@ -196,6 +196,30 @@ int sparse_attn_bwd_noalloc(const sparse_attn_params *p, sa_stream_t stream);
  */
 int sparse_attn_set_timing_events(void *const *events);
 
+/* Largest k that topk_select supports. */
+#define SA_TOPK_MAX_K 4096
+
+/*
+ * topk_select -- xtuner PR #2096, "[Feature] Add optional TileLang Top-K selector", Main
+ * Changes 1: the Top-K stage that turns fp32 indexer scores into the int32 key indices
+ * (-1 for invalid positions) of index mode.
+ *   scores  device fp32 [rows][ld]; row r's candidates are the columns j of its valid
+ *           range [starts[r], ends[r]) (the whole row [0, cols) when starts / ends are
+ *           NULL).  Requires 0 <= starts[r] <= ends[r] <= cols, cols <= ld.
+ *   starts, ends  optional device int32 [rows].
+ *   k       1 <= k <= SA_TOPK_MAX_K.
+ *   out_idx device int32 [rows][k]: the columns of the k largest scores of the range,
+ *           largest first (the order of torch.topk with sorted=True); ties go to the
+ *           smaller column, -0 equals +0, NaN ranks above +inf; when the range holds
+ *           n < k columns, slots n..k-1 are -1.
+ *   out_val optional device fp32 [rows][k]: the selected scores (-inf in -1 slots).
+ * A row whose range is invalid yields k times -1 and sets bit 1 of *dev_status.  Needs
+ * no workspace.  Returns SA_ERR_INVALID for a bad size, k or null pointer.
+ */
+int topk_select(const float *scores, int64_t rows, int64_t cols, int64_t ld,
+                const int32_t *starts, const int32_t *ends, int32_t k, int32_t *out_idx,
+                float *out_val, int32_t *dev_status, sa_stream_t stream);
+
 /* Static description of an SA_* code. */
 const char *sparse_attn_error_string(int code);
 

@@ -15,7 +15,7 @@ from ._lib import SA_MODE_BLOCK, SA_MODE_DENSE, SA_MODE_INDEX, SA_TILE, SparseAt
 
 __all__ = ["BlockSparse", "block_mask_to_block_sparse", "index_to_block_sparse",
            "sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_bwd_workspace_size",
-           "sparse_attn_bwd_noalloc",
+           "sparse_attn_bwd_noalloc", "topk_select",
            "SparseAttnError", "SA_TILE"]
 
 
@@ -170,3 +170,27 @@ def sparse_attn_bwd_noalloc(q, k, v, o, lse, dout, sparse, softmax_scale=None, d
     _lib.check("sparse_attn_bwd_noalloc", L.sparse_attn_bwd_noalloc(ctypes.byref(p),
                                                                     _stream(q.device)))
     return dq, dk, dv
+
+
+def topk_select(scores, k, starts=None, ends=None, with_values=False, out_idx=None, out_val=None,
+                dev_status=None):
+    """Column indices (int32 [rows, k]) of the k largest fp32 scores of each row's range
+    [starts[r], ends[r]), largest first, ties to the smaller column, -1 past the number
+    of valid columns; with ``with_values`` also the selected scores (fp32 [rows, k])."""
+    L = _lib.load()
+    assert scores.dtype == torch.float32 and scores.dim() == 2 and scores.is_cuda
+    assert scores.stride(1) == 1
+    rows, cols = scores.shape
+    for t in (starts, ends):
+        if t is not None:
+            assert t.dtype == torch.int32 and t.is_contiguous() and t.numel() == rows
+    if out_idx is None:
+        out_idx = torch.empty((rows, k), dtype=torch.int32, device=scores.device)
+    if with_values and out_val is None:
+        out_val = torch.empty((rows, k), dtype=torch.float32, device=scores.device)
+    _lib.check("topk_select",
+               L.topk_select(_ptr(scores), rows, cols, scores.stride(0), _ptr(starts), _ptr(ends),
+                             k, _ptr(out_idx), _ptr(out_val), _ptr(dev_status),
+                             _stream(scores.device)))
+    return (out_idx, out_val) if with_values else out_idx
+

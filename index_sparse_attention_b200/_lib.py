@@ -20,6 +20,7 @@ SA_ERR_CUDA = -5
 SA_ERR_WORKSPACE = -7
 SA_ERR_SCRATCH_LIMIT = -8
 SA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+SA_TOPK_MAX_K = 4096
 
 SA_MODE_DENSE, SA_MODE_BLOCK, SA_MODE_INDEX = 0, 1, 2
 SA_TILE = 128
@@ -37,6 +38,7 @@ EXPORTS = (
     "sparse_attn_bwd_noalloc",
     "sparse_attn_set_timing_events",
     "sparse_attn_error_string",
+    "topk_select",
 )
 
 
@@ -89,6 +91,9 @@ def load():
     L.sparse_attn_bwd_noalloc.restype = ctypes.c_int
     L.sparse_attn_set_timing_events.argtypes = [vp]
     L.sparse_attn_set_timing_events.restype = ctypes.c_int
+    i64 = ctypes.c_int64
+    L.topk_select.argtypes = [vp, i64, i64, i64, vp, vp, ctypes.c_int32, vp, vp, vp, vp]
+    L.topk_select.restype = ctypes.c_int
     L.sparse_attn_error_string.argtypes = [ctypes.c_int]
     L.sparse_attn_error_string.restype = ctypes.c_char_p
     _lib = L

@@ -167,3 +167,36 @@ def make_inputs(w: Workload, with_grad: bool = True) -> Inputs:
     mask = block_mask(w) if w.mode == "block" else None
     idx = topk_indices(w) if w.mode == "index" else None
     return Inputs(w, q, k, v, do, mask, idx)
+
+
+# ---------------------------------------------------------------------------------
+# Top-k selector inputs: fp32 indexer scores of one packed sequence
+# ---------------------------------------------------------------------------------
+def packed_causal_ranges(L, segments=None):
+    """Per-row valid key ranges [start, end) of a packed causal sequence of length L
+    made of the given segment lengths (one segment by default): row i of a segment
+    [s, e) may attend to [s, i + 1)."""
+    segments = (L,) if segments is None else tuple(segments)
+    assert sum(segments) == L
+    starts = np.empty(L, np.int32)
+    ends = np.empty(L, np.int32)
+    s0 = 0
+    for n in segments:
+        starts[s0:s0 + n] = s0
+        ends[s0:s0 + n] = np.arange(s0 + 1, s0 + n + 1, dtype=np.int32)
+        s0 += n
+    return starts, ends
+
+
+def topk_scores(rows, cols, seed, dist="normal"):
+    """fp32 scores [rows, cols]: ``normal`` -- standard normal draws; ``concentrated``
+    -- 5 + 1e-3 * standard normal, all in one narrow band that shares its leading radix
+    digits, with many exact ties after rounding to fp32."""
+    g = np.random.default_rng(seed)
+    x = g.standard_normal((rows, cols), dtype=np.float32)
+    if dist == "concentrated":
+        x = (np.float32(5.0) + np.float32(1e-3) * x).astype(np.float32)
+    elif dist != "normal":
+        raise ValueError(dist)
+    return x
+
