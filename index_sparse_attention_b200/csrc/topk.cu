@@ -13,11 +13,15 @@
 //  1. Radix select of the k-th largest key in three digit passes (11, 11 and 10 bits):
 //     each pass histograms the keys that match the digits fixed so far (shared-memory
 //     atomics), and a block-wide scan from the top bin finds the bin holding the k-th
-//     key.  Every pass streams the row from global memory (L2 after the first pass);
-//     the row is read with coalesced loads and no candidate buffer can overflow.
-//  2. Gather: keys above the k-th key are appended in any order; keys equal to it are
-//     compacted in column order (warp ballots and a prefix over the warps) and only the
-//     first `need` of them are kept, so ties resolve to the smaller column.
+//     key.  Every pass streams the row from global memory (L2 after the first pass)
+//     with 16-byte loads, two in flight per thread, so no candidate buffer can
+//     overflow and a pass costs about two memory latencies for an 8K-column row.
+//  2. Gather: keys above the k-th key are appended in any order.  When every key equal
+//     to the k-th is needed (the count the last pass found equals the number still
+//     missing, the usual case), those are appended in any order too: the sort puts them
+//     in column order.  Otherwise the equal keys are compacted in column order (warp
+//     ballots and a prefix over the warps) and only the first `need` of them are kept,
+//     so ties resolve to the smaller column.
 //  3. Bitonic sort of the k winners (as 64-bit (key, ~column) words, descending) and the
 //     write of the indices (and optionally the scores).
 // Rows with no more valid columns than k skip step 1 and 2.
@@ -48,6 +52,37 @@ __device__ __forceinline__ uint64_t word(uint32_t key, int64_t col) {
   return (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(col));
 }
 
+// Calls f(i, key) for every element i < n of the row (any order across threads):
+// scalar loads up to the first 16-byte boundary, then float4 loads two per thread per
+// iteration, then the scalar tail.
+template <class F>
+__device__ __forceinline__ void for_each_key(const float* __restrict__ xr, int64_t n, F&& f) {
+  const int tid = threadIdx.x;
+  int64_t head = static_cast<int64_t>(((16u - (reinterpret_cast<uintptr_t>(xr) & 15u)) & 15u) >> 2);
+  if (head > n) head = n;
+  if (tid < head) f(static_cast<int64_t>(tid), score_key(__ldg(xr + tid)));
+  const float4* x4 = reinterpret_cast<const float4*>(xr + head);
+  const int64_t n4 = (n - head) >> 2;
+  for (int64_t q = tid; q < n4; q += 2 * kThreads) {
+    const float4 a = __ldg(x4 + q);
+    const bool has_b = q + kThreads < n4;
+    const float4 b = has_b ? __ldg(x4 + q + kThreads) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const int64_t i = head + 4 * q;
+    f(i, score_key(a.x));
+    f(i + 1, score_key(a.y));
+    f(i + 2, score_key(a.z));
+    f(i + 3, score_key(a.w));
+    if (has_b) {
+      const int64_t ib = i + 4 * kThreads;
+      f(ib, score_key(b.x));
+      f(ib + 1, score_key(b.y));
+      f(ib + 2, score_key(b.z));
+      f(ib + 3, score_key(b.w));
+    }
+  }
+  for (int64_t i = head + 4 * n4 + tid; i < n; i += kThreads) f(i, score_key(__ldg(xr + i)));
+}
+
 __global__ void __launch_bounds__(kThreads)
     topk_kernel(const float* __restrict__ x, int64_t ld, int64_t cols,
                 const int32_t* __restrict__ starts, const int32_t* __restrict__ ends, int k,
@@ -55,7 +90,7 @@ __global__ void __launch_bounds__(kThreads)
                 int32_t* status) {
   __shared__ uint32_t hist[2048];
   __shared__ uint32_t wsum[kWarps];
-  __shared__ uint32_t found[2];  // bin holding the k-th key, count of keys above it
+  __shared__ uint32_t found[3];  // bin holding the k-th key, keys above it, keys in it
   __shared__ uint32_t n_gt;
   extern __shared__ uint64_t sel[];  // kp sort words
 
@@ -77,17 +112,16 @@ __global__ void __launch_bounds__(kThreads)
   } else {
     // ---- radix select of the k-th largest key
     uint32_t prefix = 0u, pmask = 0u;
-    uint32_t need = static_cast<uint32_t>(k);
+    uint32_t need = static_cast<uint32_t>(k), n_eq = 0u;
 #pragma unroll 1
     for (int pass = 0; pass < 3; ++pass) {
       const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
       const int nb = pass < 2 ? 2048 : 1024;
       for (int bq = tid; bq < nb; bq += kThreads) hist[bq] = 0u;
       __syncthreads();
-      for (int64_t i = tid; i < n; i += kThreads) {
-        const uint32_t key = score_key(__ldg(xr + i));
+      for_each_key(xr, n, [&](int64_t, uint32_t key) {
         if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
-      }
+      });
       __syncthreads();
       // bins in descending order: thread t owns ranks [4t, 4t+4) (rank r = bin nb-1-r)
       const int per = nb / kThreads;  // 4 or 2
@@ -113,6 +147,7 @@ __global__ void __launch_bounds__(kThreads)
         if (e < per && above < need && above + c[e] >= need) {
           found[0] = static_cast<uint32_t>(nb - 1 - (tid * per + e));
           found[1] = above;
+          found[2] = c[e];
         }
         above += c[e];
       }
@@ -120,6 +155,7 @@ __global__ void __launch_bounds__(kThreads)
       prefix |= found[0] << shift;
       pmask |= static_cast<uint32_t>(nb - 1) << shift;
       need -= found[1];
+      n_eq = found[2];  // after the last pass: the number of keys equal to the k-th
       __syncthreads();  // found[] and wsum[] are rewritten by the next pass
     }
     // ---- gather: keys above the threshold in any order, equal keys in column order
@@ -127,6 +163,12 @@ __global__ void __launch_bounds__(kThreads)
     const uint32_t base_eq = static_cast<uint32_t>(k) - need;
     if (tid == 0) n_gt = 0u;
     __syncthreads();
+    if (n_eq == need) {
+      // every key >= the k-th is selected: append in any order
+      for_each_key(xr, n, [&](int64_t i, uint32_t key) {
+        if (key >= thr) sel[atomicAdd(&n_gt, 1u)] = word(key, st + i);
+      });
+    } else {
     uint32_t eq_seen = 0u;  // equal keys in the chunks before this one (uniform)
     for (int64_t c0 = 0; c0 < n; c0 += kThreads) {
       const int64_t i = c0 + tid;
@@ -149,13 +191,20 @@ __global__ void __launch_bounds__(kThreads)
       eq_seen += tot;
       __syncthreads();  // wsum[] is rewritten by the next chunk
     }
+    }
   }
   __syncthreads();
 
-  // ---- bitonic sort of sel[0, kp), descending
-  for (int size = 2; size <= kp; size <<= 1) {
+  // ---- bitonic sort of sel[0, ks), descending (ks: kp, or the power of two that
+  // holds a short row's n entries; the slots past them are empty and stay last)
+  int ks = kp;
+  if (n < k) {
+    ks = 2;
+    while (ks < n) ks <<= 1;
+  }
+  for (int size = 2; size <= ks; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int t = tid; t < (kp >> 1); t += kThreads) {
+      for (int t = tid; t < (ks >> 1); t += kThreads) {
         const int i = 2 * t - (t & (stride - 1));
         const int j = i + stride;
         const uint64_t a = sel[i], b = sel[j];
