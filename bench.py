@@ -327,7 +327,7 @@ def run_gpu(args):
         bsp = lists()
         sa.sparse_attn_fwd(g["q"], g["k"], g["v"], bsp, w.scale, o=o, lse=lse)
         sa.sparse_attn_bwd(g["q"], g["k"], g["v"], o, lse, g["do"], bsp, w.scale, dq=dq, dk=dk,
-                           dv=dv, workspace=ws)
+                           dv=dv, workspace=ws, deterministic=args.deterministic)
         return bsp
 
     bsp = step()
@@ -410,7 +410,9 @@ def run_gpu(args):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": workload_config(w, active),
+            "data": "synthetic",
+            "config": dict(workload_config(w, active),
+                           **({"backward": "deterministic"} if args.deterministic else {})),
             "pct_of_bf16_peak": 100.0 * (value / world) / peak,
             "pct_basis": f"bf16_tflops_sustained {peak:.1f} TFLOP/s ({peak_src})",
             "flop_per_step": flop_step, "kernel_ms": per_kernel,
@@ -546,6 +548,8 @@ def main():
                     help="CPU seconds per reference step (default: the run ends in ~2.5 min)")
     ap.add_argument("--seq", type=int, default=0,
                     help="override Sq = Sk (smaller profiling captures of the same kernels)")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="use the deterministic backward (fixed-order dQ accumulation)")
     ap.add_argument("--op", default="attention", choices=["attention", "topk"],
                     help="topk: time the top-k selector alone on one packed sequence")
     ap.add_argument("--pack", type=int, default=16384, help="--op topk: packed sequence length")

@@ -160,6 +160,20 @@ size_t sparse_attn_bwd_workspace_size(const sparse_attn_params *p);
 int sparse_attn_bwd(const sparse_attn_params *p, void *workspace, size_t workspace_bytes,
                     sa_stream_t stream);
 
+/*
+ * sparse_attn_bwd_deterministic -- the same backward with a bitwise reproducible dQ
+ * (the deterministic backward of sgl-flash-attn PR #28; fixed-order reduction).  dK and
+ * dV are accumulated in a fixed order in every mode; dQ, which many key-tile CTAs add
+ * into, is here accumulated in ascending key-tile order for every (batch, query head,
+ * query tile): a CTA waits for its turn on a counter in the workspace (same size as for
+ * sparse_attn_bwd).  Same arguments, outputs and errors as sparse_attn_bwd; results
+ * equal those of sparse_attn_bwd up to the rounding order of dQ, and two calls on the
+ * same inputs give identical bits.  Slower where several key tiles reach the same
+ * query tile at the same time.
+ */
+int sparse_attn_bwd_deterministic(const sparse_attn_params *p, void *workspace,
+                                  size_t workspace_bytes, sa_stream_t stream);
+
 /* Size of the fixed device scratch array used by sparse_attn_bwd_noalloc: 16 MiB. */
 #define SA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 

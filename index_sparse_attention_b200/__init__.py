@@ -134,8 +134,9 @@ def sparse_attn_bwd_workspace_size(q, k, v, sparse):
 
 
 def sparse_attn_bwd(q, k, v, o, lse, dout, sparse, softmax_scale=None, dq=None, dk=None,
-                    dv=None, workspace=None, dev_status=None):
-    """dQ, dK, dV (bf16, layouts of q, k, v) of sparse attention."""
+                    dv=None, workspace=None, dev_status=None, deterministic=False):
+    """dQ, dK, dV (bf16, layouts of q, k, v) of sparse attention; with
+    ``deterministic`` dQ is accumulated in a fixed order (bitwise reproducible)."""
     L = _lib.load()
     Dqk = q.shape[3]
     if softmax_scale is None:
@@ -147,9 +148,9 @@ def sparse_attn_bwd(q, k, v, o, lse, dout, sparse, softmax_scale=None, dq=None, 
     need = int(L.sparse_attn_bwd_workspace_size(ctypes.byref(p)))
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    fn = L.sparse_attn_bwd_deterministic if deterministic else L.sparse_attn_bwd
     _lib.check("sparse_attn_bwd",
-               L.sparse_attn_bwd(ctypes.byref(p), _ptr(workspace), workspace.numel(),
-                                 _stream(q.device)))
+               fn(ctypes.byref(p), _ptr(workspace), workspace.numel(), _stream(q.device)))
     return dq, dk, dv
 
 

@@ -35,6 +35,7 @@ EXPORTS = (
     "sparse_attn_fwd",
     "sparse_attn_bwd_workspace_size",
     "sparse_attn_bwd",
+    "sparse_attn_bwd_deterministic",
     "sparse_attn_bwd_noalloc",
     "sparse_attn_set_timing_events",
     "sparse_attn_error_string",
@@ -87,6 +88,8 @@ def load():
     L.sparse_attn_bwd_workspace_size.restype = ctypes.c_size_t
     L.sparse_attn_bwd.argtypes = [P_p, vp, ctypes.c_size_t, vp]
     L.sparse_attn_bwd.restype = ctypes.c_int
+    L.sparse_attn_bwd_deterministic.argtypes = [P_p, vp, ctypes.c_size_t, vp]
+    L.sparse_attn_bwd_deterministic.restype = ctypes.c_int
     L.sparse_attn_bwd_noalloc.argtypes = [P_p, vp]
     L.sparse_attn_bwd_noalloc.restype = ctypes.c_int
     L.sparse_attn_set_timing_events.argtypes = [vp]

@@ -190,27 +190,43 @@ extern "C" int sparse_attn_fwd(const sparse_attn_params* p, sa_stream_t stream) 
   return launch_fwd(a, m, reinterpret_cast<cudaStream_t>(stream));
 }
 
+// workspace layout: Delta fp32 [B][HQ][Sq] | dQ accumulator fp32 [B][Sq][HQ][Dqk] |
+// deterministic mode's turn counters int32 [B][HQ][Tm][2]
 extern "C" size_t sparse_attn_bwd_workspace_size(const sparse_attn_params* p) {
   if (!p || p->B <= 0 || p->HQ <= 0 || p->Sq <= 0 || p->Dqk <= 0) return 0;
   const size_t delta = sizeof(float) * static_cast<size_t>(p->B) * p->HQ * p->Sq;
   const size_t dq = sizeof(float) * static_cast<size_t>(p->B) * p->Sq * p->HQ * p->Dqk;
-  return round256(delta) + round256(dq);
+  const size_t sem = sizeof(int32_t) * 2 * static_cast<size_t>(p->B) * p->HQ *
+                     static_cast<size_t>((p->Sq + kTile - 1) / kTile);
+  return round256(delta) + round256(dq) + round256(sem);
 }
 
-extern "C" int sparse_attn_bwd(const sparse_attn_params* p, void* workspace,
-                               size_t workspace_bytes, sa_stream_t stream) {
+static int run_bwd(const sparse_attn_params* p, void* workspace, size_t workspace_bytes,
+                   sa_stream_t stream, int det) {
   AttnArgs a;
   int rc = fill_args(p, &a, true);
   if (rc) return rc;
   const size_t need = sparse_attn_bwd_workspace_size(p);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SA_ERR_WORKSPACE;
+  const size_t delta_b = round256(sizeof(float) * static_cast<size_t>(p->B) * p->HQ * p->Sq);
+  const size_t dq_b = round256(sizeof(float) * static_cast<size_t>(p->B) * p->Sq * p->HQ * p->Dqk);
   a.delta = static_cast<float*>(workspace);
-  a.dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                      round256(sizeof(float) * static_cast<size_t>(p->B) * p->HQ *
-                                               p->Sq));
+  a.dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + delta_b);
+  a.det = det;
+  a.sem = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + delta_b + dq_b);
   TensorMaps m;
   rc = fill_maps(p, &m, true);
   if (rc) return rc;
   if (!make_map_f32(&m.dq_acc, a.dq_acc, p->Dqk, p->Sq, p->HQ, p->B)) return SA_ERR_CUDA;
   return launch_bwd(a, m, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int sparse_attn_bwd(const sparse_attn_params* p, void* workspace,
+                               size_t workspace_bytes, sa_stream_t stream) {
+  return run_bwd(p, workspace, workspace_bytes, stream, 0);
+}
+
+extern "C" int sparse_attn_bwd_deterministic(const sparse_attn_params* p, void* workspace,
+                                             size_t workspace_bytes, sa_stream_t stream) {
+  return run_bwd(p, workspace, workspace_bytes, stream, 1);
 }

@@ -28,6 +28,7 @@
 // dK/dV/dQ is split over two CTAs, each recomputing S^T and dP^T.  Head dims 256/256
 // run on a 2-CTA cluster that splits the work instead (bwd_pair.cu).
 // Every mbarrier wait is bounded (see sa_device.cuh).
+#include "det_order.cuh"
 #include "sa_device.cuh"
 #include "sa_kernels.h"
 
@@ -42,7 +43,9 @@ namespace sa {
 __global__ void bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                const __nv_bfloat16* __restrict__ dout, float* __restrict__ delta,
                                float* __restrict__ dq_acc, int64_t rows, int64_t Sq, int HQ,
-                               int Dv, int Dqk) {
+                               int Dv, int Dqk, int32_t* __restrict__ sem, int64_t nsem) {
+  const int64_t gid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (sem && gid < nsem) sem[gid] = 0;  // deterministic mode's dQ turn counters
   const int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -554,6 +557,17 @@ __global__ void __launch_bounds__(448, 1)
       mbar_arrive(BAR(kBDQE + bi));
       float* stage = reinterpret_cast<float*>(smem + C::kDQOff);
       const uint32_t stage_s = sbase + C::kDQOff;
+      // deterministic mode: this CTA's turn on the query tile starts at the first add of
+      // its first 64-row half and ends after the last add of its second half
+      const int mt = m0 >> 7, qhalf = (m0 >> 6) & 1;
+      bool turn_ok = true;
+      if (a.det && qhalf == 0 && dtid == 0)
+        turn_ok = det_wait_turn(det_slot(a, b, h, mt, split), key_tile_rank(a, bg, mt, nt), abort_flag,
+                                a.status);
+      if (a.det && !named_bar_and(1, 128, turn_ok)) {
+        ok = false;
+        break;
+      }
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         // the previous reduce (this step's first half, or the last step's second half)
@@ -570,6 +584,7 @@ __global__ void __launch_bounds__(448, 1)
           bulk_commit_group();
         }
       }
+      if (a.det && qhalf == 1 && dtid == 0) det_pass_turn(det_slot(a, b, h, mt, split));
     }
     if (dtid == 0) bulk_wait_group0();  // every reduce has landed before the CTA ends
   }
@@ -630,9 +645,10 @@ int launch_bwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
     const int warps = 8;
     const int64_t blocks = (rows + warps - 1) / warps;
     record_event(2, st);
+    const int64_t nsem = a.det ? static_cast<int64_t>(a.B) * a.HQ * a.Tm * 2 : 0;
     bwd_pre_kernel<<<static_cast<unsigned>(blocks), warps * 32, 0, st>>>(
         static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.delta,
-        a.dq_acc, rows, a.Sq, a.HQ, a.Dv, a.Dqk);
+        a.dq_acc, rows, a.Sq, a.HQ, a.Dv, a.Dqk, a.det ? a.sem : nullptr, nsem);
     if (check_launch("backward preprocess launch")) return SA_ERR_CUDA;
   }
   int rc;

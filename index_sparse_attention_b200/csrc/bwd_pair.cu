@@ -48,6 +48,7 @@
 // queued batch would delay the contractions the exchange chain waits for.
 //
 // No TMA multicast and no multicast commit are used.  Every wait is bounded.
+#include "det_order.cuh"
 #include "sa_device.cuh"
 #include "sa_kernels.h"
 
@@ -671,6 +672,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       const uint32_t soff = rank == 0 ? kOffX0 + xb * kTile : kOffDQ1;
       float* stage = reinterpret_cast<float*>(smem + soff);
       const uint32_t stage_s = sbase + soff;
+      // deterministic mode: this CTA's turn on the query tile (its dQ column half) starts
+      // at the first add of its first 64-row half and ends after the last add of its
+      // second half
+      const int mt = m0 >> 7, qhalf = (m0 >> 6) & 1;
+      bool turn_ok = true;
+      if (a.det && qhalf == 0 && dtid == 0)
+        turn_ok = det_wait_turn(det_slot(a, b, h, mt, static_cast<int>(rank)),
+                                key_tile_rank(a, bg, mt, nt), abort_flag, a.status);
+      if (a.det && !named_bar_and(1, 128, turn_ok)) {
+        ok = false;
+        break;
+      }
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         // the previous reduce (this step's first half; on rank 1 also the last step's
@@ -690,6 +703,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
           bulk_commit_group();
         }
       }
+      if (a.det && qhalf == 1 && dtid == 0) det_pass_turn(det_slot(a, b, h, mt, static_cast<int>(rank)));
       // rank 0: the tile is free once the reduces have read it
       if (rank == 0 && dtid == 0) {
         bulk_wait_group_read0();

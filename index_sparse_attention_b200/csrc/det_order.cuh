@@ -1,0 +1,68 @@
+// det_order.cuh -- sequencing of the dQ reduce-adds for the deterministic backward.
+//
+// dQ is the one output that many CTAs add into (every key tile that a query tile
+// attends to contributes a partial dQ for it, as fp32 bulk reduce-adds into the
+// accumulator).  Floating-point addition is not associative, so the default backward's
+// dQ depends on the order in which those CTAs happen to finish.  In deterministic mode
+// the contributions to each (batch, query head, query tile, dQ column part) are added
+// in ascending key-tile order: a CTA waits until a counter equals the rank of its key
+// tile among the query tile's active key tiles, adds both 64-row halves, waits for its
+// adds to complete and increments the counter.  A CTA only waits for CTAs of smaller
+// key tiles of the same (batch, KV head), which the grid launches before it, so the
+// waits cannot form a cycle; every wait is bounded all the same.
+#pragma once
+
+#include "sa_device.cuh"
+#include "sa_kernels.h"
+
+namespace sa {
+
+// Rank of key tile nt among the active key tiles of query tile mt of (b, kv head) row
+// bg, in ascending order, from the forward lists (full tiles ascending, then partial
+// tiles ascending): two binary searches.
+__device__ __forceinline__ int key_tile_rank(const AttnArgs& a, int64_t bg, int mt, int nt) {
+  const int64_t row = bg * a.Tm + mt;
+  const int nf = __ldg(a.cnt + 2 * row), np = __ldg(a.cnt + 2 * row + 1);
+  const int32_t* lst = a.idx + row * a.Tn;
+  auto lower = [&](const int32_t* v, int n) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(v + mid) < nt) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+  };
+  return lower(lst, nf) + lower(lst + nf, np);
+}
+
+__device__ __forceinline__ int32_t* det_slot(const AttnArgs& a, int b, int h, int mt, int part) {
+  return a.sem + ((static_cast<int64_t>(b) * a.HQ + h) * a.Tm + mt) * 2 + part;
+}
+
+// Waits until the counter equals `rank` (bounded); then orders the caller's following
+// TMA reduce-adds after the acquire.  False on a timeout or an abort.
+__device__ __forceinline__ bool det_wait_turn(const int32_t* slot, int rank, volatile int* abort,
+                                              int32_t* status) {
+  const uint64_t t0 = globaltimer_ns();
+  while (ld_acquire_gpu(slot) != rank) {
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      report_status(status, kStatusTimeout);
+      return false;
+    }
+    __nanosleep(128);
+  }
+  fence_proxy_async_global();
+  return true;
+}
+
+// After the caller's last reduce-add of its turn: wait for the adds to complete, then
+// pass the turn on.
+__device__ __forceinline__ void det_pass_turn(int32_t* slot) {
+  bulk_wait_group0();
+  fence_proxy_async_global();
+  red_release_gpu_add(slot, 1);
+}
+
+}  // namespace sa

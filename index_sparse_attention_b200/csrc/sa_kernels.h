@@ -32,6 +32,11 @@ struct AttnArgs {
   float scale;       // softmax_scale
   float scale_log2;  // softmax_scale * log2(e)
   int32_t* status;
+  // deterministic backward: dQ contributions to each (b, query head, query tile, dQ
+  // column part) are added in ascending key-tile order, sequenced by sem
+  // [B][HQ][Tm][2] (backward workspace, zeroed by the preprocess)
+  int det;
+  int32_t* sem;
 };
 
 struct TensorMaps {

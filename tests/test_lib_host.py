@@ -78,10 +78,12 @@ def test_unsupported_and_inconsistent_shapes(lib):
 def test_bwd_workspace_is_checked_on_host(lib):
     p, s = _fake_params()
     need = lib.sparse_attn_bwd_workspace_size(ctypes.byref(p))
-    # Delta [1,4,256] fp32 and the dQ accumulator [1,256,4,128] fp32, each 256-B rounded
-    assert need == 4 * 256 * 4 + 256 * 4 * 128 * 4
-    assert lib.sparse_attn_bwd(ctypes.byref(p), None, 0, None) == _lib.SA_ERR_WORKSPACE
-    assert lib.sparse_attn_bwd(ctypes.byref(p), 0x2000, need - 1, None) == _lib.SA_ERR_WORKSPACE
+    # Delta [1,4,256] fp32, the dQ accumulator [1,256,4,128] fp32 and the deterministic
+    # mode's turn counters [1,4,2,2] int32, each 256-B rounded
+    assert need == 4 * 256 * 4 + 256 * 4 * 128 * 4 + 256
+    for fn in (lib.sparse_attn_bwd, lib.sparse_attn_bwd_deterministic):
+        assert fn(ctypes.byref(p), None, 0, None) == _lib.SA_ERR_WORKSPACE
+        assert fn(ctypes.byref(p), 0x2000, need - 1, None) == _lib.SA_ERR_WORKSPACE
 
 
 def test_block_mask_validation(lib):
