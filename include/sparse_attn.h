@@ -164,7 +164,7 @@ int sparse_attn_bwd(const sparse_attn_params *p, void *workspace, size_t workspa
  * sparse_attn_bwd_deterministic -- the same backward with a bitwise reproducible dQ
  * (the deterministic backward of sgl-flash-attn PR #28; fixed-order reduction).  dK and
  * dV are accumulated in a fixed order in every mode; dQ, which many key-tile CTAs add
- * into, is here accumulated in ascending key-tile order for every (batch, query head,
+ * into, is here accumulated in descending key-tile order for every (batch, query head,
  * query tile): a CTA waits for its turn on a counter in the workspace (same size as for
  * sparse_attn_bwd).  Same arguments, outputs and errors as sparse_attn_bwd; results
  * equal those of sparse_attn_bwd up to the rounding order of dQ, and two calls on the

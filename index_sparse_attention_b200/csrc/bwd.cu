@@ -164,7 +164,9 @@ __global__ void __launch_bounds__(448, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = static_cast<int>(blockIdx.x) % NSPLIT;
-  const int nt = static_cast<int>(blockIdx.x) / NSPLIT;
+  // deterministic mode launches the key tiles from the last one down (det_order.cuh)
+  const int nt = a.det ? a.Tn - 1 - static_cast<int>(blockIdx.x) / NSPLIT
+                       : static_cast<int>(blockIdx.x) / NSPLIT;
   const int g = blockIdx.y, b = blockIdx.z;
   const int G = a.HQ / a.HK;
   const int64_t bg = static_cast<int64_t>(b) * a.HK + g;
@@ -221,8 +223,14 @@ __global__ void __launch_bounds__(448, 1)
     const int rest = it - hh * per_head;
     const int k = rest >> 1;
     h = g * G + hh;
-    m0 = __ldg(tlist + k) * 128 + (rest & 1) * BM;
-    partial = k >= n_full;
+    if (a.det) {  // ascending query tiles (det_order.cuh)
+      int tile;
+      merged_tile(tlist, n_full, n_mt - n_full, k, tile, partial);
+      m0 = tile * 128 + (rest & 1) * BM;
+    } else {
+      m0 = __ldg(tlist + k) * 128 + (rest & 1) * BM;
+      partial = k >= n_full;
+    }
   };
 
   if (warp == 0) {
