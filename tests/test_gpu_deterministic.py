@@ -1,6 +1,7 @@
 """Deterministic backward (sparse_attn_bwd_deterministic): dQ, dK and dV are bitwise
-identical across calls and within the parity tolerance of the oracle, for the three
-backward kernels (D=128 single CTA, the 192/128 head-dim split, the 256/256 pair)."""
+identical across calls, within the parity tolerance of the oracle, and close to the
+default backward, for the three backward kernels (D=128 single CTA, the 192/128
+head-dim split, the 256/256 pair)."""
 import numpy as np
 import pytest
 
@@ -46,10 +47,10 @@ def test_bitwise_reproducible_and_correct(w):
     assert_close("dQ", bf16_to_f64(dq), rQ)
     assert_close("dK", bf16_to_f64(dk), rK)
     assert_close("dV", bf16_to_f64(dv), rV)
-    # the default backward gives the same dK, dV bits and dQ up to rounding order
+    # the default backward agrees up to summation order (the deterministic mode walks
+    # each key tile's query tiles in ascending order, the default full tiles first)
     dq2, dk2, dv2 = sa.sparse_attn_bwd(g["q"], g["k"], g["v"], o, lse, g["do"], bsp, w.scale,
                                        dev_status=status)
     torch.cuda.synchronize()
-    assert torch.equal(dk.view(torch.int16), dk2.view(torch.int16))
-    assert torch.equal(dv.view(torch.int16), dv2.view(torch.int16))
-    assert_close("dQ (default vs deterministic)", bf16_to_f64(dq2), bf16_to_f64(dq), tol=1e-2)
+    for name, x, y in (("dQ", dq2, dq), ("dK", dk2, dk), ("dV", dv2, dv)):
+        assert_close(f"{name} (default vs deterministic)", bf16_to_f64(x), bf16_to_f64(y), tol=1e-2)
