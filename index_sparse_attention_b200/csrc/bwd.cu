@@ -143,7 +143,9 @@ enum : int {
 // (one head-dim row of the dQ^T window per thread).
 // Bf16 P^T / dS^T of query columns [32h, 32h+32) are packed into TMEM columns
 // [32h, 32h+16) of the S^T / dP^T buffer, inside the range that half itself read.
-template <int DQK, int DV, int NSPLIT>
+// DET: deterministic mode (det_order.cuh), a separate instance so that the default
+// kernel carries none of its code.
+template <int DQK, int DV, int NSPLIT, bool DET>
 __global__ void __launch_bounds__(448, 1)
     sparse_bwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -165,7 +167,7 @@ __global__ void __launch_bounds__(448, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = static_cast<int>(blockIdx.x) % NSPLIT;
   // deterministic mode launches the key tiles from the last one down (det_order.cuh)
-  const int nt = a.det ? a.Tn - 1 - static_cast<int>(blockIdx.x) / NSPLIT
+  const int nt = DET ? a.Tn - 1 - static_cast<int>(blockIdx.x) / NSPLIT
                        : static_cast<int>(blockIdx.x) / NSPLIT;
   const int g = blockIdx.y, b = blockIdx.z;
   const int G = a.HQ / a.HK;
@@ -223,7 +225,7 @@ __global__ void __launch_bounds__(448, 1)
     const int rest = it - hh * per_head;
     const int k = rest >> 1;
     h = g * G + hh;
-    if (a.det) {  // ascending query tiles (det_order.cuh)
+    if constexpr (DET) {  // ascending query tiles (det_order.cuh)
       int tile;
       merged_tile(tlist, n_full, n_mt - n_full, k, tile, partial);
       m0 = tile * 128 + (rest & 1) * BM;
@@ -569,10 +571,10 @@ __global__ void __launch_bounds__(448, 1)
       // its first 64-row half and ends after the last add of its second half
       const int mt = m0 >> 7, qhalf = (m0 >> 6) & 1;
       bool turn_ok = true;
-      if (a.det && qhalf == 0 && dtid == 0)
+      if (DET && qhalf == 0 && dtid == 0)
         turn_ok = det_wait_turn(det_slot(a, b, h, mt, split), key_tile_rank(a, bg, mt, nt), abort_flag,
                                 a.status);
-      if (a.det && !named_bar_and(1, 128, turn_ok)) {
+      if (DET && !named_bar_and(1, 128, turn_ok)) {
         ok = false;
         break;
       }
@@ -592,7 +594,7 @@ __global__ void __launch_bounds__(448, 1)
           bulk_commit_group();
         }
       }
-      if (a.det && qhalf == 1 && dtid == 0) det_pass_turn(det_slot(a, b, h, mt, split));
+      if (DET && qhalf == 1 && dtid == 0) det_pass_turn(det_slot(a, b, h, mt, split));
     }
     if (dtid == 0) bulk_wait_group0();  // every reduce has landed before the CTA ends
   }
@@ -612,12 +614,12 @@ __global__ void __launch_bounds__(448, 1)
   }
 }
 
-template <int DQK, int DV, int NSPLIT>
-static int launch_bwd_main(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
+template <int DQK, int DV, int NSPLIT, bool DET>
+static int launch_bwd_main_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
   using C = BwdCfg<DQK, DV, NSPLIT>;
   static bool attr_set = false;
   if (!attr_set) {
-    const int rc = cuda_error(cudaFuncSetAttribute(sparse_bwd_kernel<DQK, DV, NSPLIT>,
+    const int rc = cuda_error(cudaFuncSetAttribute(sparse_bwd_kernel<DQK, DV, NSPLIT, DET>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                    C::kSmem),
                               "backward smem attribute");
@@ -625,10 +627,10 @@ static int launch_bwd_main(const AttnArgs& a, const TensorMaps& m, cudaStream_t 
     attr_set = true;
     if (std::getenv("SA_DEBUG")) {
       cudaFuncAttributes fa;
-      const cudaError_t qe = cudaFuncGetAttributes(&fa, sparse_bwd_kernel<DQK, DV, NSPLIT>);
+      const cudaError_t qe = cudaFuncGetAttributes(&fa, sparse_bwd_kernel<DQK, DV, NSPLIT, DET>);
       int occ = -1;
       const cudaError_t oe = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-          &occ, sparse_bwd_kernel<DQK, DV, NSPLIT>, C::kThreads, C::kSmem);
+          &occ, sparse_bwd_kernel<DQK, DV, NSPLIT, DET>, C::kThreads, C::kSmem);
       std::fprintf(stderr, "sparse_attn: attribute query %s, occupancy query %s -> %d\n",
                    cudaGetErrorName(qe), cudaGetErrorName(oe), occ);
       if (qe == cudaSuccess)
@@ -641,10 +643,16 @@ static int launch_bwd_main(const AttnArgs& a, const TensorMaps& m, cudaStream_t 
   }
   dim3 grid(a.Tn * NSPLIT, a.HK, a.B);
   record_event(3, st);
-  sparse_bwd_kernel<DQK, DV, NSPLIT><<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.v, m.dout,
+  sparse_bwd_kernel<DQK, DV, NSPLIT, DET><<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.v, m.dout,
                                                                            m.dq_acc, a);
   record_event(4, st);
   return check_launch("backward main kernel launch");
+}
+
+template <int DQK, int DV, int NSPLIT>
+static int launch_bwd_main(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
+  return a.det ? launch_bwd_main_t<DQK, DV, NSPLIT, true>(a, m, st)
+               : launch_bwd_main_t<DQK, DV, NSPLIT, false>(a, m, st);
 }
 
 int launch_bwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {

@@ -123,6 +123,9 @@ enum : int {
 };
 static_assert(8 * kNumBars + 8 <= 512, "barrier area");
 
+// DET: deterministic mode (det_order.cuh), a separate instance so that the default
+// kernel carries none of its code.
+template <bool DET>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     sparse_bwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_k,
@@ -142,7 +145,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
   // deterministic mode launches the key tiles from the last one down (det_order.cuh)
-  const int nt = a.det ? a.Tn - 1 - (static_cast<int>(blockIdx.x) >> 1)
+  const int nt = DET ? a.Tn - 1 - (static_cast<int>(blockIdx.x) >> 1)
                        : static_cast<int>(blockIdx.x) >> 1;
   const int g = blockIdx.y, b = blockIdx.z;
   const int G = a.HQ / a.HK;
@@ -221,7 +224,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     const int rest = it - hh * per_head;
     const int k = rest >> 1;
     h = g * G + hh;
-    if (a.det) {  // ascending query tiles (det_order.cuh)
+    if constexpr (DET) {  // ascending query tiles (det_order.cuh)
       int tile;
       merged_tile(tlist, n_full, n_mt - n_full, k, tile, partial);
       m0 = tile * 128 + (rest & 1) * BM;
@@ -685,10 +688,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       // second half
       const int mt = m0 >> 7, qhalf = (m0 >> 6) & 1;
       bool turn_ok = true;
-      if (a.det && qhalf == 0 && dtid == 0)
+      if (DET && qhalf == 0 && dtid == 0)
         turn_ok = det_wait_turn(det_slot(a, b, h, mt, static_cast<int>(rank)),
                                 key_tile_rank(a, bg, mt, nt), abort_flag, a.status);
-      if (a.det && !named_bar_and(1, 128, turn_ok)) {
+      if (DET && !named_bar_and(1, 128, turn_ok)) {
         ok = false;
         break;
       }
@@ -711,7 +714,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
           bulk_commit_group();
         }
       }
-      if (a.det && qhalf == 1 && dtid == 0) det_pass_turn(det_slot(a, b, h, mt, static_cast<int>(rank)));
+      if (DET && qhalf == 1 && dtid == 0) det_pass_turn(det_slot(a, b, h, mt, static_cast<int>(rank)));
       // rank 0: the tile is free once the reduces have read it
       if (rank == 0 && dtid == 0) {
         bulk_wait_group_read0();
@@ -741,10 +744,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
 
 }  // namespace pairbwd
 
-int launch_bwd_pair(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
+template <bool DET>
+static int launch_bwd_pair_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
   static bool attr_set = false;
   if (!attr_set) {
-    const int rc = cuda_error(cudaFuncSetAttribute(pairbwd::sparse_bwd_pair_kernel,
+    const int rc = cuda_error(cudaFuncSetAttribute(pairbwd::sparse_bwd_pair_kernel<DET>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                    pairbwd::kSmem),
                               "pair backward smem attribute");
@@ -753,10 +757,14 @@ int launch_bwd_pair(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
   }
   dim3 grid(a.Tn * 2, a.HK, a.B);
   record_event(3, st);
-  pairbwd::sparse_bwd_pair_kernel<<<grid, pairbwd::kThreads, pairbwd::kSmem, st>>>(
+  pairbwd::sparse_bwd_pair_kernel<DET><<<grid, pairbwd::kThreads, pairbwd::kSmem, st>>>(
       m.q, m.k, m.v, m.dout, m.dq_acc, a);
   record_event(4, st);
   return check_launch("pair backward kernel launch");
+}
+
+int launch_bwd_pair(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
+  return a.det ? launch_bwd_pair_t<true>(a, m, st) : launch_bwd_pair_t<false>(a, m, st);
 }
 
 }  // namespace sa
