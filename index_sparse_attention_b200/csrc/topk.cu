@@ -23,7 +23,11 @@
 //     ballots and a prefix over the warps) and only the first `need` of them are kept,
 //     so ties resolve to the smaller column.
 //  3. Bitonic sort of the k winners (as 64-bit (key, ~column) words, descending) and the
-//     write of the indices (and optionally the scores).
+//     write of the indices (and optionally the scores).  For 2048 or 4096 words each
+//     thread holds E = 4 or 8 consecutive words in registers: compare-exchanges whose
+//     partner is in the same thread run in registers, those whose partner is in the same
+//     warp use shuffles, and only those across warps go through shared memory (10 or 15
+//     of the 66 or 78 stages need a barrier).
 // Rows with no more valid columns than k skip step 1 and 2.
 #include "sa_device.cuh"
 #include "sa_kernels.h"
@@ -83,7 +87,77 @@ __device__ __forceinline__ void for_each_key(const float* __restrict__ xr, int64
   for (int64_t i = head + 4 * n4 + tid; i < n; i += kThreads) f(i, score_key(__ldg(xr + i)));
 }
 
-__global__ void __launch_bounds__(kThreads)
+// Descending bitonic sort of w[0, 512 * E) (see step 3 above); ends with the words back
+// in w and a barrier.
+template <int E>
+__device__ __forceinline__ void sort_desc_blocked(uint64_t* w) {
+  constexpr int kp = kThreads * E;
+  const int tid = threadIdx.x, lane = tid & 31;
+  uint64_t r[E];
+#pragma unroll
+  for (int u = 0; u < E; ++u) r[u] = w[tid * E + u];
+  for (int size = 2; size <= kp; size <<= 1) {
+    int stride = size >> 1;
+    if (stride >= 32 * E) {
+      // partners in other warps: through shared memory, one barrier per stage
+#pragma unroll
+      for (int u = 0; u < E; ++u) w[tid * E + u] = r[u];
+      __syncthreads();
+      for (; stride >= 32 * E; stride >>= 1) {
+        for (int t = tid; t < (kp >> 1); t += kThreads) {
+          const int i = 2 * t - (t & (stride - 1));
+          const int j = i + stride;
+          const uint64_t a = w[i], b = w[j];
+          const bool desc = (i & size) == 0;
+          if (desc ? (a < b) : (a > b)) {
+            w[i] = b;
+            w[j] = a;
+          }
+        }
+        __syncthreads();
+      }
+#pragma unroll
+      for (int u = 0; u < E; ++u) r[u] = w[tid * E + u];
+      __syncthreads();  // w is rewritten at the next size
+    }
+    // partners in other lanes of this warp: shuffles
+    for (; stride >= E; stride >>= 1) {
+      const int lm = stride / E;
+      const bool lower = (lane & lm) == 0;
+#pragma unroll
+      for (int u = 0; u < E; ++u) {
+        const uint64_t o = __shfl_xor_sync(0xFFFFFFFFu, r[u], lm);
+        const bool desc = ((tid * E + u) & size) == 0;
+        const bool keep_max = lower == desc;
+        const uint64_t hi = r[u] > o ? r[u] : o, lo = r[u] > o ? o : r[u];
+        r[u] = keep_max ? hi : lo;
+      }
+    }
+    // partners in this thread: registers (strides unrolled at compile time so that the
+    // words stay in registers)
+#pragma unroll
+    for (int sh = 2; sh >= 0; --sh) {
+      constexpr int kMaxSh = E == 8 ? 2 : 1;
+      if (sh > kMaxSh || (1 << sh) > stride) continue;
+      const int st = 1 << sh;
+#pragma unroll
+      for (int u = 0; u < E; ++u) {
+        if (u & st) continue;
+        const uint64_t a = r[u], b = r[u + st];
+        const bool desc = ((tid * E + u) & size) == 0;
+        if (desc ? (a < b) : (a > b)) {
+          r[u] = b;
+          r[u + st] = a;
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < E; ++u) w[tid * E + u] = r[u];
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kThreads, 4)
     topk_kernel(const float* __restrict__ x, int64_t ld, int64_t cols,
                 const int32_t* __restrict__ starts, const int32_t* __restrict__ ends, int k,
                 int kp, int32_t* __restrict__ out_idx, float* __restrict__ out_val,
@@ -202,19 +276,25 @@ __global__ void __launch_bounds__(kThreads)
     ks = 2;
     while (ks < n) ks <<= 1;
   }
-  for (int size = 2; size <= ks; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int t = tid; t < (ks >> 1); t += kThreads) {
-        const int i = 2 * t - (t & (stride - 1));
-        const int j = i + stride;
-        const uint64_t a = sel[i], b = sel[j];
-        const bool desc = (i & size) == 0;
-        if (desc ? (a < b) : (a > b)) {
-          sel[i] = b;
-          sel[j] = a;
+  if (ks == 4 * kThreads) {
+    sort_desc_blocked<4>(sel);
+  } else if (ks == 8 * kThreads) {
+    sort_desc_blocked<8>(sel);
+  } else {
+    for (int size = 2; size <= ks; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int t = tid; t < (ks >> 1); t += kThreads) {
+          const int i = 2 * t - (t & (stride - 1));
+          const int j = i + stride;
+          const uint64_t a = sel[i], b = sel[j];
+          const bool desc = (i & size) == 0;
+          if (desc ? (a < b) : (a > b)) {
+            sel[i] = b;
+            sel[j] = a;
+          }
         }
+        __syncthreads();
       }
-      __syncthreads();
     }
   }
 
