@@ -72,13 +72,18 @@ constexpr int kOffK0 = 0;
 constexpr int kOffStage0 = 32 * 1024;
 constexpr int kOffX0 = kOffStage0 + kStages0 * kStageBytes;
 constexpr int kOffL0 = kOffX0 + kNX * kTile;
-// rank 1: K columns 128..255 | 3 dO stages | 4 exchange tiles | dQ staging | delta per
-// stage.  V passes through stages 1 and 2 on its way into TMEM.
+// rank 1: K columns 128..255 | 3 dO stages | 2 P^T tiles | 3 dS^T tiles | dQ staging |
+// delta per stage.  V passes through stages 1 and 2 on its way into TMEM.
 constexpr int kOffK1 = 0;
 constexpr int kOffStage1 = 32 * 1024;
 constexpr int kOffV1 = kOffStage1 + kStageBytes;
-constexpr int kOffX1 = kOffStage1 + kStages1 * kStageBytes;
-constexpr int kOffDQ1 = kOffX1 + kNX * kTile;
+// rank 1: incoming P^T tiles (free once dV and the elementwise warps have read them) and
+// outgoing dS^T tiles (free once dQ^T has read them and their copy has landed in rank 0)
+constexpr int kNPI = 3;
+constexpr int kNDO = 2;
+constexpr int kOffPI1 = kOffStage1 + kStages1 * kStageBytes;
+constexpr int kOffDO1 = kOffPI1 + kNPI * kTile;
+constexpr int kOffDQ1 = kOffDO1 + kNDO * kTile;
 constexpr int kOffL1 = kOffDQ1 + kTile;
 // barriers at the same offset on both ranks (a rank addresses the peer's barriers
 // through its own offsets)
@@ -111,15 +116,15 @@ enum : int {
   kBLF = 10,   // [4] per-stage LSE / Delta written (32 producer lanes)
   kBSF = 14,   // [4] S^T / dP^T of step complete (commit), indexed by step % stages
   kBEW = 18,   // [4] elementwise work of the step done (256 threads)
-  kBXF = 22,   // [4] exchange tile received (receiver's arrival + 16 KB)
+  kBXF = 22,   // [4] rank 0: dS^T arrived in its tile; rank 1 [3]: P^T arrived
   kBXT = 26,   // [4] rank 0: own tile free after its dQ drain
-  kBXE = 30,   // [4] rank 0: rank 1's tile free (remote)
-  kBXS = 34,   // [4] rank 1: its dS^T copy has landed in rank 0 (remote)
-  kBPV = 38,   // [4] rank 1: dV has read P^T from the tile (commit)
-  kBDQF = 42,  // [2] dQ^T complete (commit); rank 0 uses slot 0 only
-  kBDQE = 44,  // [2] dQ^T drained from TMEM (128 threads)
-  kBSR = 46,   // rank 0: the elementwise warps have loaded S^T (256 threads)
-  kBFin = 47, kBDrain = 48, kNumBars = 49
+  kBXE = 30,   // [3] rank 0: rank 1's P^T tile free (remote)
+  kBDF = 33,   // [2] rank 1: dS^T tile free (dQ^T commit + remote arrival report)
+  kBPR = 35,   // [3] rank 1: P^T tile read (256 elementwise threads + the dV commit)
+  kBDQF = 38,  // [2] dQ^T complete (commit); rank 0 uses slot 0 only
+  kBDQE = 40,  // [2] dQ^T drained from TMEM (128 threads)
+  kBSR = 42,   // rank 0: the elementwise warps have loaded S^T (256 threads)
+  kBFin = 43, kBDrain = 44, kNumBars = 45
 };
 static_assert(8 * kNumBars + 8 <= 512, "barrier area");
 
@@ -156,7 +161,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
   const int32_t* tlist = a.tidx + trow * a.Tm;
   const int n_iter = G * n_mt * 2;  // (query head, query tile, 64-row half)
   const uint32_t off_stage = rank == 0 ? kOffStage0 : kOffStage1;
-  const uint32_t off_x = rank == 0 ? kOffX0 : kOffX1;
   const uint32_t off_l = rank == 0 ? kOffL0 : kOffL1;
   const uint32_t col_acc = rank == 0 ? kColAcc0 : kColAcc1;
   const int ns = rank == 0 ? kStages0 : kStages1;  // Q / dO stages of this rank
@@ -174,10 +178,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     for (int s = 0; s < kNX; ++s) {
       mbar_init(BAR(kBXF + s), 1);
       mbar_init(BAR(kBXT + s), 1);
-      mbar_init(BAR(kBXE + s), 1);
-      mbar_init(BAR(kBXS + s), 1);
-      mbar_init(BAR(kBPV + s), 1);
     }
+    for (int s = 0; s < kNPI; ++s) {
+      mbar_init(BAR(kBXE + s), 1);
+      mbar_init(BAR(kBPR + s), 257);
+    }
+    for (int s = 0; s < kNDO; ++s) mbar_init(BAR(kBDF + s), 2);
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(kBDQF + s), 1);
       mbar_init(BAR(kBDQE + s), 128);
@@ -187,7 +193,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     mbar_init(BAR(kBDrain), 1);
     *abort_flag = 0;
     // the first exchange tiles may arrive from the peer at any time
-    for (int s = 0; s < kNX && s < n_iter; ++s) mbar_arrive_expect_tx(BAR(kBXF + s), kTile);
+    for (int s = 0; s < (rank == 0 ? kNX : kNPI) && s < n_iter; ++s)
+      mbar_arrive_expect_tx(BAR(kBXF + s), kTile);
     fence_mbar_init();
     // K / V do not depend on the tile list: start their loads before the TMEM
     // allocation and the cluster handshake
@@ -315,6 +322,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       int jv = 0;  // rank 1: next dV
       int jk = 0;  // next dK + dQ^T (rank 0) / dQ^T (rank 1)
       int jx = 0;  // rank 0: next step whose dS^T arrival is reported back to rank 1
+      int jp = 0;  // rank 1: next step whose P^T tile is handed back to rank 0
       uint64_t t_last = globaltimer_ns();
       while (ok && jk < n_iter) {
         bool prog = false;
@@ -322,29 +330,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         // uses the tile next
         if (rank == 0 && jx < js && ready(kBXF + jx % kNX, (jx / kNX) & 1)) {
           if (elect_one()) {
-            mbar_arrive_remote_relaxed(mapa_shared(BAR(kBXS + jx % kNX), peer));
+            mbar_arrive_remote_relaxed(mapa_shared(BAR(kBDF + jx % kNDO), peer));
             if (jx + kNX < n_iter) mbar_arrive_expect_tx(BAR(kBXF + jx % kNX), kTile);
           }
           __syncwarp();
           ++jx;
           prog = true;
         }
+        // rank 1: hand a consumed P^T tile back to rank 0 (arm its barrier for the step
+        // after next first)
+        if (rank == 1 && jp < jv && ready(kBPR + jp % kNPI, (jp / kNPI) & 1)) {
+          if (jp + kNPI < n_iter && elect_one()) {
+            mbar_arrive_expect_tx(BAR(kBXF + jp % kNPI), kTile);
+            mbar_arrive_remote_relaxed(mapa_shared(BAR(kBXE + jp % kNPI), peer));
+          }
+          __syncwarp();
+          ++jp;
+          prog = true;
+        }
         // rank 1: dV += P^T dO as soon as P^T of the oldest step has arrived
-        if (rank == 1 && jv < js && ready(kBXF + jv % kNX, (jv / kNX) & 1)) {
+        if (rank == 1 && jv < js && ready(kBXF + jv % kNPI, (jv / kNPI) & 1)) {
           tc_fence_after();
-          const int xb = jv % kNX;
-          const uint64_t xk = sw128_desc(sbase + off_x + xb * kTile, 16, 1024);
+          const uint64_t xk = sw128_desc(sbase + kOffPI1 + (jv % kNPI) * kTile, 16, 1024);
           const uint64_t bmn = sw128_desc(sbase + off_stage + (jv % ns) * kStageBytes, kQPanel, 1024);
           if (elect_one()) {
-            // every reader of this phase has passed it (the elementwise warps read the
-            // tile before P^T of step jv+4 can be sent): arm the barrier for step jv+4
-            if (jv + kNX < n_iter) mbar_arrive_expect_tx(BAR(kBXF + xb), kTile);
 #pragma unroll
             for (int kk = 0; kk < BM / 16; ++kk)
               umma_ss(tmem + col_acc, xk + ((kk * 32) >> 4), bmn + ((kk * 2048) >> 4), idesc_acc,
                       (jv > 0 || kk > 0) ? 1u : 0u);
-            umma_commit(BAR(kBPV + xb));            // P^T read: dS^T may replace it
-            umma_commit(BAR(kBQE + jv % ns));  // dO stage free (dP^T read it earlier)
+            umma_commit(BAR(kBPR + jv % kNPI));  // P^T read by dV
+            umma_commit(BAR(kBQE + jv % ns));    // dO stage free (dP^T read it earlier)
           }
           __syncwarp();
           ++jv;
@@ -355,7 +370,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         if (rank == 0 ? (jk < jx && (jk == 0 || ready(kBDQE, (jk - 1) & 1)))
                       : (jk < jv && ready(kBEW + jk % ns, (jk / ns) & 1))) {
           tc_fence_after();
-          const uint32_t xt = sbase + off_x + (jk % kNX) * kTile;
+          // rank 0: the dS^T that arrived in its tile; rank 1: its own dS^T tile
+          const uint32_t xt = rank == 0 ? sbase + kOffX0 + (jk % kNX) * kTile
+                                        : sbase + kOffDO1 + (jk % kNDO) * kTile;
           const uint64_t xmn = sw128_desc(xt, kKPanel, 1024);  // exchange tile, MN-major B
           if (rank == 0) {
             const uint64_t xk = sw128_desc(xt, 16, 1024);      // exchange tile, K-major A
@@ -376,6 +393,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
               umma_ss(tmem + dq_col, kwd + ((kk * 2048) >> 4), xmn + ((kk * 2048) >> 4), idesc_dq,
                       kk > 0 ? 1u : 0u);
             umma_commit(BAR(kBDQF + (rank == 0 ? 0 : (jk & 1))));
+            if (rank == 1) umma_commit(BAR(kBDF + jk % kNDO));  // dS^T tile read by dQ^T
           }
           __syncwarp();
           ++jk;
@@ -481,7 +499,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         if (it >= kNX)
           w_ok = w_ok && mbar_wait(BAR(kBXT + xb), phx ^ 1, abort_flag, a.status);
       } else {
-        w_ok = w_ok && mbar_wait(BAR(kBXF + xb), phx, abort_flag, a.status);  // P^T arrived
+        w_ok = w_ok && mbar_wait(BAR(kBXF + it % kNPI), (it / kNPI) & 1, abort_flag,
+                                 a.status);  // P^T arrived
       }
       if (!__all_sync(0xFFFFFFFFu, w_ok)) {
         ok = false;
@@ -489,7 +508,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       }
       tc_fence_after();
       const float* ls = lbuf + s * BM + 32 * hc;
-      const uint32_t row_off = off_x + xb * kTile + r * 128;  // row r of own tile xb
+      // row r of the tile written (rank 0: own tile xb; rank 1: dS^T tile it % 3)
+      const uint32_t row_off = (rank == 0 ? kOffX0 + xb * kTile : kOffDO1 + (it % kNDO) * kTile) +
+                               r * 128;
       uint32_t s_u[32];
       tmem_ld32(tl + (rank == 0 ? kColS0 : kColP1 + 64 * (it & 1)) + 32 * hc, s_u);
       uint32_t pk[16];
@@ -555,23 +576,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         // one thread copies the tile into rank 1's tile xb once every row is in and that
         // tile is free (rank 1 is done with step it-4 there)
         if (threadIdx.x == 64 && mbar_wait(BAR(kBEW + s), ph, abort_flag, a.status) &&
-            (it < kNX || mbar_wait(BAR(kBXE + xb), phx ^ 1, abort_flag, a.status))) {
-          bulk_copy_to_cluster(mapa_shared(sbase + kOffX1 + xb * kTile, peer),
-                               sbase + kOffX0 + xb * kTile, kTile, mapa_shared(BAR(kBXF + xb), peer));
+            (it < kNPI ||
+             mbar_wait(BAR(kBXE + it % kNPI), ((it / kNPI) & 1) ^ 1, abort_flag, a.status))) {
+          bulk_copy_to_cluster(mapa_shared(sbase + kOffPI1 + (it % kNPI) * kTile, peer),
+                               sbase + kOffX0 + xb * kTile, kTile,
+                               mapa_shared(BAR(kBXF + it % kNPI), peer));
         }
       } else {
-        // P^T row (copied in by rank 0)
+        // P^T row (copied in by rank 0); once read, the tile may go back to rank 0
+        const uint32_t pi_off = kOffPI1 + (it % kNPI) * kTile + r * 128;
         uint32_t pw[16];
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
           const int c = hc * 4 + c4;
-          const uint4 v = *reinterpret_cast<const uint4*>(smem + row_off + ((c ^ (r & 7)) << 4));
+          const uint4 v = *reinterpret_cast<const uint4*>(smem + pi_off + ((c ^ (r & 7)) << 4));
           pw[4 * c4] = v.x;
           pw[4 * c4 + 1] = v.y;
           pw[4 * c4 + 2] = v.z;
           pw[4 * c4 + 3] = v.w;
         }
         tmem_wait_ld();
+        mbar_arrive(BAR(kBPR + it % kNPI));
         const float4* dl4 = reinterpret_cast<const float4*>(ls);
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
@@ -588,9 +613,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
           pk[2 * e4] = pack_bf16x2(dsv[0], dsv[1]);
           pk[2 * e4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
         }
-        // dV of this step must have read P^T before dS^T replaces it in the tile
-        const bool pv_ok = mbar_wait(BAR(kBPV + xb), phx, abort_flag, a.status);
-        if (!__all_sync(0xFFFFFFFFu, pv_ok)) {
+        // dS^T tile it % 3: dQ^T of step it-3 has read it and its copy has landed in rank 0
+        const bool df_ok =
+            it < kNDO || mbar_wait(BAR(kBDF + it % kNDO), ((it / kNDO) & 1) ^ 1, abort_flag, a.status);
+        if (!__all_sync(0xFFFFFFFFu, df_ok)) {
           ok = false;
           break;
         }
@@ -607,7 +633,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         // (that tile held P^T of this step, which rank 1 has already received)
         if (threadIdx.x == 64 && mbar_wait(BAR(kBEW + s), ph, abort_flag, a.status)) {
           bulk_copy_to_cluster(mapa_shared(sbase + kOffX0 + xb * kTile, peer),
-                               sbase + kOffX1 + xb * kTile, kTile, mapa_shared(BAR(kBXF + xb), peer));
+                               sbase + kOffDO1 + (it % kNDO) * kTile, kTile,
+                               mapa_shared(BAR(kBXF + xb), peer));
         }
       }
     }
@@ -676,10 +703,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(BAR(kBDQE + qb));
-      // rank 1: its tile xb is free once dQ^T has read it (done) and its dS^T copy has
-      // landed in rank 0; tell rank 0, which sends P^T of step it+4 into it
-      if (rank == 1 && dtid == 0 && mbar_wait(BAR(kBXS + xb), phx, abort_flag, a.status))
-        mbar_arrive_remote_relaxed(mapa_shared(BAR(kBXE + xb), peer));
       const uint32_t soff = rank == 0 ? kOffX0 + xb * kTile : kOffDQ1;
       float* stage = reinterpret_cast<float*>(smem + soff);
       const uint32_t stage_s = sbase + soff;
