@@ -146,8 +146,13 @@ int fill_maps(const sparse_attn_params* p, TensorMaps* m, bool backward) {
   if (!make_map(&m->q, p->q, p->Dqk, p->Sq, p->HQ, p->B, qrows)) return SA_ERR_CUDA;
   if (!make_map(&m->k, p->k, p->Dqk, p->Sk, p->HK, p->B, 128)) return SA_ERR_CUDA;
   if (!make_map(&m->v, p->v, p->Dv, p->Sk, p->HK, p->B, 128)) return SA_ERR_CUDA;
+  // O output of the forward (written by TMA stores in 128-row boxes)
+  if (!backward && !make_map(&m->o, p->o, p->Dv, p->Sq, p->HQ, p->B, 128)) return SA_ERR_CUDA;
   if (backward && !make_map(&m->dout, p->dout, p->Dv, p->Sq, p->HQ, p->B, qrows))
     return SA_ERR_CUDA;
+  // dK / dV outputs (written by TMA stores in 128-row boxes)
+  if (backward && !make_map(&m->dk, p->dk, p->Dqk, p->Sk, p->HK, p->B, 128)) return SA_ERR_CUDA;
+  if (backward && !make_map(&m->dv, p->dv, p->Dv, p->Sk, p->HK, p->B, 128)) return SA_ERR_CUDA;
   return SA_OK;
 }
 

@@ -136,7 +136,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                            const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v,
                            const __grid_constant__ CUtensorMap tm_do,
-                           const __grid_constant__ CUtensorMap tm_dq, const AttnArgs a) {
+                           const __grid_constant__ CUtensorMap tm_dq,
+                           const __grid_constant__ CUtensorMap tm_dk,
+                           const __grid_constant__ CUtensorMap tm_dv, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -645,10 +647,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       have = __all_sync(0xFFFFFFFFu, w_ok);
       tc_fence_after();
     }
-    // rank 0 stores dK (times softmax_scale), rank 1 stores dV
-    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(rank == 0 ? a.dk : a.dv) +
-                         ((static_cast<int64_t>(b) * a.Sk + j) * a.HK + g) * 256;
+    // rank 0 stores dK (times softmax_scale), rank 1 stores dV: the rows go to the idle
+    // stages as four [128 keys][64 dims] 128-byte-swizzled panels (the output map's box)
+    // and leave by four TMA stores, which drop rows past Sk
     const float sc = rank == 0 ? a.scale : 1.f;
+    const uint32_t ep = off_stage;
     for (int c = 32 * hc; c < 256; c += 64) {
       uint32_t v[32];
       if (have) {
@@ -658,16 +661,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = 0u;
       }
-      if (key_ok) {
-        uint32_t pq[16];
+      uint32_t pq[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pq[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
-        uint4* dst = reinterpret_cast<uint4*>(out + c);
+      for (int e = 0; e < 16; ++e)
+        pq[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
+      // columns [c, c+32) = 16-byte chunks (c % 64) / 8 .. +3 of row r in panel c / 64
+      uint8_t* prow = smem + ep + (c >> 6) * kKPanel + r * 128;
+      const int ch0 = (c & 63) >> 3;
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          dst[e] = make_uint4(pq[4 * e], pq[4 * e + 1], pq[4 * e + 2], pq[4 * e + 3]);
-      }
+      for (int e = 0; e < 4; ++e)
+        *reinterpret_cast<uint4*>(prow + (((ch0 + e) ^ (r & 7)) << 4)) =
+            make_uint4(pq[4 * e], pq[4 * e + 1], pq[4 * e + 2], pq[4 * e + 3]);
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(2, 256);
+    if (threadIdx.x == 64) {
+      const CUtensorMap* om = rank == 0 ? &tm_dk : &tm_dv;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) tma_store_4d(om, sbase + ep + p * kKPanel, p * 64, nt * 128, g, b);
+      bulk_commit_group();
+      bulk_wait_group_read0();  // the stages are read before the CTA may leave
     }
   } else {
     // ------------------------------------------------------------------ dQ drain
@@ -781,7 +794,7 @@ static int launch_bwd_pair_t(const AttnArgs& a, const TensorMaps& m, cudaStream_
   dim3 grid(a.Tn * 2, a.HK, a.B);
   record_event(3, st);
   pairbwd::sparse_bwd_pair_kernel<DET><<<grid, pairbwd::kThreads, pairbwd::kSmem, st>>>(
-      m.q, m.k, m.v, m.dout, m.dq_acc, a);
+      m.q, m.k, m.v, m.dout, m.dq_acc, m.dk, m.dv, a);
   record_event(4, st);
   return check_launch("pair backward kernel launch");
 }

@@ -58,7 +58,8 @@ template <int DQK, int DV>
 __global__ void __launch_bounds__(224, 1)
     sparse_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_o, const AttnArgs a) {
   using C = FwdCfg<DQK, DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -337,8 +338,9 @@ __global__ void __launch_bounds__(224, 1)
     }
     const bool have_o = n_iter > 0 && ok;  // warp-uniform
     const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
-    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) +
-                          ((b * a.Sq + i) * a.HQ + h) * static_cast<int64_t>(DV);
+    // O rows go to the Q buffer (idle once the last P V is done: every S MMA came
+    // before it) as [128 rows][64 cols] 128-byte-swizzled panels, the output map's box,
+    // and leave by TMA stores, which drop rows past Sq
 #pragma unroll 1
     for (int c = 0; c < DV; c += 32) {
       uint32_t ov[32];
@@ -349,17 +351,26 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) ov[e] = 0u;
       }
-      if (row_ok) {
-        uint32_t pk[16];
+      uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv,
-                              __uint_as_float(ov[2 * e + 1]) * inv);
-        uint4* dst = reinterpret_cast<uint4*>(orow + c);
+      for (int e = 0; e < 16; ++e)
+        pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
+      // columns [c, c+32) = 16-byte chunks (c % 64) / 8 .. +3 of row r in panel c / 64
+      uint8_t* prow = smem + C::kQOff + (c >> 6) * C::kPanel + r * 128;
+      const int ch0 = (c & 63) >> 3;
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-      }
+      for (int e = 0; e < 4; ++e)
+        *reinterpret_cast<uint4*>(prow + (((ch0 + e) ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(1, 128);
+    if (threadIdx.x == 64) {
+#pragma unroll
+      for (int p = 0; p < DV / 64; ++p)
+        tma_store_4d(&tm_o, sbase + C::kQOff + p * C::kPanel, p * 64, mt * 128, h, b);
+      bulk_commit_group();
+      bulk_wait_group_read0();  // the Q buffer is read before the CTA may leave
     }
     if (row_ok) {
       const float m_eff = (m_run == -INFINITY) ? 0.f : m_run;
@@ -390,7 +401,7 @@ static int launch_fwd_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st)
   }
   dim3 grid(a.Tm, a.HQ, a.B);
   record_event(0, st);
-  sparse_fwd_kernel<DQK, DV><<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.v, a);
+  sparse_fwd_kernel<DQK, DV><<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.v, m.o, a);
   record_event(1, st);
   return check_launch("forward kernel launch");
 }

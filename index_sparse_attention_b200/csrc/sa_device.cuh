@@ -178,6 +178,17 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
+// Store of a shared-memory tile (laid out as the map's box, with the map's swizzle) into
+// global memory through a tensor map; parts of the box outside the tensor are not
+// written.  Part of the calling thread's current bulk-async group.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                                             int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group"
+      " [%0, {%2, %3, %4, %5}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
 // Element-wise add of a shared-memory tile into global memory through a tensor map
 // (the tile's layout is the map's box, innermost dimension contiguous).  Part of
 // the calling thread's current bulk-async group.

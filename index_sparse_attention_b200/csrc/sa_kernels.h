@@ -40,7 +40,7 @@ struct AttnArgs {
 };
 
 struct TensorMaps {
-  CUtensorMap q, k, v, dout, dq_acc;
+  CUtensorMap q, k, v, dout, dq_acc, dk, dv, o;
 };
 
 // Caller-owned events recorded around the launches (see sparse_attn_set_timing_events);
