@@ -151,7 +151,9 @@ __global__ void __launch_bounds__(448, 1)
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_do,
-                      const __grid_constant__ CUtensorMap tm_dq, const AttnArgs a) {
+                      const __grid_constant__ CUtensorMap tm_dq,
+                      const __grid_constant__ CUtensorMap tm_dk,
+                      const __grid_constant__ CUtensorMap tm_dv, const AttnArgs a) {
   using C = BwdCfg<DQK, DV, NSPLIT>;
   constexpr int BM = C::kBM;
   extern __shared__ uint8_t smem_raw[];
@@ -497,18 +499,15 @@ __global__ void __launch_bounds__(448, 1)
       have = __all_sync(0xFFFFFFFFu, w_ok);
       tc_fence_after();
     }
-    __nv_bfloat16* dkrow = reinterpret_cast<__nv_bfloat16*>(a.dk) +
-                           ((static_cast<int64_t>(b) * a.Sk + j) * a.HK + g) * dqk_real;
-    __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(a.dv) +
-                           ((static_cast<int64_t>(b) * a.Sk + j) * a.HK + g) * dv_real;
-    // the two halves of the elementwise warps store alternating 32-column chunks
+    // The rows go to the idle stages as [128 keys][64 dims] 128-byte-swizzled panels
+    // (dK's, then dV's; the output maps' box) and leave by TMA stores, which drop rows
+    // past Sk; panels past the real head dim are not stored.  The two halves of the
+    // elementwise warps fill alternating 32-column chunks.
     for (int pass = 0; pass < 2; ++pass) {
       const int n = pass == 0 ? kcn : vcn;
-      const int d0 = pass == 0 ? kc0 : vc0;
-      const int dreal = pass == 0 ? dqk_real : dv_real;
       const uint32_t col = pass == 0 ? C::kColDK : C::kColDV;
       const float sc = pass == 0 ? a.scale : 1.f;
-      __nv_bfloat16* out = pass == 0 ? dkrow : dvrow;
+      const uint32_t pbase = C::kQOff + (pass == 0 ? 0 : (kcn / 64) * C::kKPanel);
       for (int c = 32 * hc; c < n; c += 64) {
         uint32_t v[32];
         if (have) {
@@ -518,17 +517,31 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] = 0u;
         }
-        if (key_ok && d0 + c < dreal) {
-          uint32_t pk[16];
+        uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
-          uint4* dst = reinterpret_cast<uint4*>(out + d0 + c);
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
+        // columns [c, c+32) = 16-byte chunks (c % 64) / 8 .. +3 of row r in panel c / 64
+        uint8_t* prow = smem + pbase + (c >> 6) * C::kKPanel + r * 128;
+        const int ch0 = (c & 63) >> 3;
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-        }
+        for (int e = 0; e < 4; ++e)
+          *reinterpret_cast<uint4*>(prow + (((ch0 + e) ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
       }
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(2, 256);
+    if (threadIdx.x == 64) {
+      for (int pp = 0; pp < kcn / 64; ++pp)
+        if (kc0 + 64 * pp < dqk_real)
+          tma_store_4d(&tm_dk, sbase + C::kQOff + pp * C::kKPanel, kc0 + 64 * pp, nt * 128, g, b);
+      for (int pp = 0; pp < vcn / 64; ++pp)
+        if (vc0 + 64 * pp < dv_real)
+          tma_store_4d(&tm_dv, sbase + C::kQOff + (kcn / 64 + pp) * C::kKPanel, vc0 + 64 * pp,
+                       nt * 128, g, b);
+      bulk_commit_group();
+      bulk_wait_group_read0();  // the stages are read before the CTA may leave
     }
   } else {
     // ------------------------------------------------------------------ dQ drain
@@ -643,8 +656,8 @@ static int launch_bwd_main_t(const AttnArgs& a, const TensorMaps& m, cudaStream_
   }
   dim3 grid(a.Tn * NSPLIT, a.HK, a.B);
   record_event(3, st);
-  sparse_bwd_kernel<DQK, DV, NSPLIT, DET><<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.v, m.dout,
-                                                                           m.dq_acc, a);
+  sparse_bwd_kernel<DQK, DV, NSPLIT, DET><<<grid, C::kThreads, C::kSmem, st>>>(
+      m.q, m.k, m.v, m.dout, m.dq_acc, m.dk, m.dv, a);
   record_event(4, st);
   return check_launch("backward main kernel launch");
 }
