@@ -124,7 +124,11 @@ enum : int {
   kBDQF = 38,  // [2] dQ^T complete (commit); rank 0 uses slot 0 only
   kBDQE = 40,  // [2] dQ^T drained from TMEM (128 threads)
   kBSR = 42,   // rank 0: the elementwise warps have loaded S^T (256 threads)
-  kBFin = 43, kBDrain = 44, kNumBars = 45
+  kBFin = 43, kBDrain = 44,
+  kBQH = 45,   // [2][4] exchange rows 32q..32q+31 of a step written (the 64 threads of
+               // quarter q), by step parity: a warp reaches step it+2 only after every
+               // elementwise thread has passed step it (S^T / dP^T of it+2 wait for that)
+  kNumBars = 53
 };
 static_assert(8 * kNumBars + 8 <= 512, "barrier area");
 
@@ -191,6 +195,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       mbar_init(BAR(kBDQE + s), 128);
     }
     mbar_init(BAR(kBSR), 256);
+    for (int q = 0; q < 8; ++q) mbar_init(BAR(kBQH + q), 64);
     mbar_init(BAR(kBFin), 1);
     mbar_init(BAR(kBDrain), 1);
     *abort_flag = 0;
@@ -574,15 +579,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         }
         fence_proxy_async_smem();
         tc_fence_before();
+        mbar_arrive(BAR(kBQH + (it & 1) * 4 + quarter));
         mbar_arrive(BAR(kBEW + s));
-        // one thread copies the tile into rank 1's tile xb once every row is in and that
-        // tile is free (rank 1 is done with step it-4 there)
-        if (threadIdx.x == 64 && mbar_wait(BAR(kBEW + s), ph, abort_flag, a.status) &&
+        // each quarter's 32 rows (4 KB) go to rank 1's P^T tile as soon as its two warps
+        // have written them and that tile is free (rank 1 is done with step it-3 there):
+        // four copies in flight instead of one
+        if (hc == 0 && lane == 0 &&
+            mbar_wait(BAR(kBQH + (it & 1) * 4 + quarter), (it >> 1) & 1, abort_flag, a.status) &&
             (it < kNPI ||
              mbar_wait(BAR(kBXE + it % kNPI), ((it / kNPI) & 1) ^ 1, abort_flag, a.status))) {
-          bulk_copy_to_cluster(mapa_shared(sbase + kOffPI1 + (it % kNPI) * kTile, peer),
-                               sbase + kOffX0 + xb * kTile, kTile,
-                               mapa_shared(BAR(kBXF + it % kNPI), peer));
+          bulk_copy_to_cluster(
+              mapa_shared(sbase + kOffPI1 + (it % kNPI) * kTile + quarter * (kTile / 4), peer),
+              sbase + kOffX0 + xb * kTile + quarter * (kTile / 4), kTile / 4,
+              mapa_shared(BAR(kBXF + it % kNPI), peer));
         }
       } else {
         // P^T row (copied in by rank 0); once read, the tile may go back to rank 0
@@ -630,13 +639,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         }
         fence_proxy_async_smem();
         tc_fence_before();
+        mbar_arrive(BAR(kBQH + (it & 1) * 4 + quarter));
         mbar_arrive(BAR(kBEW + s));
-        // one thread copies the dS^T tile into rank 0's tile xb once every row is in
+        // each quarter's 32 rows of dS^T go to rank 0's tile xb as soon as they are in
         // (that tile held P^T of this step, which rank 1 has already received)
-        if (threadIdx.x == 64 && mbar_wait(BAR(kBEW + s), ph, abort_flag, a.status)) {
-          bulk_copy_to_cluster(mapa_shared(sbase + kOffX0 + xb * kTile, peer),
-                               sbase + kOffDO1 + (it % kNDO) * kTile, kTile,
-                               mapa_shared(BAR(kBXF + xb), peer));
+        if (hc == 0 && lane == 0 &&
+            mbar_wait(BAR(kBQH + (it & 1) * 4 + quarter), (it >> 1) & 1, abort_flag, a.status)) {
+          bulk_copy_to_cluster(mapa_shared(sbase + kOffX0 + xb * kTile + quarter * (kTile / 4), peer),
+                               sbase + kOffDO1 + (it % kNDO) * kTile + quarter * (kTile / 4),
+                               kTile / 4, mapa_shared(BAR(kBXF + xb), peer));
         }
       }
     }
