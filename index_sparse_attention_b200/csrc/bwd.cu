@@ -167,11 +167,16 @@ __global__ void __launch_bounds__(448, 1)
   auto BAR = [&](int k) { return bar0 + 8u * static_cast<uint32_t>(k); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Default: key tiles of one head run together (they share that head's Q / dO in L2).
+  // Deterministic mode: key tiles from the last one down (det_order.cuh) with the heads
+  // interleaved, so that the key tiles that wait for one another's dQ turns are spread
+  // out in time (measured: 8.3 -> 5.8 ms at S=32768, D=256).
   const int split = static_cast<int>(blockIdx.x) % NSPLIT;
+  const int lin = static_cast<int>(blockIdx.x) / NSPLIT;
+  const int ord = DET ? lin / a.HK : lin;
   // deterministic mode launches the key tiles from the last one down (det_order.cuh)
-  const int nt = DET ? a.Tn - 1 - static_cast<int>(blockIdx.x) / NSPLIT
-                       : static_cast<int>(blockIdx.x) / NSPLIT;
-  const int g = blockIdx.y, b = blockIdx.z;
+  const int nt = DET ? a.Tn - 1 - ord : ord;
+  const int g = DET ? lin - ord * a.HK : static_cast<int>(blockIdx.y), b = blockIdx.z;
   const int G = a.HQ / a.HK;
   const int64_t bg = static_cast<int64_t>(b) * a.HK + g;
   const int64_t trow = bg * a.Tn + nt;
@@ -654,7 +659,7 @@ static int launch_bwd_main_t(const AttnArgs& a, const TensorMaps& m, cudaStream_
                      fa.maxDynamicSharedSizeBytes, C::kThreads, C::kSmem);
     }
   }
-  dim3 grid(a.Tn * NSPLIT, a.HK, a.B);
+  const dim3 grid = DET ? dim3(a.Tn * NSPLIT * a.HK, 1, a.B) : dim3(a.Tn * NSPLIT, a.HK, a.B);
   record_event(3, st);
   sparse_bwd_kernel<DQK, DV, NSPLIT, DET><<<grid, C::kThreads, C::kSmem, st>>>(
       m.q, m.k, m.v, m.dout, m.dq_acc, m.dk, m.dv, a);

@@ -155,10 +155,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
-  // deterministic mode launches the key tiles from the last one down (det_order.cuh)
-  const int nt = DET ? a.Tn - 1 - (static_cast<int>(blockIdx.x) >> 1)
-                       : static_cast<int>(blockIdx.x) >> 1;
-  const int g = blockIdx.y, b = blockIdx.z;
+  // One cluster per (key tile, head).  Default: key tiles of one head run together
+  // (they share that head's Q / dO in L2).  Deterministic mode: key tiles from the last
+  // one down (det_order.cuh) with the heads interleaved, so that the key tiles that wait
+  // for one another's dQ turns are spread out in time.
+  const int cl = static_cast<int>(blockIdx.x) >> 1;
+  const int ord = DET ? cl / a.HK : cl;
+  const int nt = DET ? a.Tn - 1 - ord : ord;
+  const int g = DET ? cl - ord * a.HK : static_cast<int>(blockIdx.y), b = blockIdx.z;
   const int G = a.HQ / a.HK;
   const int64_t bg = static_cast<int64_t>(b) * a.HK + g;
   const int64_t trow = bg * a.Tn + nt;
@@ -802,7 +806,7 @@ static int launch_bwd_pair_t(const AttnArgs& a, const TensorMaps& m, cudaStream_
     if (rc) return rc;
     attr_set = true;
   }
-  dim3 grid(a.Tn * 2, a.HK, a.B);
+  const dim3 grid = DET ? dim3(a.Tn * 2 * a.HK, 1, a.B) : dim3(a.Tn * 2, a.HK, a.B);
   record_event(3, st);
   pairbwd::sparse_bwd_pair_kernel<DET><<<grid, pairbwd::kThreads, pairbwd::kSmem, st>>>(
       m.q, m.k, m.v, m.dout, m.dq_acc, m.dk, m.dv, a);
