@@ -714,7 +714,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       int h, m0;
       bool partial;
       decode(it, h, m0, partial);
-      const int xb = it % kNX, phx = (it / kNX) & 1;
+      const int xb = it % kNX;
       const int qb = rank == 0 ? 0 : (it & 1);
       // the four drain warps leave together (they share named barrier 1 below)
       const bool w_ok = mbar_wait(BAR(kBDQF + qb), rank == 0 ? (it & 1) : ((it >> 1) & 1),
