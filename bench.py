@@ -74,11 +74,22 @@ def bwd_kernel_name(w):
     return f"sparse_bwd_kernel<{inst.get((w.Dqk, w.Dv), '?')}>"
 
 
-def bwd_source_sha():
+def source_code_sha(paths):
+    """Hash of the code in `paths`: whole-line comments, blank lines and indentation are
+    left out, so that a comment edit keeps a committed measurement of the code valid."""
     h = hashlib.sha256()
-    for f in ("bwd.cu", "bwd_pair.cu", "sa_device.cuh"):
-        h.update(open(os.path.join(ROOT, "index_sparse_attention_b200", "csrc", f), "rb").read())
+    for p in paths:
+        with open(p, encoding="utf-8") as fh:
+            for line in fh:
+                t = line.strip()
+                if t and not t.startswith("//"):
+                    h.update(t.encode("utf-8") + b"\n")
     return h.hexdigest()[:16]
+
+
+def bwd_source_sha():
+    return source_code_sha(os.path.join(ROOT, "index_sparse_attention_b200", "csrc", f)
+                           for f in ("bwd.cu", "bwd_pair.cu", "sa_device.cuh"))
 
 
 def profiled_traffic(workload):

@@ -26,18 +26,23 @@
 // exchanges and the dQ staging share the same bandwidth).  Rank 0 keeps four Q stages
 // (its stages are held from the load to dK, across both exchanges), rank 1 three.
 //
-// Exchanges.  Per step, P^T (rank 0 -> 1) and dS^T (rank 1 -> 0) cross as one 16 KB
-// bulk copy each (cp.async.bulk shared::cta -> shared::cluster, no multicast) that
-// completes its bytes on the receiver's barrier XF; the receiver arms XF itself (one
-// local arrival expecting 16 KB) for the step that will use the tile next, so a sender
-// issues nothing but the copy.  Each rank has four exchange tiles, step it using tile
-// it % 4: on rank 0 it stages P^T, then receives dS^T, then stages the dQ drain; on
-// rank 1 it receives P^T and is overwritten by dS^T once dV has read it (rank 1 stages
-// its dQ drain in a buffer of its own).  A copy signals only its receiver, so the
-// receivers report back with relaxed remote arrivals, which order no data (the readers
-// have finished when they are sent):
-//   XS[b] on rank 1: its dS^T copy from tile b has landed in rank 0;
-//   XE[b] on rank 0: rank 1's tile b is free again (dQ^T has read it, and XS[b] came).
+// Exchanges.  Per step, P^T (rank 0 -> 1) and dS^T (rank 1 -> 0) cross as bulk copies
+// (cp.async.bulk shared::cta -> shared::cluster, no multicast) of 4 KB each, one per
+// 32-row quarter of the 16 KB tile, issued as soon as that quarter's two warps have
+// written it (barriers QH).  They complete their bytes on the receiver's barrier XF; the
+// receiver arms XF itself (one local arrival expecting 16 KB) for the step that will use
+// the tile next, so a sender issues nothing but the copies.
+//   rank 0 has four tiles, step it using tile it % 4: it stages P^T, then receives
+//           dS^T, then stages the dQ drain (XT: free again after the drain);
+//   rank 1 receives P^T into three tiles (it % 3), each free once dV and the
+//           elementwise warps have read it (PR), and writes dS^T into two tiles of its
+//           own (it % 2), each free once dQ^T has read it and its copy has landed in
+//           rank 0 (DF); it stages its dQ drain in a buffer of its own.
+// A copy signals only its receiver, so the receivers report back with relaxed remote
+// arrivals, which order no data (the readers have finished when they are sent):
+//   XE[b] on rank 0: rank 1's P^T tile b is free again (sent by rank 1's MMA warp);
+//   DF[b] on rank 1: its dS^T copy from tile b has landed in rank 0 (sent by rank 0's
+//         MMA warp; DF also counts the commit of the dQ^T that reads the tile).
 // A release at cluster scope is never used on the step path: it stalls the signalling
 // thread on all of its earlier memory operations (about a microsecond on B200).
 //
@@ -46,6 +51,10 @@
 // oldest step, else the next S^T; rank 1: dV, else dQ^T, else the next dP^T), and keeps
 // S^T / dP^T at most a step or two ahead, because the tensor pipe runs in order and a
 // queued batch would delay the contractions the exchange chain waits for.
+//
+// dK (rank 0) and dV (rank 1) leave through the idle stages: the elementwise warps write
+// the bf16 rows there in the 128-byte-swizzled layout of the output map's box, and one
+// thread issues four TMA tensor stores.
 //
 // No TMA multicast and no multicast commit are used.  Every wait is bounded.
 #include "det_order.cuh"

@@ -1,0 +1,41 @@
+"""Host-side helpers of bench.py that need no GPU: the code hash that keeps a committed
+DRAM-traffic measurement tied to the kernel source it was taken on."""
+import json
+import os
+
+import bench
+
+
+def _write(tmp_path, name, text):
+    p = tmp_path / name
+    p.write_text(text)
+    return str(p)
+
+
+def test_code_hash_ignores_comments_and_layout(tmp_path):
+    a = _write(tmp_path, "a.cu", "// header\nint f(int x) {\n  return x + 1;  \n}\n")
+    b = _write(tmp_path, "b.cu", "// another header\n\n  // note\nint f(int x) {\n    return x + 1;\n}\n")
+    assert bench.source_code_sha([a]) == bench.source_code_sha([b])
+
+
+def test_code_hash_follows_code(tmp_path):
+    a = _write(tmp_path, "a.cu", "int f(int x) {\n  return x + 1;\n}\n")
+    b = _write(tmp_path, "b.cu", "int f(int x) {\n  return x + 2;\n}\n")
+    assert bench.source_code_sha([a]) != bench.source_code_sha([b])
+    # a trailing comment sits on a code line and counts as code
+    c = _write(tmp_path, "c.cu", "int f(int x) {\n  return x + 1;  // one\n}\n")
+    assert bench.source_code_sha([a]) != bench.source_code_sha([c])
+
+
+def test_traffic_reported_only_for_the_measured_code(tmp_path, monkeypatch):
+    """bench.py reports the committed figure while the hash matches, else null."""
+    d = json.load(open(os.path.join(bench.ROOT, "profiles", "bwd_main_traffic.json")))
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "bwd_source_sha", lambda: "abc")
+    (prof / "bwd_main_traffic.json").write_text(json.dumps(dict(d, source_sha="abc")))
+    assert bench.profiled_traffic(d["workload"]) == d["dram_bytes_per_launch"]
+    assert bench.profiled_traffic("another_workload") is None
+    (prof / "bwd_main_traffic.json").write_text(json.dumps(dict(d, source_sha="old")))
+    assert bench.profiled_traffic(d["workload"]) is None
