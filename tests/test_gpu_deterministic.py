@@ -1,6 +1,6 @@
 """Deterministic backward (sparse_attn_bwd_deterministic): dQ, dK and dV are bitwise
 identical across calls, within the parity tolerance of the oracle, and close to the
-default backward, for the three backward kernels (D=128 single CTA, the 192/128
+default backward, for the three backward kernels (D=64/128 single CTA, the 192/128
 head-dim split, the 256/256 pair)."""
 import numpy as np
 import pytest
@@ -19,6 +19,15 @@ CASES = [
              topk=200, name="det_index_d192_128"),
     I.scaled(W["long_causal_blocksparse_h16_s32768_d256"], Sq=1024, Sk=1024, HQ=2, HK=2,
              density=0.5, name="det_d256"),
+    # the grid interleaves heads (and batches) in this mode: GQA, batch > 1, 64-wide
+    # blocks and a ragged length on the pair kernel, index mode on it, and a ragged
+    # (64, 64) case on the single-CTA kernel
+    I.scaled(W["long_causal_blocksparse_h16_s32768_d256"], B=2, Sq=450, Sk=450, HQ=4, HK=2,
+             bs=64, density=0.5, name="det_bs64_gqa_b2_ragged_d256"),
+    I.scaled(W["long_causal_blocksparse_h16_s32768_d256"], mode="index", Sq=520, Sk=520, HQ=4,
+             HK=2, topk=150, name="det_index_gqa_d256"),
+    I.scaled(W["blocksparse_mha_s256_d64"], Sq=300, Sk=300, HQ=4, HK=2, causal=True,
+             name="det_ragged_bs64_causal_gqa_d64"),
 ]
 
 
