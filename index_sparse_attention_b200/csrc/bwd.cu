@@ -435,11 +435,10 @@ __global__ void __launch_bounds__(448, 1)
                          __ldg(a.mask + (bg * a.Mb + mb) * static_cast<int64_t>(a.Nb) + j / 64) != 0;
           if (!m) cm = 0u;
         } else if (a.mode == SA_MODE_INDEX) {
-          const uint32_t* bw = bmbuf + st * BM * 4 + (32 * hc) * 4 + (r >> 5);
-          uint32_t bits = 0u;
-#pragma unroll 8
-          for (int q = 0; q < 32; ++q) bits |= ((bw[q * 4] >> lane) & 1u) << q;
-          cm &= bits;
+          // lane L loads the presence word of query q0 + L over this warp's 32 key rows;
+          // a bit transpose across the warp leaves in lane L the word of key row r over
+          // the 32 queries (the branch is warp-uniform)
+          cm &= warp_transpose32(bmbuf[st * BM * 4 + (32 * hc + lane) * 4 + (r >> 5)], lane);
         }
       }
       tmem_wait_ld();
