@@ -87,9 +87,17 @@ def source_code_sha(paths):
     return h.hexdigest()[:16]
 
 
-def bwd_source_sha():
+# the sources each backward main kernel is compiled from
+BWD_SOURCES = {
+    "sparse_bwd_pair_kernel": ("bwd_pair.cu", "sa_device.cuh", "det_order.cuh", "sa_kernels.h"),
+    "sparse_bwd_kernel": ("bwd.cu", "sa_device.cuh", "det_order.cuh", "sa_kernels.h"),
+}
+
+
+def bwd_source_sha(kernel):
+    files = BWD_SOURCES[kernel.split("<")[0]]
     return source_code_sha(os.path.join(ROOT, "index_sparse_attention_b200", "csrc", f)
-                           for f in ("bwd.cu", "bwd_pair.cu", "sa_device.cuh"))
+                           for f in files)
 
 
 def profiled_traffic(workload):
@@ -99,7 +107,7 @@ def profiled_traffic(workload):
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    if d.get("source_sha") != bwd_source_sha() or d.get("workload") != workload:
+    if d.get("workload") != workload or d.get("source_sha") != bwd_source_sha(d["kernel"]):
         return None
     return d.get("dram_bytes_per_launch")
 

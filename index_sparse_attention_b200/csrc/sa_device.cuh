@@ -120,20 +120,6 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort, status));
 }
 
-// 32 x 32 bit-matrix transpose across a converged warp: on entry lane L holds row L
-// (bit c = column c), on exit column L (bit r = row r).  Five butterfly stages: at
-// stage j, lanes whose bit j is clear keep the low half of each 2j-bit group and take
-// the partner's low halves into their high halves, the others the reverse.
-__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
-  uint32_t m = 0x0000FFFFu;
-#pragma unroll
-  for (int j = 16; j != 0; j >>= 1, m ^= (m << j)) {
-    const uint32_t y = __shfl_xor_sync(0xFFFFFFFFu, x, j);
-    x = (lane & j) ? ((x & ~m) | ((y >> j) & m)) : ((x & m) | ((y << j) & ~m));
-  }
-  return x;
-}
-
 // Picks one active lane of a converged warp (true on that lane only).
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred = 0;

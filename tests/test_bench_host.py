@@ -33,7 +33,7 @@ def test_traffic_reported_only_for_the_measured_code(tmp_path, monkeypatch):
     prof = tmp_path / "profiles"
     prof.mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "bwd_source_sha", lambda: "abc")
+    monkeypatch.setattr(bench, "bwd_source_sha", lambda kernel: "abc")
     (prof / "bwd_main_traffic.json").write_text(json.dumps(dict(d, source_sha="abc")))
     assert bench.profiled_traffic(d["workload"]) == d["dram_bytes_per_launch"]
     assert bench.profiled_traffic("another_workload") is None
