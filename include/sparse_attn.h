@@ -143,17 +143,18 @@ typedef struct sparse_attn_params {
  */
 int sparse_attn_fwd(const sparse_attn_params *p, sa_stream_t stream);
 
-/* Bytes of device workspace sparse_attn_bwd needs for these shapes (fp32 Delta and
- * the fp32 dQ accumulator), rounded up to 256 B. */
+/* Bytes of device workspace sparse_attn_bwd needs for these shapes (fp32 Delta, the
+ * fp32 dQ accumulator and the deterministic mode's int32 turn counters, each rounded
+ * up to 256 B). */
 size_t sparse_attn_bwd_workspace_size(const sparse_attn_params *p);
 
 /*
  * sparse_attn_bwd -- backward: dq, dk, dv from q, k, v, o, lse, dout.
  * Preprocess Delta = rowsum(dO * O); main kernel over key tiles (walking the
  * transposed lists) recomputing P = exp(scale S - LSE), accumulating dV += P^T dO and
- * dK += dS^T Q in tensor memory and adding dQ += dS K into an fp32 accumulator;
- * postprocess scales dQ (and dK) by softmax_scale and casts to bf16 (MagiAttention
- * PR #334, section 1 and section 3).  `workspace` is device memory of at least
+ * dK += dS^T Q in tensor memory (dK scaled by softmax_scale as it is stored) and
+ * adding dQ += dS K into an fp32 accumulator; the postprocess scales dQ by
+ * softmax_scale and casts it to bf16 (MagiAttention PR #334, section 1 and section 3).  `workspace` is device memory of at least
  * sparse_attn_bwd_workspace_size() bytes, owned by the caller; its contents need not
  * be initialised.
  */
