@@ -27,6 +27,46 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _require(cond, msg, exc=ValueError):
+    if not cond:
+        raise exc(msg)
+
+
+def _check(name, t, dtype, shape=None, ndim=None, device=None, contiguous=True):
+    """Argument checks done here because the C ABI sees pointers and sizes only: a
+    tensor of the wrong shape would be read or written out of bounds by the kernels."""
+    _require(isinstance(t, torch.Tensor), f"{name} must be a torch.Tensor", TypeError)
+    _require(t.dtype == dtype, f"{name} must be {dtype}, got {t.dtype}", TypeError)
+    if ndim is not None:
+        _require(t.dim() == ndim, f"{name} must have {ndim} dimensions, got {t.dim()}")
+    if shape is not None:
+        _require(tuple(t.shape) == tuple(shape),
+                 f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    _require(t.is_cuda, f"{name} must be a CUDA tensor")
+    if contiguous:
+        _require(t.is_contiguous(), f"{name} must be contiguous")
+    if device is not None:
+        _require(t.device == device, f"{name} is on {t.device}, expected {device}")
+
+
+def _check_status(dev_status, device):
+    if dev_status is not None:
+        _check("dev_status", dev_status, torch.int32, device=device)
+        _require(dev_status.numel() >= 1, "dev_status must hold at least one int32")
+
+
+def _check_qkv(q, k, v):
+    _check("q", q, torch.bfloat16, ndim=4)
+    B, Sq, HQ, Dqk = q.shape
+    _check("k", k, torch.bfloat16, ndim=4, device=q.device)
+    _require(k.shape[0] == B and k.shape[3] == Dqk,
+             f"k must be [B={B}, Sk, HK, Dqk={Dqk}], got {tuple(k.shape)}")
+    _check("v", v, torch.bfloat16, ndim=4, device=q.device)
+    _require(tuple(v.shape[:3]) == tuple(k.shape[:3]),
+             f"v must be [B, Sk, HK, Dv] with k's first three sizes {tuple(k.shape[:3])}, "
+             f"got {tuple(v.shape)}")
+
+
 class BlockSparse:
     """Tile lists (and the partial-tile mask data) of one sparsity pattern.
 
@@ -68,8 +108,10 @@ def block_mask_to_block_sparse(mask, B, HK, Sq, Sk, bs=SA_TILE, causal=False, de
     """
     L = _lib.load()
     if mask is not None:
+        _check("mask", mask, torch.uint8, ndim=4)
+        _require(tuple(mask.shape[:2]) == (B, HK),
+                 f"mask must be [B={B}, HK={HK}, Mb, Nb], got {tuple(mask.shape)}")
         device = mask.device
-        assert mask.dtype == torch.uint8 and mask.is_contiguous()
         mode = SA_MODE_BLOCK
     else:
         mode = SA_MODE_DENSE
@@ -82,7 +124,8 @@ def block_mask_to_block_sparse(mask, B, HK, Sq, Sk, bs=SA_TILE, causal=False, de
 def index_to_block_sparse(idx, Sk, causal=False, dev_status=None):
     """Tile lists and presence bitmap from top-k indices int32 [B,Sq,HK,topk] (-1 = pad)."""
     L = _lib.load()
-    assert idx.dtype == torch.int32 and idx.is_contiguous() and idx.dim() == 4
+    _check("idx", idx, torch.int32, ndim=4)
+    _check_status(dev_status, idx.device)
     B, Sq, HK, topk = idx.shape
     W = -(-Sk // 32)
     bitmap = torch.empty((B, HK, Sq, W), dtype=torch.int32, device=idx.device)
@@ -95,12 +138,26 @@ def index_to_block_sparse(idx, Sk, causal=False, dev_status=None):
 
 def _params(q, k, v, o, lse, sparse, scale, dout=None, dq=None, dk=None, dv=None,
             dev_status=None):
+    _check_qkv(q, k, v)
     B, Sq, HQ, Dqk = q.shape
     _, Sk, HK, _ = k.shape
     Dv = v.shape[3]
-    for t in (q, k, v, o, dout, dq, dk, dv):
+    _require(isinstance(sparse, BlockSparse), "sparse must be a BlockSparse", TypeError)
+    dev = q.device
+    _check("o", o, torch.bfloat16, shape=(B, Sq, HQ, Dv), device=dev)
+    _check("lse", lse, torch.float32, shape=(B, HQ, Sq), device=dev)
+    for name, t, like in (("dout", dout, o), ("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
         if t is not None:
-            assert t.dtype == torch.bfloat16 and t.is_contiguous() and t.is_cuda
+            _check(name, t, torch.bfloat16, shape=like.shape, device=dev)
+    _check_status(dev_status, dev)
+    return _params_struct(q, k, v, o, lse, sparse, scale, dout, dq, dk, dv, dev_status)
+
+
+def _params_struct(q, k, v, o, lse, sparse, scale, dout=None, dq=None, dk=None, dv=None,
+                   dev_status=None):
+    B, Sq, HQ, Dqk = q.shape
+    _, Sk, HK, _ = k.shape
+    Dv = v.shape[3]
     return _lib.ParamsStruct(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
         None if dout is None else dout.data_ptr(), None if dq is None else dq.data_ptr(),
@@ -126,10 +183,11 @@ def sparse_attn_fwd(q, k, v, sparse, softmax_scale=None, o=None, lse=None, dev_s
 
 
 def sparse_attn_bwd_workspace_size(q, k, v, sparse):
+    """Bytes of device workspace sparse_attn_bwd needs for these shapes."""
     L = _lib.load()
+    _check_qkv(q, k, v)
     o = q.new_empty((1,))
-    p = _params(q, k, v, o, o, sparse, 1.0)
-    p.Dv = v.shape[3]
+    p = _params_struct(q, k, v, o, o, sparse, 1.0)
     return int(L.sparse_attn_bwd_workspace_size(ctypes.byref(p)))
 
 
@@ -144,10 +202,12 @@ def sparse_attn_bwd(q, k, v, o, lse, dout, sparse, softmax_scale=None, dq=None, 
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    _require(dout is not None, "dout is required")
     p = _params(q, k, v, o, lse, sparse, softmax_scale, dout, dq, dk, dv, dev_status)
     need = int(L.sparse_attn_bwd_workspace_size(ctypes.byref(p)))
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check("workspace", workspace, torch.uint8, device=q.device)
     fn = L.sparse_attn_bwd_deterministic if deterministic else L.sparse_attn_bwd
     _lib.check("sparse_attn_bwd",
                fn(ctypes.byref(p), _ptr(workspace), workspace.numel(), _stream(q.device)))
@@ -167,6 +227,7 @@ def sparse_attn_bwd_noalloc(q, k, v, o, lse, dout, sparse, softmax_scale=None, d
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    _require(dout is not None, "dout is required")
     p = _params(q, k, v, o, lse, sparse, softmax_scale, dout, dq, dk, dv, dev_status)
     _lib.check("sparse_attn_bwd_noalloc", L.sparse_attn_bwd_noalloc(ctypes.byref(p),
                                                                     _stream(q.device)))
@@ -179,16 +240,21 @@ def topk_select(scores, k, starts=None, ends=None, with_values=False, out_idx=No
     [starts[r], ends[r]), largest first, ties to the smaller column, -1 past the number
     of valid columns; with ``with_values`` also the selected scores (fp32 [rows, k])."""
     L = _lib.load()
-    assert scores.dtype == torch.float32 and scores.dim() == 2 and scores.is_cuda
-    assert scores.stride(1) == 1
+    _check("scores", scores, torch.float32, ndim=2, contiguous=False)
+    _require(scores.stride(1) == 1, "scores rows must be contiguous (stride(1) == 1)")
     rows, cols = scores.shape
-    for t in (starts, ends):
+    dev = scores.device
+    for name, t in (("starts", starts), ("ends", ends)):
         if t is not None:
-            assert t.dtype == torch.int32 and t.is_contiguous() and t.numel() == rows
+            _check(name, t, torch.int32, shape=(rows,), device=dev)
+    _check_status(dev_status, dev)
     if out_idx is None:
-        out_idx = torch.empty((rows, k), dtype=torch.int32, device=scores.device)
+        out_idx = torch.empty((rows, k), dtype=torch.int32, device=dev)
+    _check("out_idx", out_idx, torch.int32, shape=(rows, k), device=dev)
     if with_values and out_val is None:
-        out_val = torch.empty((rows, k), dtype=torch.float32, device=scores.device)
+        out_val = torch.empty((rows, k), dtype=torch.float32, device=dev)
+    if out_val is not None:
+        _check("out_val", out_val, torch.float32, shape=(rows, k), device=dev)
     _lib.check("topk_select",
                L.topk_select(_ptr(scores), rows, cols, scores.stride(0), _ptr(starts), _ptr(ends),
                              k, _ptr(out_idx), _ptr(out_val), _ptr(dev_status),
