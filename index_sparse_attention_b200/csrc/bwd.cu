@@ -22,8 +22,13 @@
 //   dV  += P^T dO     (M=128 keys, N=Dv chunk)      TMEM A operand   [TS]
 //   dK  += dS^T Q     (M=128 keys, N=Dqk chunk)     TMEM A operand   [TS]
 //   dQ^T = K^T dS^T   (M=128 head-dim window, N=64) both MN-major    [SS]
-//   the same warps drain dQ^T from TMEM and add it (fp32 reductions, coalesced along
-//   the head dim) into the dQ accumulator.
+//   a drain warpgroup reads dQ^T from TMEM, stages it as fp32 tiles in the consumed
+//   dS^T buffer and adds them into the dQ accumulator with TMA bulk tensor
+//   reduce-adds.
+// Element masks of partial tiles: causal and range by arithmetic, 64-wide blocks from
+// the block mask, index mode from the presence bitmap (one word per lane and a warp
+// bit transpose give each key row its 32-query word).  dK (scaled by softmax_scale)
+// and dV leave through the idle stages by TMA tensor stores.
 // When Dqk + Dv does not leave room in the 512 TMEM columns (192/128), the head dim of
 // dK/dV/dQ is split over two CTAs, each recomputing S^T and dP^T.  Head dims 256/256
 // run on a 2-CTA cluster that splits the work instead (bwd_pair.cu).
