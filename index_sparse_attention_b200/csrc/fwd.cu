@@ -12,8 +12,8 @@
 //              memory allows;
 //   warp 6     TMA producer of the V tiles, so that a K load (which S waits for)
 //              never queues behind a V load that waits for the previous P V.
-//   warp 1     allocates 512 TMEM columns and issues the tcgen05 MMAs from one
-//              thread: S = Q K^T into one of two TMEM S buffers (so the next S is
+//   warp 1     allocates 512 TMEM columns and issues the tcgen05 MMAs (one elected
+//              lane per batch): S = Q K^T into one of two TMEM S buffers (so the next S is
 //              computed while the softmax works on the current one), and
 //              O += P V with P read from TMEM (A operand in tensor memory).
 //   warps 2-5  softmax, one query row per thread (thread = TMEM lane): tcgen05.ld the
@@ -21,7 +21,8 @@
 //              mask or index bitmap), update the running max lazily (O is rescaled in
 //              TMEM only when the max grows by more than 2^8), exponentiate with
 //              ex2, write bf16 P back over the S buffer, and at the end normalise O
-//              and write O (bf16) and LSE (fp32, natural log).
+//              into the idle Q buffer (the output map's swizzled box layout, sent by
+//              TMA tensor stores) and write LSE (fp32, natural log).
 // TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+Dv).
 // Every mbarrier wait is bounded; a timeout sets SA_ERR_TIMEOUT in the status word and
 // the CTA leaves after releasing its tensor memory.
