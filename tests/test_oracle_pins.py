@@ -130,6 +130,23 @@ def test_forward_matches_sdpa(case):
     np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-10)
 
 
+@pytest.mark.parametrize("Sq,Sk", [(37, 45), (45, 37), (40, 40)])
+def test_causal_alignment_matches_sdpa_is_causal(Sq, Sk):
+    """The causal reading (top-left: key j allowed for query i iff j <= i, also when
+    Sq != Sk) equals torch SDPA's own is_causal mask, with no mask built here."""
+    q, k, v = rnd(10, (1, Sq, 2, 16)), rnd(11, (1, Sk, 2, 16)), rnd(12, (1, Sk, 2, 16))
+    dout = rnd(13, (1, Sq, 2, 16))
+    P = oracle.Problem(q, k, v, scale=0.25, causal=True, mode="dense")
+    O, lse = oracle.forward(P)
+    tq, tk, tv = (torch.from_numpy(x).permute(0, 2, 1, 3).requires_grad_(True) for x in (q, k, v))
+    o = F.scaled_dot_product_attention(tq, tk, tv, is_causal=True, scale=0.25)
+    np.testing.assert_allclose(O, o.detach().permute(0, 2, 1, 3).numpy(), rtol=0, atol=1e-12)
+    (o * torch.from_numpy(dout).permute(0, 2, 1, 3)).sum().backward()
+    dq, dk, dv = oracle.backward(P, dout, O, lse)
+    for got, t in ((dq, tq), (dk, tk), (dv, tv)):
+        np.testing.assert_allclose(got, t.grad.permute(0, 2, 1, 3).numpy(), rtol=0, atol=1e-11)
+
+
 @pytest.mark.parametrize("case", CASES, ids=[f"{c[8]}-{'causal' if c[7] else 'full'}-{c[1]}x{c[2]}" for c in CASES])
 def test_backward_matches_autograd(case):
     P, A, dout = make_case(case, seed=10)
