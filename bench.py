@@ -54,6 +54,29 @@ def whole_job_rate(flop_per_rank_step, ms_per_step_max, world):
     return world * flop_per_rank_step / (ms_per_step_max * 1e-3) / 1e12
 
 
+def peak_basis(peaks, clocks):
+    """The bf16 peak a run is measured against: the burst figure (a cuBLAS GEMM timed
+    alone) unless the run's own clock record shows power capping during the timed
+    region, then the sustained figure (the same GEMM looped for seconds under the cap)."""
+    capped = bool(clocks) and "sw_power_cap" in clocks.get("reasons", [])
+    if capped:
+        return float(peaks.get("bf16_tflops_sustained",
+                               FALLBACK_PEAKS["bf16_tflops_sustained"])), "bf16_tflops_sustained"
+    return float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])), "bf16_tflops"
+
+
+def converter_bytes(w):
+    """Algorithmic HBM bytes of one tile-list conversion: index mode reads the indices
+    once, writes the presence bitmap and reads it back once (classification); both
+    modes write the forward lists and read them back for the transposed ones."""
+    Tm, Tn = -(-w.Sq // 128), -(-w.Sk // 128)
+    lists = 4 * w.B * w.HK * (Tm * (Tn + 2) + Tn * (Tm + 2))
+    if w.mode == "index":
+        bitmap = 4 * w.B * w.HK * w.Sq * (-(-w.Sk // 32))
+        return 4 * w.B * w.Sq * w.HK * w.topk + 2 * bitmap + 2 * lists
+    return w.B * w.HK * (-(-w.Sq // w.bs)) * (-(-w.Sk // w.bs)) + 2 * lists
+
+
 def tile_flops(w):
     """(forward, backward) tensor-core FLOP of one active 128x128 tile for one query head."""
     return 2 * 128 * 128 * (w.Dqk + w.Dv), 2 * 128 * 128 * (3 * w.Dqk + 2 * w.Dv)
@@ -388,6 +411,16 @@ def run_gpu(args):
         dist.barrier()
     torch.cuda.synchronize()
     ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
+
+    # the converter alone (it is part of every step above): mean over the same number of
+    # calls, timed on the launch stream
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    for _ in range(args.steps):
+        lists()
+    c1.record(stream)
+    torch.cuda.synchronize()
+    conv_ms = c0.elapsed_time(c1) / args.steps
     per_kernel = {
         "fwd": float(np.mean([r[0].elapsed_time(r[1]) for r in evs])),
         "bwd_pre": float(np.mean([r[2].elapsed_time(r[3]) for r in evs])),
@@ -466,9 +499,14 @@ def run_gpu(args):
     peaks, peak_src = load_peaks()
     clocks = clk.summary()
     if rank == 0:
-        peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        peak, peak_kind = peak_basis(peaks, clocks)
         peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        peak_sust = float(peaks.get("bf16_tflops_sustained",
+                                    FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        of = "of measured" if peak_src == "measured" else "of fallback"
         achieved = active * bwd_f / (per_kernel["bwd_main"] * 1e-3) / 1e12
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        conv_b = converter_bytes(w)
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -477,12 +515,15 @@ def run_gpu(args):
             "config": dict(workload_config(w, active),
                            **({"backward": "deterministic"} if args.deterministic else {})),
             "pct_of_bf16_peak": 100.0 * (value / world) / peak,
-            "pct_basis": f"bf16_tflops_sustained {peak:.1f} TFLOP/s ({peak_src})",
+            "pct_basis": (f"{peak_kind} {peak:.1f} TFLOP/s ({of}); burst unless the clock record "
+                          "of the timed region shows sw_power_cap"),
+            "pct_of_bf16_burst": 100.0 * (value / world) / peak_burst,
+            "pct_of_bf16_sustained": 100.0 * (value / world) / peak_sust,
             "flop_per_step": flop_step, "kernel_ms": per_kernel,
             "roofline": {
                 "kernel": bwd_kernel_name(w), "bound": "tensor", "achieved": achieved,
                 "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "peak_kind": f"bf16_tflops_sustained ({'of measured' if peak_src == 'measured' else 'of fallback'}); burst {peak_burst:.1f}",
+                "peak_kind": f"{peak_kind} ({of}); burst {peak_burst:.1f}, sustained {peak_sust:.1f}",
                 "traffic": profiled_traffic(w.name),
                 "algorithmic": "2*128*128*(3*Dqk+2*Dv) FLOP per active tile x query head",
             },
@@ -491,6 +532,12 @@ def run_gpu(args):
                     "overlap": "H2D of step s+1 and D2H of step s-1 on their own streams "
                                "while step s computes; device inputs and outputs "
                                "double-buffered"},
+            "converter": {
+                "ms": conv_ms, "algorithmic_bytes": conv_b, "achieved_gbs": conv_b / conv_ms / 1e6,
+                "peak_gbs": hbm, "frac": conv_b / conv_ms / 1e6 / hbm,
+                "kernels": ("scatter_bits + classify_index + compact + transpose" if w.mode == "index"
+                            else "classify_block + compact + transpose"),
+                "note": "timed alone, same launches as inside each step"},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
         }

@@ -41,6 +41,10 @@
  *  - Supported (Dqk, Dv): (64,64), (128,128), (192,128), (256,256).  HQ % HK == 0.
  *  - Work is enqueued on `stream` and runs asynchronously; the call returns once it
  *    is enqueued.  Errors found on the host are returned before anything is enqueued.
+ *  - Kernels run on the CURRENT device (cudaSetDevice); every pointer must be memory of
+ *    that device and `stream` must belong to it (a stream created on another device is
+ *    refused with SA_ERR_DEVICE).  Per-device set-up (kernel attributes, the no-alloc
+ *    scratch address) is done on first use on each device, thread-safely.
  *  - Return value: SA_OK (0) or a negative SA_ERR_* code.  Errors found on the GPU
  *    (an index outside [-1, Sk), a pipeline wait that timed out) are OR-ed into the
  *    optional device int32 `dev_status` (bit 1: index, bit 2: timeout); read it after
@@ -66,6 +70,7 @@ typedef struct CUstream_st *sa_stream_t; /* the same handle as cudaStream_t */
 #define SA_ERR_CUDA (-5)        /* a CUDA call or kernel launch failed */
 #define SA_ERR_WORKSPACE (-7)   /* workspace missing or too small */
 #define SA_ERR_SCRATCH_LIMIT (-8) /* sparse_attn_bwd_noalloc: problem exceeds its fixed scratch */
+#define SA_ERR_DEVICE (-9)      /* the stream belongs to a device other than the current one */
 
 #define SA_MODE_DENSE 0
 #define SA_MODE_BLOCK 1
@@ -191,8 +196,10 @@ int sparse_attn_bwd_deterministic(const sparse_attn_params *p, void *workspace,
  *  - Returns SA_ERR_SCRATCH_LIMIT, before enqueuing anything, when
  *    sparse_attn_bwd_workspace_size(p) exceeds SA_NOALLOC_SCRATCH_BYTES.
  *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current); make it before any stream
- *    capture.
+ *    (cudaGetSymbolAddress, with that device current; a failed lookup is retried by the
+ *    next call); make it before any stream capture.
+ *  - The array used is the current device's: `stream` must belong to the current
+ *    device (SA_ERR_DEVICE otherwise).
  *  - All calls on a device share the array and overwrite it; calls whose GPU work
  *    overlaps (unordered streams, several host threads) race: serialise them.
  *  - Allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
@@ -210,6 +217,18 @@ int sparse_attn_bwd_noalloc(const sparse_attn_params *p, sa_stream_t stream);
  * thread calls into the library.  Returns SA_OK.
  */
 int sparse_attn_set_timing_events(void *const *events);
+
+/*
+ * sparse_attn_set_wait_limit_ns -- test instrumentation (no counterpart on the pages).
+ * Every pipeline wait inside the attention kernels is bounded: a wait that has not
+ * completed after the limit gives up, sets bit 2 of *dev_status, and its CTA drains the
+ * copies and tensor-core operations it has in flight and leaves (the outputs of that
+ * call are then undefined, the CUDA context stays usable).  The default limit is 2 s.
+ * This call sets the limit, in nanoseconds, for the calls enqueued after it (0 restores
+ * the default).  A limit of a few microseconds makes ordinary waits run out: that is
+ * how the tests exercise the timeout path.  Process-wide; returns SA_OK.
+ */
+int sparse_attn_set_wait_limit_ns(uint64_t ns);
 
 /* Largest k that topk_select supports. */
 #define SA_TOPK_MAX_K 4096

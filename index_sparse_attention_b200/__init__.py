@@ -6,6 +6,7 @@ computation (tile-list conversion, forward, backward) runs in the library's CUDA
 kernels.  The functions carry the names of the C entry points.
 """
 import ctypes
+import functools
 import math
 
 import torch
@@ -15,12 +16,34 @@ from ._lib import SA_MODE_BLOCK, SA_MODE_DENSE, SA_MODE_INDEX, SA_TILE, SparseAt
 
 __all__ = ["BlockSparse", "block_mask_to_block_sparse", "index_to_block_sparse",
            "sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_bwd_workspace_size",
-           "sparse_attn_bwd_noalloc", "topk_select",
+           "sparse_attn_bwd_noalloc", "topk_select", "sparse_attn_set_wait_limit_ns",
            "SparseAttnError", "SA_TILE"]
 
 
 def _stream(device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _on_device(arg):
+    """Runs the wrapped entry point with the device of its tensor argument `arg` (name)
+    made current: the C ABI launches on the current device and refuses a stream of
+    another device, so a tensor on cuda:1 must not be handed over while cuda:0 is
+    current."""
+    def deco(fn):
+        import inspect
+        pos = list(inspect.signature(fn).parameters).index(arg)
+
+        @functools.wraps(fn)
+        def wrapper(*args, **kw):
+            t = kw.get(arg) if arg in kw else (args[pos] if pos < len(args) else None)
+            if isinstance(t, torch.Tensor) and t.is_cuda:
+                with torch.cuda.device(t.device):
+                    return fn(*args, **kw)
+            return fn(*args, **kw)
+
+        wrapper.device_arg = arg
+        return wrapper
+    return deco
 
 
 def _ptr(t):
@@ -101,6 +124,7 @@ class BlockSparse:
         return int(self.cnt.sum().item())
 
 
+@_on_device("mask")
 def block_mask_to_block_sparse(mask, B, HK, Sq, Sk, bs=SA_TILE, causal=False, device=None):
     """Tile lists from a block mask uint8 [B,HK,Mb,Nb] at granularity bs (64 or 128).
 
@@ -115,12 +139,16 @@ def block_mask_to_block_sparse(mask, B, HK, Sq, Sk, bs=SA_TILE, causal=False, de
         mode = SA_MODE_BLOCK
     else:
         mode = SA_MODE_DENSE
-    bsp = BlockSparse(mode, B, HK, Sq, Sk, causal, device, bs=bs, mask=mask)
-    _lib.check("block_mask_to_block_sparse",
-               L.block_mask_to_block_sparse(ctypes.byref(bsp.c), _stream(device)))
+        device = torch.device("cuda") if device is None else torch.device(device)
+        _require(device.type == "cuda", "device must be a CUDA device")
+    with torch.cuda.device(device):
+        bsp = BlockSparse(mode, B, HK, Sq, Sk, causal, device, bs=bs, mask=mask)
+        _lib.check("block_mask_to_block_sparse",
+                   L.block_mask_to_block_sparse(ctypes.byref(bsp.c), _stream(device)))
     return bsp
 
 
+@_on_device("idx")
 def index_to_block_sparse(idx, Sk, causal=False, dev_status=None):
     """Tile lists and presence bitmap from top-k indices int32 [B,Sq,HK,topk] (-1 = pad)."""
     L = _lib.load()
@@ -166,6 +194,7 @@ def _params_struct(q, k, v, o, lse, sparse, scale, dout=None, dq=None, dk=None, 
         None if dev_status is None else dev_status.data_ptr())
 
 
+@_on_device("q")
 def sparse_attn_fwd(q, k, v, sparse, softmax_scale=None, o=None, lse=None, dev_status=None):
     """O [B,Sq,HQ,Dv] (bf16) and LSE [B,HQ,Sq] (fp32) of sparse attention."""
     L = _lib.load()
@@ -182,6 +211,7 @@ def sparse_attn_fwd(q, k, v, sparse, softmax_scale=None, o=None, lse=None, dev_s
     return o, lse
 
 
+@_on_device("q")
 def sparse_attn_bwd_workspace_size(q, k, v, sparse):
     """Bytes of device workspace sparse_attn_bwd needs for these shapes."""
     L = _lib.load()
@@ -191,6 +221,7 @@ def sparse_attn_bwd_workspace_size(q, k, v, sparse):
     return int(L.sparse_attn_bwd_workspace_size(ctypes.byref(p)))
 
 
+@_on_device("q")
 def sparse_attn_bwd(q, k, v, o, lse, dout, sparse, softmax_scale=None, dq=None, dk=None,
                     dv=None, workspace=None, dev_status=None, deterministic=False):
     """dQ, dK, dV (bf16, layouts of q, k, v) of sparse attention; with
@@ -214,6 +245,7 @@ def sparse_attn_bwd(q, k, v, o, lse, dout, sparse, softmax_scale=None, dq=None, 
     return dq, dk, dv
 
 
+@_on_device("q")
 def sparse_attn_bwd_noalloc(q, k, v, o, lse, dout, sparse, softmax_scale=None, dq=None, dk=None,
                             dv=None, dev_status=None):
     """dQ, dK, dV like sparse_attn_bwd, with the scratch taken from the library's fixed
@@ -234,6 +266,7 @@ def sparse_attn_bwd_noalloc(q, k, v, o, lse, dout, sparse, softmax_scale=None, d
     return dq, dk, dv
 
 
+@_on_device("scores")
 def topk_select(scores, k, starts=None, ends=None, with_values=False, out_idx=None, out_val=None,
                 dev_status=None):
     """Column indices (int32 [rows, k]) of the k largest fp32 scores of each row's range
@@ -261,3 +294,10 @@ def topk_select(scores, k, starts=None, ends=None, with_values=False, out_idx=No
                              _stream(scores.device)))
     return (out_idx, out_val) if with_values else out_idx
 
+
+def sparse_attn_set_wait_limit_ns(ns):
+    """Test instrumentation: the limit (ns) of every pipeline wait of the attention
+    kernels enqueued after this call (0 restores the default of 2 s).  A wait that runs
+    out sets bit 2 of the device status word and its CTA leaves; see
+    include/sparse_attn.h."""
+    _lib.check("sparse_attn_set_wait_limit_ns", _lib.load().sparse_attn_set_wait_limit_ns(int(ns)))

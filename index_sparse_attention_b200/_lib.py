@@ -19,6 +19,7 @@ SA_ERR_ALIGN = -4
 SA_ERR_CUDA = -5
 SA_ERR_WORKSPACE = -7
 SA_ERR_SCRATCH_LIMIT = -8
+SA_ERR_DEVICE = -9
 SA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 SA_TOPK_MAX_K = 4096
 
@@ -38,6 +39,7 @@ EXPORTS = (
     "sparse_attn_bwd_deterministic",
     "sparse_attn_bwd_noalloc",
     "sparse_attn_set_timing_events",
+    "sparse_attn_set_wait_limit_ns",
     "sparse_attn_error_string",
     "topk_select",
 )
@@ -94,6 +96,8 @@ def load():
     L.sparse_attn_bwd_noalloc.restype = ctypes.c_int
     L.sparse_attn_set_timing_events.argtypes = [vp]
     L.sparse_attn_set_timing_events.restype = ctypes.c_int
+    L.sparse_attn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    L.sparse_attn_set_wait_limit_ns.restype = ctypes.c_int
     i64 = ctypes.c_int64
     L.topk_select.argtypes = [vp, i64, i64, i64, vp, vp, ctypes.c_int32, vp, vp, vp, vp]
     L.topk_select.restype = ctypes.c_int

@@ -21,6 +21,7 @@ int cuda_error(cudaError_t e, const char* what) {
 }
 cudaEvent_t* g_timing_events = nullptr;
 static cudaEvent_t g_events_copy[6];
+std::atomic<uint64_t> g_wait_limit_ns{0};
 }  // namespace sa
 
 namespace {
@@ -136,6 +137,8 @@ int fill_args(const sparse_attn_params* p, AttnArgs* a, bool backward) {
   a->scale = p->softmax_scale;
   a->scale_log2 = p->softmax_scale * 1.4426950408889634f;
   a->status = p->dev_status;
+  const uint64_t lim = g_wait_limit_ns.load(std::memory_order_relaxed);
+  a->wait_limit_ns = lim ? lim : kWaitLimitNs;
   return SA_OK;
 }
 
@@ -171,6 +174,8 @@ extern "C" const char* sparse_attn_error_string(int code) {
     case SA_ERR_WORKSPACE: return "workspace missing or too small";
     case SA_ERR_SCRATCH_LIMIT:
       return "problem needs more backward scratch than the fixed SA_NOALLOC_SCRATCH_BYTES array";
+    case SA_ERR_DEVICE:
+      return "the stream belongs to a device other than the current device";
     default: return "unknown error code";
   }
 }
@@ -185,9 +190,16 @@ extern "C" int sparse_attn_set_timing_events(void* const* events) {
   return SA_OK;
 }
 
+extern "C" int sparse_attn_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns.store(ns, std::memory_order_relaxed);
+  return SA_OK;
+}
+
 extern "C" int sparse_attn_fwd(const sparse_attn_params* p, sa_stream_t stream) {
   AttnArgs a;
   int rc = fill_args(p, &a, false);
+  if (rc) return rc;
+  rc = check_stream_device(reinterpret_cast<cudaStream_t>(stream));
   if (rc) return rc;
   TensorMaps m;
   rc = fill_maps(p, &m, false);
@@ -213,6 +225,8 @@ static int run_bwd(const sparse_attn_params* p, void* workspace, size_t workspac
   if (rc) return rc;
   const size_t need = sparse_attn_bwd_workspace_size(p);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SA_ERR_WORKSPACE;
+  rc = check_stream_device(reinterpret_cast<cudaStream_t>(stream));
+  if (rc) return rc;
   const size_t delta_b = round256(sizeof(float) * static_cast<size_t>(p->B) * p->HQ * p->Sq);
   const size_t dq_b = round256(sizeof(float) * static_cast<size_t>(p->B) * p->Sq * p->HQ * p->Dqk);
   a.delta = static_cast<float*>(workspace);

@@ -181,8 +181,8 @@ __global__ void __launch_bounds__(448, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + C::kBarOff;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * kNumBarsB);
-  volatile int* abort_flag =
-      reinterpret_cast<volatile int*>(smem + C::kBarOff + 8 * kNumBarsB + 4);
+  volatile WaitCtl* abort_flag =
+      reinterpret_cast<volatile WaitCtl*>(smem + C::kBarOff + 8 * kNumBarsB + 8);
   auto BAR = [&](int k) { return bar0 + 8u * static_cast<uint32_t>(k); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -203,6 +203,7 @@ __global__ void __launch_bounds__(448, 1)
   const int n_mt = n_full + __ldg(a.tcnt + 2 * trow + 1);
   const int32_t* tlist = a.tidx + trow * a.Tm;
   const int n_iter = G * n_mt * 2;  // (query head, query tile, 64-row half)
+  int issued = 0;  // Q/dO stage loads issued (the abort path drains the last ones)
 
   // head-dim chunks owned by this CTA
   int kc0, kcn, vc0, vcn, qw0;  // qw0: first head-dim row of the 128-wide dQ^T window
@@ -231,7 +232,8 @@ __global__ void __launch_bounds__(448, 1)
     }
     mbar_init(BAR(kBFin), 1);
     mbar_init(BAR(kBDrainB), 1);
-    *abort_flag = 0;
+    abort_flag->abort = 0;
+    abort_flag->limit_ns = a.wait_limit_ns;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -294,6 +296,7 @@ __global__ void __launch_bounds__(448, 1)
             tma_load_4d(qs + C::kQBytes + c * C::kQPanel, &tm_do, BAR(kBQF + st), c * 64, m0, h, b);
         }
         __syncwarp();
+        issued = it + 1;
         // LSE (in log2 units) and Delta of the 64 queries; +inf / 0 past Sq
         float* ls = lbuf + st * 2 * BM;
 #pragma unroll
@@ -319,11 +322,6 @@ __global__ void __launch_bounds__(448, 1)
           }
         }
         mbar_arrive(BAR(kBLF + st));
-      }
-      if (lane == 0 && *abort_flag) {
-        mbar_wait_limited(BAR(kBKV), 0);
-        for (int it = max(0, n_iter - C::kStages); it < n_iter; ++it)
-          mbar_wait_limited(BAR(kBQF + it % C::kStages), (it / C::kStages) & 1);
       }
     }
   } else if (warp == 1) {
@@ -635,15 +633,32 @@ __global__ void __launch_bounds__(448, 1)
     if (dtid == 0) bulk_wait_group0();  // every reduce has landed before the CTA ends
   }
 
-  if (warp == 1 && *abort_flag) {
-    if (elect_one()) {
-      umma_commit(BAR(kBDrainB));
-      mbar_wait_limited(BAR(kBDrainB), 0);
-    }
-    __syncwarp();
-  }
   tc_fence_before();
   __syncthreads();
+  // Abort path.  Past the barrier above no warp issues another copy or MMA, and the
+  // abort flag no longer changes (the branch is uniform).  A stage is reloaded only after
+  // the MMAs that read its previous contents have completed, so at most the last
+  // kStages stage loads (and the K/V load) can still be in flight: wait for them, and
+  // for every MMA this CTA issued, before shared memory and TMEM are released
+  // (time-limited waits).  The dQ reduce-adds and the dK/dV stores were waited for by
+  // the threads that issued them.
+  if (abort_flag->abort) {
+    if (warp == 0 && lane == 0 && n_iter > 0) {
+      mbar_wait_limited(BAR(kBKV), 0);
+      for (int it = max(0, issued - C::kStages); it < issued; ++it)
+        mbar_wait_limited(BAR(kBQF + it % C::kStages), (it / C::kStages) & 1);
+    }
+    if (warp == 1 && n_iter > 0) {
+      tc_fence_after();
+      if (elect_one()) {
+        umma_commit(BAR(kBDrainB));
+        mbar_wait_limited(BAR(kBDrainB), 0);
+      }
+      __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
@@ -653,15 +668,13 @@ __global__ void __launch_bounds__(448, 1)
 template <int DQK, int DV, int NSPLIT, bool DET>
 static int launch_bwd_main_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
   using C = BwdCfg<DQK, DV, NSPLIT>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    const int rc = cuda_error(cudaFuncSetAttribute(sparse_bwd_kernel<DQK, DV, NSPLIT, DET>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   C::kSmem),
-                              "backward smem attribute");
-    if (rc) return rc;
-    attr_set = true;
-    if (std::getenv("SA_DEBUG")) {
+  static PerDeviceOnce attr;
+  const int rc = once_per_device(attr, [] {
+    const int r = cuda_error(cudaFuncSetAttribute(sparse_bwd_kernel<DQK, DV, NSPLIT, DET>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  C::kSmem),
+                             "backward smem attribute");
+    if (r == SA_OK && std::getenv("SA_DEBUG")) {
       cudaFuncAttributes fa;
       const cudaError_t qe = cudaFuncGetAttributes(&fa, sparse_bwd_kernel<DQK, DV, NSPLIT, DET>);
       int occ = -1;
@@ -676,7 +689,9 @@ static int launch_bwd_main_t(const AttnArgs& a, const TensorMaps& m, cudaStream_
                      fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes, fa.localSizeBytes,
                      fa.maxDynamicSharedSizeBytes, C::kThreads, C::kSmem);
     }
-  }
+    return r;
+  });
+  if (rc) return rc;
   const dim3 grid = DET ? dim3(a.Tn * NSPLIT * a.HK, 1, a.B) : dim3(a.Tn * NSPLIT, a.HK, a.B);
   record_event(3, st);
   sparse_bwd_kernel<DQK, DV, NSPLIT, DET><<<grid, C::kThreads, C::kSmem, st>>>(

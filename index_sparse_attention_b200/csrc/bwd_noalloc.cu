@@ -14,8 +14,10 @@
 //    (sparse_attn_bwd_workspace_size) exceeds it are rejected with
 //    SA_ERR_SCRATCH_LIMIT before anything is enqueued.
 //  - The first call on each device looks up the array's device address with
-//    cudaGetSymbolAddress (with that device current).  Make that first call before
-//    any stream capture.
+//    cudaGetSymbolAddress (with that device current; a failed lookup is retried by the
+//    next call).  Make that first call before any stream capture.
+//  - The array used is the current device's, so `stream` must belong to the current
+//    device (checked: SA_ERR_DEVICE otherwise).
 //  - Every call on a device shares the one array, and each call overwrites it (the
 //    preprocess kernel writes Delta and zeroes the dQ accumulator before use).  Calls
 //    whose work overlaps on the GPU (different streams without ordering, or several
@@ -34,19 +36,22 @@ constexpr int kMaxDevices = 64;
 // device address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_bwd_scratch[SA_NOALLOC_SCRATCH_BYTES];
 
-void* g_scratch_ptr[kMaxDevices];
-cudaError_t g_scratch_rc[kMaxDevices];
-std::once_flag g_scratch_once[kMaxDevices];
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices];  // guarded by g_scratch_mutex; null until a lookup succeeds
 
-// Device address of the scratch array on the current device (looked up once per device).
-void* scratch_address(int device, cudaError_t* rc) {
-  std::call_once(g_scratch_once[device], [device] {
+// Device address of the scratch array on the current device `device`.  The address is
+// stored only once a lookup has succeeded, so a lookup that failed (made during a
+// stream capture, say) is retried by the next call.
+cudaError_t scratch_address(int device, void** out) {
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_ptr[device]) {
     void* p = nullptr;
-    g_scratch_rc[device] = cudaGetSymbolAddress(&p, g_bwd_scratch);
-    g_scratch_ptr[device] = g_scratch_rc[device] == cudaSuccess ? p : nullptr;
-  });
-  *rc = g_scratch_rc[device];
-  return g_scratch_ptr[device];
+    const cudaError_t rc = cudaGetSymbolAddress(&p, g_bwd_scratch);
+    if (rc != cudaSuccess) return rc;
+    g_scratch_ptr[device] = p;
+  }
+  *out = g_scratch_ptr[device];
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -59,8 +64,10 @@ extern "C" int sparse_attn_bwd_noalloc(const sparse_attn_params* p, sa_stream_t 
   int device = -1;
   if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= kMaxDevices)
     return SA_ERR_CUDA;
-  cudaError_t rc;
-  void* scratch = scratch_address(device, &rc);
-  if (rc != cudaSuccess || scratch == nullptr) return SA_ERR_CUDA;
+  // the scratch used is the current device's: the stream must belong to that device
+  const int drc = sa::check_stream_device(reinterpret_cast<cudaStream_t>(stream));
+  if (drc) return drc;
+  void* scratch = nullptr;
+  if (scratch_address(device, &scratch) != cudaSuccess || scratch == nullptr) return SA_ERR_CUDA;
   return sparse_attn_bwd(p, scratch, static_cast<size_t>(SA_NOALLOC_SCRATCH_BYTES), stream);
 }

@@ -139,7 +139,7 @@ enum : int {
                // elementwise thread has passed step it (S^T / dP^T of it+2 wait for that)
   kNumBars = 53
 };
-static_assert(8 * kNumBars + 8 <= 512, "barrier area");
+static_assert(8 * kNumBars + 8 + sizeof(WaitCtl) <= 512, "barrier area");
 
 // DET: deterministic mode (det_order.cuh), a separate instance so that the default
 // kernel carries none of its code.
@@ -158,7 +158,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + kOffBar;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + 8 * kNumBars);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBar + 8 * kNumBars + 4);
+  volatile WaitCtl* abort_flag =
+      reinterpret_cast<volatile WaitCtl*>(smem + kOffBar + 8 * kNumBars + 8);
   auto BAR = [&](int k) { return bar0 + 8u * static_cast<uint32_t>(k); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -183,6 +184,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
   const uint32_t off_l = rank == 0 ? kOffL0 : kOffL1;
   const uint32_t col_acc = rank == 0 ? kColAcc0 : kColAcc1;
   const int ns = rank == 0 ? kStages0 : kStages1;  // Q / dO stages of this rank
+  int issued = 0;  // stage loads issued (the abort path drains the last ones)
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(kBKV), 1);
@@ -211,7 +213,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     for (int q = 0; q < 8; ++q) mbar_init(BAR(kBQH + q), 64);
     mbar_init(BAR(kBFin), 1);
     mbar_init(BAR(kBDrain), 1);
-    *abort_flag = 0;
+    abort_flag->abort = 0;
+    abort_flag->peer_abort = 0;
+    abort_flag->limit_ns = a.wait_limit_ns;
     // the first exchange tiles may arrive from the peer at any time
     for (int s = 0; s < (rank == 0 ? kNX : kNPI) && s < n_iter; ++s)
       mbar_arrive_expect_tx(BAR(kBXF + s), kTile);
@@ -306,6 +310,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
           for (int c = 0; c < 4; ++c) tma_load_4d(qs + c * kQPanel, tm_stage, BAR(kBQF + s), c * 64, m0, h, b);
         }
         __syncwarp();
+        issued = it + 1;
         // rank 1 frees a stage when dV is done, which can precede the elementwise warps'
         // read of the step's Delta: wait for them before overwriting it
         if (rank == 1 && it >= ns &&
@@ -316,11 +321,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         ls[lane + 32] = rows[1];
         mbar_arrive(BAR(kBLF + s));
         if (it + 1 < n_iter) load_rows(it + 1, rows);
-      }
-      if (lane == 0 && *abort_flag) {
-        mbar_wait_limited(BAR(kBKV), 0);
-        for (int it = max(0, n_iter - ns); it < n_iter; ++it)
-          mbar_wait_limited(BAR(kBQF + it % ns), (it / ns) & 1);
       }
     }
   } else if (warp == 1) {
@@ -449,10 +449,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         if (prog) {
           t_last = globaltimer_ns();
         } else {
-          if (__shfl_sync(0xFFFFFFFFu, *abort_flag, 0) != 0) break;
-          if (globaltimer_ns() - t_last > kWaitLimitNs) {
+          if (__shfl_sync(0xFFFFFFFFu, abort_flag->abort, 0) != 0) break;
+          if (globaltimer_ns() - t_last > abort_flag->limit_ns) {
             if (lane == 0) {
-              *abort_flag = 1;
+              abort_flag->abort = 1;
               report_status(a.status, kStatusTimeout);
             }
             __syncwarp();
@@ -784,18 +784,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     if (dtid == 0) bulk_wait_group0();
   }
 
-  if (warp == 1 && *abort_flag) {
-    if (elect_one()) {
-      umma_commit(BAR(kBDrain));
-      mbar_wait_limited(BAR(kBDrain), 0);
-      // the peer may have a 16 KB copy into this CTA in flight: give it time to land
-      for (int k = 0; k < 100; ++k) __nanosleep(1000);
-    }
-    __syncwarp();
-  }
   tc_fence_before();
   __syncthreads();
-  cluster_sync_all();  // no CTA leaves while its peer may still write to it
+  // This CTA's abort flag no longer changes: hand it to the peer (a store into the peer's
+  // shared memory while both CTAs are certainly resident), then meet.
+  if (threadIdx.x == 0)
+    st_shared_cluster_u32(
+        mapa_shared(smem_u32(const_cast<int*>(&abort_flag->peer_abort)), peer),
+        static_cast<uint32_t>(abort_flag->abort));
+  cluster_sync_all();  // past this point neither CTA issues a copy or an arrival to the other
+  // Abort path, taken by both CTAs when either aborted (each reads both flags from its
+  // own shared memory; neither changes any more).  A stage is reloaded only after the
+  // MMAs that read its previous contents have completed, so at most the last `ns` stage
+  // loads (and the K/V load) can still be in flight: wait for them and for every MMA this
+  // CTA issued (time-limited waits).  Copies between the two CTAs issued before the barrier above may still be
+  // landing, and nothing here can wait for them (they complete on the receiver's
+  // barriers, whose phases an abort leaves unknown): both CTAs stay resident for 50 us,
+  // against about a microsecond per copy, and meet once more before either leaves.
+  const bool any_abort = abort_flag->abort != 0 || abort_flag->peer_abort != 0;
+  if (any_abort) {
+    if (warp == 0 && lane == 0 && n_iter > 0) {
+      mbar_wait_limited(BAR(kBKV), 0);
+      for (int it = max(0, issued - ns); it < issued; ++it)
+        mbar_wait_limited(BAR(kBQF + it % ns), (it / ns) & 1);
+    }
+    if (warp == 1 && n_iter > 0) {
+      tc_fence_after();
+      if (elect_one()) {
+        umma_commit(BAR(kBDrain));
+        mbar_wait_limited(BAR(kBDrain), 0);
+      }
+      __syncwarp();
+    }
+    if (threadIdx.x == 0) {
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 50000) __nanosleep(1000);
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -806,15 +834,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
 
 template <bool DET>
 static int launch_bwd_pair_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    const int rc = cuda_error(cudaFuncSetAttribute(pairbwd::sparse_bwd_pair_kernel<DET>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   pairbwd::kSmem),
-                              "pair backward smem attribute");
-    if (rc) return rc;
-    attr_set = true;
-  }
+  static PerDeviceOnce attr;
+  const int rc = once_per_device(attr, [] {
+    return cuda_error(cudaFuncSetAttribute(pairbwd::sparse_bwd_pair_kernel<DET>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           pairbwd::kSmem),
+                      "pair backward smem attribute");
+  });
+  if (rc) return rc;
   const dim3 grid = DET ? dim3(a.Tn * 2 * a.HK, 1, a.B) : dim3(a.Tn * 2, a.HK, a.B);
   record_event(3, st);
   pairbwd::sparse_bwd_pair_kernel<DET><<<grid, pairbwd::kThreads, pairbwd::kSmem, st>>>(

@@ -188,8 +188,10 @@ extern "C" int index_to_block_sparse(const int32_t* idx, int32_t topk, sa_block_
   if (!idx || topk <= 0 || !out->bitmap) return SA_ERR_INVALID;
   const int64_t W = (out->Sk + 31) / 32;
   if (W * 4 > 96 * 1024) return SA_ERR_UNSUPPORTED;  // one presence row in shared memory
-  out->mode = SA_MODE_INDEX;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  rc = check_stream_device(st);
+  if (rc) return rc;
+  out->mode = SA_MODE_INDEX;
   const int Tm = static_cast<int>((out->Sq + kTile - 1) / kTile);
   const int Tn = static_cast<int>((out->Sk + kTile - 1) / kTile);
   const int64_t rows = static_cast<int64_t>(out->B) * out->Sq * out->HK;
@@ -224,6 +226,8 @@ extern "C" int block_mask_to_block_sparse(sa_block_sparse* out, sa_stream_t stre
     return SA_ERR_INVALID;
   }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  rc = check_stream_device(st);
+  if (rc) return rc;
   const int Tm = static_cast<int>((out->Sq + kTile - 1) / kTile);
   const int Tn = static_cast<int>((out->Sk + kTile - 1) / kTile);
   const int64_t n_tiles = static_cast<int64_t>(out->B) * out->HK * Tm * Tn;

@@ -60,13 +60,14 @@ __device__ __forceinline__ int32_t* det_slot(const AttnArgs& a, int b, int h, in
 
 // Waits until the counter equals `rank` (bounded); then orders the caller's following
 // TMA reduce-adds after the acquire.  False on a timeout or an abort.
-__device__ __forceinline__ bool det_wait_turn(const int32_t* slot, int rank, volatile int* abort,
+__device__ __forceinline__ bool det_wait_turn(const int32_t* slot, int rank, volatile WaitCtl* ctl,
                                               int32_t* status) {
   const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = ctl->limit_ns;
   while (ld_acquire_gpu(slot) != rank) {
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      *abort = 1;
+    if (ctl->abort) return false;
+    if (globaltimer_ns() - t0 > limit) {
+      ctl->abort = 1;
       report_status(status, kStatusTimeout);
       return false;
     }

@@ -68,7 +68,8 @@ __global__ void __launch_bounds__(224, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + C::kBarOff;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * kNumBars);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 8 * kNumBars + 4);
+  volatile WaitCtl* abort_flag =
+      reinterpret_cast<volatile WaitCtl*>(smem + C::kBarOff + 8 * kNumBars + 8);
   auto BAR = [&](int k) { return bar0 + 8u * static_cast<uint32_t>(k); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -80,6 +81,8 @@ __global__ void __launch_bounds__(224, 1)
   const int n_full = __ldg(a.cnt + 2 * lrow);
   const int n_iter = n_full + __ldg(a.cnt + 2 * lrow + 1);
   const int32_t* list = a.idx + lrow * a.Tn;
+  // loads issued by the two producers (the abort path drains the last ones in flight)
+  int issued_k = 0, issued_v = 0;
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(kBQ), 1);
@@ -94,7 +97,8 @@ __global__ void __launch_bounds__(224, 1)
     mbar_init(BAR(kBOD), 1);
     mbar_init(BAR(kBDrain), 1);
     mbar_init(BAR(kBOFin), 1);
-    *abort_flag = 0;
+    abort_flag->abort = 0;
+    abort_flag->limit_ns = a.wait_limit_ns;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -133,12 +137,7 @@ __global__ void __launch_bounds__(224, 1)
                         c * 64, nt * 128, g, b);
         }
         __syncwarp();
-      }
-      if (*abort_flag && lane == 0) {
-        // Let the loads already issued land before the CTA may leave (time-limited).
-        mbar_wait_limited(BAR(kBQ), 0);
-        for (int it = max(0, n_iter - 2); it < n_iter; ++it)
-          mbar_wait_limited(BAR(kBKF + it % C::kKStages), (it / C::kKStages) & 1);
+        issued_k = it + 1;
       }
     }
   } else if (warp == 6) {
@@ -155,10 +154,7 @@ __global__ void __launch_bounds__(224, 1)
                         c * 64, nt * 128, g, b);
         }
         __syncwarp();
-      }
-      if (*abort_flag && lane == 0) {
-        for (int it = max(0, n_iter - 2); it < n_iter; ++it)
-          mbar_wait_limited(BAR(kBVF + it % C::kVStages), (it / C::kVStages) & 1);
+        issued_v = it + 1;
       }
     }
   } else if (warp == 1) {
@@ -205,14 +201,6 @@ __global__ void __launch_bounds__(224, 1)
           umma_commit(BAR(kBOD));
           umma_commit(BAR(kBVE + vs));
           if (it == n_iter - 1) umma_commit(BAR(kBOFin));  // the final O is complete
-        }
-        __syncwarp();
-      }
-      if (*abort_flag) {
-        // Drain: wait (time-limited) for the MMAs issued so far before TMEM is released.
-        if (elect_one()) {
-          umma_commit(BAR(kBDrain));
-          mbar_wait_limited(BAR(kBDrain), 0);
         }
         __syncwarp();
       }
@@ -382,6 +370,34 @@ __global__ void __launch_bounds__(224, 1)
 
   tc_fence_before();
   __syncthreads();
+  // Abort path.  Past the barrier above no warp issues another copy or MMA, and the
+  // abort flag no longer changes (the branch is uniform).  A K or V buffer is reloaded
+  // only after the MMA that read its previous tile has completed, so at most the last
+  // kKStages K loads and kVStages V loads can still be in flight: wait for them, and for
+  // every MMA this CTA issued, before shared memory and TMEM are released
+  // (time-limited waits).
+  if (abort_flag->abort) {
+    if (n_iter > 0 && lane == 0) {
+      if (warp == 0) {
+        mbar_wait_limited(BAR(kBQ), 0);
+        for (int it = max(0, issued_k - C::kKStages); it < issued_k; ++it)
+          mbar_wait_limited(BAR(kBKF + it % C::kKStages), (it / C::kKStages) & 1);
+      } else if (warp == 6) {
+        for (int it = max(0, issued_v - C::kVStages); it < issued_v; ++it)
+          mbar_wait_limited(BAR(kBVF + it % C::kVStages), (it / C::kVStages) & 1);
+      }
+    }
+    if (warp == 1 && n_iter > 0) {
+      tc_fence_after();
+      if (elect_one()) {
+        umma_commit(BAR(kBDrain));
+        mbar_wait_limited(BAR(kBDrain), 0);
+      }
+      __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
@@ -391,15 +407,13 @@ __global__ void __launch_bounds__(224, 1)
 template <int DQK, int DV>
 static int launch_fwd_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
   using C = FwdCfg<DQK, DV>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    const int rc = cuda_error(cudaFuncSetAttribute(sparse_fwd_kernel<DQK, DV>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   C::kSmem),
-                              "forward smem attribute");
-    if (rc) return rc;
-    attr_set = true;
-  }
+  static PerDeviceOnce attr;
+  const int rc = once_per_device(attr, [] {
+    return cuda_error(cudaFuncSetAttribute(sparse_fwd_kernel<DQK, DV>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem),
+                      "forward smem attribute");
+  });
+  if (rc) return rc;
   dim3 grid(a.Tm, a.HQ, a.B);
   record_event(0, st);
   sparse_fwd_kernel<DQK, DV><<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.v, m.o, a);

@@ -17,8 +17,18 @@ namespace sa {
 constexpr int kTile = 128;
 
 // Bounded waits: a wait that has not completed after this many nanoseconds gives up,
-// records SA_ERR_TIMEOUT in the caller's status word and makes the CTA leave.
+// records SA_ERR_TIMEOUT in the caller's status word and makes the CTA leave.  This is
+// the default; a launch may carry a shorter limit (AttnArgs::wait_limit_ns).  The
+// drains of the abort path always use this default.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Per-CTA wait control, kept in shared memory: the abort flag every bounded wait of
+// the CTA watches, and this launch's wait limit.
+struct WaitCtl {
+  int abort;
+  int peer_abort;  // 2-CTA kernels: the other CTA's final abort flag, stored there by it
+  uint64_t limit_ns;
+};
 
 // Device status bits (OR-ed into the caller's int32 status word).
 constexpr int kStatusIndex = 1;    // an index outside [-1, Sk)
@@ -58,17 +68,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 // try_wait with a suspend-time hint: a waiting thread sleeps in hardware (up to the
-// hint, 0.5 ms) until the phase completes instead of spinning on issue slots that the
-// working warps of its SM sub-partition need.
+// hint, at most 0.5 ms) until the phase completes instead of spinning on issue slots
+// that the working warps of its SM sub-partition need.
 constexpr uint32_t kSuspendHintNs = 500000;
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity,
+                                              uint32_t hint_ns = kSuspendHintNs) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
@@ -87,17 +98,19 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 }
 
 // Waits until the phase of parity `parity` of the barrier has completed.  Gives up
-// (returns false) when *abort becomes non-zero or after kWaitLimitNs; on a timeout it
-// sets *abort and reports SA_ERR_TIMEOUT through `status`.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+// (returns false) when ctl->abort becomes non-zero or after ctl->limit_ns; on a timeout
+// it sets ctl->abort and reports SA_ERR_TIMEOUT through `status`.  The hardware suspend
+// hint never exceeds the limit, so a wait gives up within about twice the limit.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile WaitCtl* ctl,
                                           int32_t* status) {
-  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t limit = ctl->limit_ns;
+  const uint32_t hint = limit < kSuspendHintNs ? static_cast<uint32_t>(limit) : kSuspendHintNs;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      *abort = 1;
+    if (mbar_try_wait(bar, parity, hint)) return true;
+    if (ctl->abort) return false;
+    if (globaltimer_ns() - t0 > limit) {
+      ctl->abort = 1;
       report_status(status, kStatusTimeout);
       return false;
     }
@@ -115,9 +128,9 @@ __device__ __forceinline__ bool mbar_wait_limited(uint32_t bar, uint32_t parity)
 }
 
 // Warp-collective form: every lane waits; the result is the same on every lane.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile WaitCtl* ctl,
                                           int32_t* status) {
-  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort, status));
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, ctl, status));
 }
 
 // Picks one active lane of a converged warp (true on that lane only).
@@ -162,6 +175,11 @@ __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t remote_dst, uint32
           remote_dst),
       "r"(local_src), "r"(bytes), "r"(remote_bar)
       : "memory");
+}
+// Store of a 32-bit word into the shared memory of a CTA of the cluster (address from
+// mapa_shared).
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");

@@ -323,15 +323,16 @@ extern "C" int topk_select(const float* scores, int64_t rows, int64_t cols, int6
   int kp = 2;
   while (kp < k) kp <<= 1;
   const size_t smem = static_cast<size_t>(kp) * sizeof(uint64_t);
-  static bool attr_set = false;
-  if (!attr_set) {
-    const int rc = cuda_error(cudaFuncSetAttribute(topk::topk_kernel,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   SA_TOPK_MAX_K * static_cast<int>(sizeof(uint64_t))),
-                              "top-k smem attribute");
-    if (rc) return rc;
-    attr_set = true;
-  }
+  const int drc = check_stream_device(reinterpret_cast<cudaStream_t>(stream));
+  if (drc) return drc;
+  static PerDeviceOnce attr;
+  const int rc = once_per_device(attr, [] {
+    return cuda_error(cudaFuncSetAttribute(topk::topk_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           SA_TOPK_MAX_K * static_cast<int>(sizeof(uint64_t))),
+                      "top-k smem attribute");
+  });
+  if (rc) return rc;
   topk::topk_kernel<<<static_cast<unsigned>(rows), topk::kThreads, smem,
                       reinterpret_cast<cudaStream_t>(stream)>>>(scores, ld, cols, starts, ends, k, kp,
                                                                out_idx, out_val, dev_status);

@@ -14,8 +14,12 @@ Structures (the workloads the pages and the benchmark are about):
     kept with probability ``density``; diagonal blocks are always kept; with
     ``causal`` only the lower triangle is eligible.
   * index mode: per (query, KV head), ``topk`` distinct int32 key positions drawn
-    uniformly from the causal range [0, q], stored in random order, with -1 padding
-    at the tail when fewer than ``topk`` are valid.  This is the int32 / -1 output
+    uniformly from the causal range [0, q] (``span="causal"``) or from every key
+    [0, Sk) (``span="all"``: entries above the diagonal, which a causal call must mask
+    and a non-causal call must attend), stored in random order, with -1 padding at the
+    tail when fewer than ``topk`` are valid.  With ``dup`` > 0 each filled slot is,
+    with that probability, overwritten by a copy of a random slot of its own row, so
+    rows hold repeated keys (the attended set is still the row's set of keys).  This is the int32 / -1 output
     format of the Top-K selector in xtuner PR #2096 ("Add optional TileLang Top-K
     selector", Main Changes 1) that feeds IndexSparse attention (MagiAttention
     PR #334, section 2).
@@ -40,6 +44,8 @@ class Workload:
     bs: int = 128  # block-mask granularity (block mode)
     density: float = 1.0  # keep probability of an eligible off-diagonal block
     topk: int = 0  # index mode
+    span: str = "causal"  # index mode: keys drawn from [0, q] ("causal") or [0, Sk) ("all")
+    dup: float = 0.0  # index mode: probability that a slot repeats another key of its row
     seed: int = 0
     tags: tuple = field(default_factory=tuple)
 
@@ -108,9 +114,11 @@ def block_mask(w: Workload) -> np.ndarray:
 
 
 def topk_indices(w: Workload, rows_per_chunk: int = 4096) -> np.ndarray:
-    """int32 [B, Sq, HK, topk]: distinct keys drawn uniformly from [0, q], -1 padded.
+    """int32 [B, Sq, HK, topk]: distinct keys drawn uniformly from [0, q] (or [0, Sk)
+    with span "all"), -1 padded, optionally with repeated entries (``dup``).
 
-    Each (query, KV head) row with n = min(q, Sk-1) + 1 candidates draws
+    Each (query, KV head) row with n = min(q, Sk-1) + 1 candidates (n = Sk with span
+    "all") draws
     k = min(n, topk) of them by R. W. Floyd's sampling algorithm (step s: draw t
     uniformly from [0, n-k+s]; take t unless already taken, else take n-k+s), which
     yields every k-subset with equal probability; the k entries are then put in a
@@ -119,7 +127,12 @@ def topk_indices(w: Workload, rows_per_chunk: int = 4096) -> np.ndarray:
     """
     rng = np.random.default_rng(w.seed + 4)
     out = np.full((w.B, w.Sq, w.HK, w.topk), -1, dtype=np.int32)
-    n_all = np.repeat(np.minimum(np.arange(w.Sq), w.Sk - 1) + 1, w.HK).astype(np.int64)
+    if w.span == "causal":
+        n_all = np.repeat(np.minimum(np.arange(w.Sq), w.Sk - 1) + 1, w.HK).astype(np.int64)
+    elif w.span == "all":
+        n_all = np.full(w.Sq * w.HK, w.Sk, dtype=np.int64)
+    else:
+        raise ValueError(f"span must be 'causal' or 'all', got {w.span!r}")
     for b in range(w.B):
         sel_b = out[b].reshape(-1, w.topk)
         for r0 in range(0, len(n_all), rows_per_chunk):
@@ -142,6 +155,14 @@ def topk_indices(w: Workload, rows_per_chunk: int = 4096) -> np.ndarray:
             for r in np.nonzero(~full)[0]:
                 sel[r, :k[r]] = rng.permutation(sel[r, :k[r]])
             sel_b[r0:r0 + rows] = sel
+    if w.dup > 0:
+        flat = out.reshape(-1, w.topk)
+        filled = np.count_nonzero(flat >= 0, axis=1)
+        slot = np.arange(w.topk)[None, :]
+        over = (rng.random(flat.shape) < w.dup) & (slot < filled[:, None])
+        src = np.minimum((rng.random(flat.shape) * filled[:, None]).astype(np.int64),
+                         np.maximum(filled[:, None] - 1, 0))
+        flat[over] = np.take_along_axis(flat, src, axis=1)[over]
     return out
 
 

@@ -39,3 +39,21 @@ def test_traffic_reported_only_for_the_measured_code(tmp_path, monkeypatch):
     assert bench.profiled_traffic("another_workload") is None
     (prof / "bwd_main_traffic.json").write_text(json.dumps(dict(d, source_sha="old")))
     assert bench.profiled_traffic(d["workload"]) is None
+
+
+def test_peak_basis_follows_the_runs_own_clock_record():
+    """Burst peak unless the timed region saw power capping; then the sustained one."""
+    peaks = {"bf16_tflops": 1661.7, "bf16_tflops_sustained": 1406.6}
+    assert bench.peak_basis(peaks, {"reasons": []}) == (1661.7, "bf16_tflops")
+    assert bench.peak_basis(peaks, None) == (1661.7, "bf16_tflops")
+    assert bench.peak_basis(peaks, {"reasons": ["sw_power_cap"]}) == (1406.6,
+                                                                      "bf16_tflops_sustained")
+
+
+def test_converter_bytes_index_workload():
+    from index_sparse_attention_b200 import inputs as I
+    w = I.WORKLOADS["indexsparse_gqa_q16384_hq32_hk4_d192_128_top2048"]
+    idx = 16384 * 4 * 2048 * 4          # 512 MiB of indices, read once
+    bitmap = 4 * 16384 * 512 * 4        # 128 MiB, written and read back once
+    lists = 4 * 4 * (128 * 130 + 128 * 130)
+    assert bench.converter_bytes(w) == idx + 2 * bitmap + 2 * lists

@@ -111,3 +111,47 @@ def test_mismatched_shapes_are_rejected(cuda_check_off):
         sa._params(q, k, v, o, lse, None, 0.1)
     with pytest.raises(TypeError, match="dev_status must be torch.int32"):
         sa._params(q, k, v, o, lse, bsp, 0.1, dev_status=torch.zeros(1))
+
+
+ENTRY_POINTS = ("block_mask_to_block_sparse", "index_to_block_sparse", "sparse_attn_fwd",
+                "sparse_attn_bwd_workspace_size", "sparse_attn_bwd", "sparse_attn_bwd_noalloc",
+                "topk_select")
+
+
+def test_every_entry_point_runs_on_its_tensors_device():
+    """The C ABI launches on the current device, so each binding entry point makes the
+    device of its tensor argument current for the call."""
+    for name in ENTRY_POINTS:
+        fn = getattr(sa, name)
+        assert getattr(fn, "device_arg", None), f"{name} has no device guard"
+
+
+def test_device_guard_enters_the_tensor_device(monkeypatch):
+    entered = []
+
+    class Recorder:
+        def __init__(self, dev):
+            self.dev = dev
+
+        def __enter__(self):
+            entered.append(self.dev)
+
+        def __exit__(self, *exc):
+            return False
+
+    class FakeCuda(torch.Tensor):
+        @property
+        def is_cuda(self):
+            return True
+
+        @property
+        def device(self):
+            return torch.device("cuda", 3)
+
+    monkeypatch.setattr(torch.cuda, "device", Recorder)
+    t = torch.zeros(2).as_subclass(FakeCuda)
+    guarded = sa._on_device("x")(lambda a, x=None: (a, x))
+    assert guarded(1, x=t)[0] == 1 and entered == [torch.device("cuda", 3)]
+    assert guarded(1, t)[0] == 1 and len(entered) == 2
+    guarded(1, x=torch.zeros(2))  # a CPU tensor: no device switch
+    assert len(entered) == 2

@@ -72,21 +72,36 @@ def test_backward_small(w):
     assert_close("dQ", dq, rQ)
 
 
+def _rows_attending(w, inp, b, g, keys_j):
+    """Query rows i (of batch b, KV head g) whose allowed set may hold one of the keys:
+    a superset read off the block mask or the index tensor (the causal cut is left to
+    the oracle)."""
+    need = np.zeros(w.Sq, bool)
+    for j in keys_j:
+        if w.mode == "block":
+            col = inp.mask[b, g, :, j // w.bs].astype(bool)          # per query block
+            need |= np.repeat(col, w.bs)[:w.Sq]
+        else:
+            need |= (inp.idx[b, :, g, :] == j).any(axis=1)
+    return np.nonzero(need)[0]
+
+
 def _sampled_reference(w, inp, n_rows=24):
-    """Oracle dQ at sampled rows and dK/dV at sampled keys of KV head 0 of batch B-1."""
+    """Oracle dQ at sampled rows and dK/dV at sampled keys of KV head 0 of batch B-1.
+
+    The keys span the sequence: key tile 0 (under causal masking the longest transposed
+    list, so the deepest dK/dV accumulation), a mid-sequence tile and the last keys.
+    The oracle's LSE and Delta are evaluated at every row that can attend them."""
     P = oracle_problem(inp)
     rng = np.random.default_rng(7)
     G = w.HQ // w.HK
     b, g = w.B - 1, 0
-    if w.causal:  # keys near the end: few query rows attend them
-        keys_j = np.array([w.Sk - 300, w.Sk - 129, w.Sk - 100, w.Sk - 1], dtype=np.int64)
-    else:
-        keys_j = np.array([5, 200, w.Sk // 2 + 3, w.Sk - 1], dtype=np.int64)
-    keys_j = np.clip(keys_j, 0, w.Sk - 1)
+    mid = (w.Sk // 256) * 128  # first key of a mid-sequence tile
+    keys_j = np.unique(np.clip(np.array([0, 5, 127, mid + 3, mid + 100, w.Sk - 129, w.Sk - 1]),
+                               0, w.Sk - 1)).astype(np.int64)
     keys = np.stack([np.full(len(keys_j), b), np.full(len(keys_j), g), keys_j], 1)
-    jmin = int(keys_j.min()) if w.causal else 0
-    # every (b, h in group g, i) that can attend a sampled key
-    hh, ii = np.meshgrid(np.arange(g * G, (g + 1) * G), np.arange(jmin, w.Sq), indexing="ij")
+    ii = _rows_attending(w, inp, b, g, keys_j)
+    hh, ii = np.meshgrid(np.arange(g * G, (g + 1) * G), ii, indexing="ij")
     rows_k = np.stack([np.full(hh.size, b), hh.ravel(), ii.ravel()], 1)
     rows_q = np.stack([rng.integers(0, w.B, n_rows), rng.integers(0, w.HQ, n_rows),
                        rng.integers(0, w.Sq, n_rows)], 1)

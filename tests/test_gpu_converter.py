@@ -21,7 +21,7 @@ SMALL = [
     I.scaled(W["indexsparse_gqa_q16384_hq32_hk4_d192_128_top2048"], Sq=600, Sk=600, HQ=2, HK=1,
              topk=700, name="index_topk_gt_seq"),
     I.scaled(W["indexsparse_gqa_q16384_hq32_hk4_d192_128_top2048"], Sq=256, Sk=256, HQ=2, HK=2,
-             topk=64, causal=False, name="index_noncausal"),
+             topk=64, causal=False, span="all", dup=0.2, name="index_noncausal"),
 ]
 FULL = [W[k] for k in ("blocksparse_mha_s256_d64", "dense_full_b2_h16_s4096_d128",
                        "dense_causal_b2_h16_s4096_d128", "gqa_blocksparse_b2_hq32_hk8_s8192_d128",

@@ -80,3 +80,36 @@ def test_topk_score_distributions():
     assert len(np.unique(x)) < x.size // 3
     y = I.topk_scores(64, 512, seed=1)
     assert abs(float(y.mean())) < 0.05 and abs(float(y.std()) - 1.0) < 0.05
+
+
+def test_topk_index_span_all_and_duplicates():
+    """span "all": distinct keys of every position [0, Sk), above the diagonal too;
+    dup > 0: repeated keys inside a row, drawn from that row's own set, -1 tail kept."""
+    base = I.scaled(I.WORKLOADS["indexsparse_gqa_q16384_hq32_hk4_d192_128_top2048"], B=1,
+                    Sq=300, Sk=260, HQ=2, HK=1, topk=40, span="all")
+    idx = I.topk_indices(base)
+    above = 0
+    counts = np.zeros(260)
+    for i in range(300):
+        row = idx[0, i, 0]
+        assert (row >= 0).all() and row.max() < 260            # k = min(Sk, topk) = 40
+        assert len(set(row.tolist())) == 40                     # distinct
+        above += int((row > i).sum())
+        counts[row] += 1
+    assert above > 40 * 40                                      # entries above the diagonal
+    expect = 300 * 40 / 260                                     # per key; sd about 6.2
+    assert np.abs(counts - expect).max() < 5 * np.sqrt(expect * (1 - 40 / 260))  # uniform
+    dup = I.topk_indices(I.scaled(base, dup=0.3))
+    assert dup.shape == idx.shape
+    n_dup_rows = 0
+    for i in range(300):
+        row, ref = dup[0, i, 0], idx[0, i, 0]
+        assert set(row.tolist()) <= set(ref.tolist())           # copies of the row's own keys
+        n_dup_rows += len(set(row.tolist())) < 40
+    assert n_dup_rows > 290                                     # almost every row repeats keys
+    # the -1 tail survives duplication (topk > Sk: 260 keys then 40 pads)
+    big = I.topk_indices(I.scaled(base, topk=300, dup=0.3))
+    assert (big[0, :, 0, 260:] == -1).all() and (big[0, :, 0, :260] >= 0).all()
+    # the default span and dup leave the causal recipe untouched
+    causal = I.topk_indices(I.scaled(base, span="causal"))
+    assert all(causal[0, i, 0][causal[0, i, 0] >= 0].max() <= i for i in range(300))
