@@ -225,10 +225,13 @@ int sparse_attn_set_timing_events(void *const *events);
  * copies and tensor-core operations it has in flight and leaves (the outputs of that
  * call are then undefined, the CUDA context stays usable).  The default limit is 2 s.
  * This call sets the limit, in nanoseconds, for the calls enqueued after it (0 restores
- * the default).  A limit of a few microseconds makes ordinary waits run out: that is
- * how the tests exercise the timeout path.  Process-wide; returns SA_OK.
+ * the default).  A limit below 1000 ns means that a wait gives up at its first test if
+ * the phase it waits for has not completed: ordinary waits (a TMA load just issued, the
+ * first MMA) then run out, which is how the tests exercise the timeout path.
+ * Process-wide; returns SA_OK.
  */
 int sparse_attn_set_wait_limit_ns(uint64_t ns);
+
 
 /* Largest k that topk_select supports. */
 #define SA_TOPK_MAX_K 4096

@@ -123,12 +123,16 @@ struct BwdCfg {
   static constexpr int kVBytes = 128 * DV * 2;
   static constexpr int kQBytes = kBM * DQK * 2;
   static constexpr int kOBytes = kBM * DV * 2;
-  // Q/dO stages: three at D=128, two at (192,128)
-  static constexpr int kStages = DQK == 128 ? 3 : 2;
+  // (192,128): V is held in TMEM (columns kColV, bf16 pairs) and dP^T = V dO^T reads it
+  // from there, which leaves shared memory for a third Q/dO stage (the kernel is bound by
+  // how long a stage is held: load latency plus one step).  V first lands in the last
+  // stage's region and is copied into TMEM by the elementwise warps.
+  static constexpr bool kVT = DQK == 192;
+  static constexpr int kStages = 3;
   static constexpr int kDSBytes = 128 * kBM * 2;     // dS^T [128 keys][64 q] bf16 (16 KB)
   static constexpr int kKOff = 0;
-  static constexpr int kVOff = kKOff + kKBytes;
-  static constexpr int kQOff = kVOff + kVBytes;                    // per stage: Q then dO
+  static constexpr int kQOff = kKOff + kKBytes + (kVT ? 0 : kVBytes);  // per stage: Q then dO
+  static constexpr int kVOff = kVT ? kQOff + (kStages - 1) * (kQBytes + kOBytes) : kKOff + kKBytes;
   static constexpr int kStageBytes = kQBytes + kOBytes;
   static constexpr int kDSOff = kQOff + kStages * kStageBytes;     // two dS^T buffers
   // fp32 dQ staging tile [2 panels][32 q][64 d]
@@ -146,15 +150,20 @@ struct BwdCfg {
   static constexpr uint32_t kColDP = 128;  // + 64 * buffer
   static constexpr uint32_t kColDK = 256;
   static constexpr uint32_t kColDV = kColDK + kDKMax;
+  static constexpr uint32_t kColV = kColDV + kDVMax;  // V (kVT), DV / 2 columns
   static constexpr uint32_t kTmemCols = 512;
   static_assert(DQK + DV < 512, "head dims 256/256 run in the 2-CTA kernel");
   static_assert(kColDV + kDVMax <= kTmemCols, "tensor memory budget");
+  static_assert(!kVT || kColV + DV / 2 <= kTmemCols, "tensor memory budget (V)");
+  static_assert(!kVT || kVBytes <= kQBytes + kOBytes, "V lands in one stage's region");
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
 
 enum : int {
   kBKV = 0, kBQF = 1, kBQE = 4, kBLF = 7, kBSF = 10, kBPF = 12, kBDQF = 14, kBDQE = 16,
-  kBFin = 18, kBDrainB = 19, kNumBarsB = 20
+  kBFin = 18, kBDrainB = 19,
+  kBVT = 20,  // V copied into TMEM (256 elementwise threads; (192,128) only)
+  kNumBarsB = 21
 };
 
 // Warp roles: 0 producer, 1 MMA, 2-9 elementwise (one key row and 32 of the 64 query
@@ -232,6 +241,7 @@ __global__ void __launch_bounds__(448, 1)
     }
     mbar_init(BAR(kBFin), 1);
     mbar_init(BAR(kBDrainB), 1);
+    mbar_init(BAR(kBVT), 256);
     abort_flag->abort = 0;
     abort_flag->limit_ns = a.wait_limit_ns;
     fence_mbar_init();
@@ -288,6 +298,9 @@ __global__ void __launch_bounds__(448, 1)
         const int st = it % C::kStages, u = it / C::kStages;
         const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
         if (!warp_wait(BAR(kBQE + st), (u & 1) ^ 1, abort_flag, a.status)) break;
+        // (192,128): V occupies the last stage until it has been copied into TMEM
+        if (C::kVT && it == C::kStages - 1 && !warp_wait(BAR(kBVT), 0, abort_flag, a.status))
+          break;
         if (elect_one()) {
           mbar_arrive_expect_tx(BAR(kBQF + st), C::kQBytes + C::kOBytes);
           for (int c = 0; c < DQK / 64; ++c)
@@ -339,6 +352,7 @@ __global__ void __launch_bounds__(448, 1)
       const uint64_t kd = sw128_desc(kbase, 16, 1024), vd = sw128_desc(vbase, 16, 1024);
       const uint64_t kwd = sw128_desc(kbase + (qw0 / 64) * C::kKPanel, C::kKPanel, 1024);
       bool ok = warp_wait(BAR(kBKV), 0, abort_flag, a.status);
+      if (C::kVT) ok = ok && warp_wait(BAR(kBVT), 0, abort_flag, a.status);
       // S^T(j) and dP^T(j) into TMEM buffer j & 1
       auto issue_sdp = [&](int j) -> bool {
         const int st = j % C::kStages, u = j / C::kStages, bj = j & 1;
@@ -362,8 +376,12 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const uint32_t va = p * C::kKPanel + k4 * 32, ob = p * C::kQPanel + k4 * 32;
-              umma_ss(tmem + C::kColDP + 64 * bj, vd + (va >> 4), od + (ob >> 4), idesc_s,
-                      (p > 0 || k4 > 0) ? 1u : 0u);
+              if constexpr (C::kVT)  // A = V from TMEM: 16 head dims = 8 columns per k-step
+                umma_ts(tmem + C::kColDP + 64 * bj, tmem + C::kColV + (p * 4 + k4) * 8,
+                        od + (ob >> 4), idesc_s, (p > 0 || k4 > 0) ? 1u : 0u);
+              else
+                umma_ss(tmem + C::kColDP + 64 * bj, vd + (va >> 4), od + (ob >> 4), idesc_s,
+                        (p > 0 || k4 > 0) ? 1u : 0u);
             }
           }
           umma_commit(BAR(kBSF + bj));
@@ -416,7 +434,30 @@ __global__ void __launch_bounds__(448, 1)
     const uint32_t* bmbuf = reinterpret_cast<const uint32_t*>(smem + C::kBMOff);
     const bool key_ok = j < a.Sk;
     bool ok = true;
-    for (int it = 0; it < n_iter; ++it) {
+    if (C::kVT && n_iter > 0) {
+      // V row r into TMEM (row r in lane r, head dims 2e, 2e+1 in column e): this half of
+      // the warps copies the 64-column panel hc from the swizzled smem tile
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(BAR(kBKV), 0, abort_flag, a.status));
+      if (ok) {
+        const uint8_t* prow = smem + C::kVOff + hc * C::kKPanel + r * 128;
+        uint32_t w[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint4 v = *reinterpret_cast<const uint4*>(prow + ((k ^ (r & 7)) << 4));
+          w[4 * k] = v.x;
+          w[4 * k + 1] = v.y;
+          w[4 * k + 2] = v.z;
+          w[4 * k + 3] = v.w;
+        }
+        tmem_st32(tl + C::kColV + hc * 32, w);
+        tmem_wait_st();
+      }
+      // the stage region V occupied is reloaded by TMA next
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(BAR(kBVT));
+    }
+    for (int it = 0; ok && it < n_iter; ++it) {
       int h, m0;
       bool partial;
       decode(it, h, m0, partial);

@@ -340,7 +340,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       ok = ok && warp_wait(BAR(kBVT), 0, abort_flag, a.status);
       int js = 0;  // next S^T (rank 0) / dP^T (rank 1)
       int jv = 0;  // rank 1: next dV
-      int jk = 0;  // next dK + dQ^T (rank 0) / dQ^T (rank 1)
+      int jk = 0;  // next dQ^T
+      int jd = 0;  // rank 0: next dK (issued ahead of its dQ^T)
       int jx = 0;  // rank 0: next step whose dS^T arrival is reported back to rank 1
       int jp = 0;  // rank 1: next step whose P^T tile is handed back to rank 0
       uint64_t t_last = globaltimer_ns();
@@ -385,27 +386,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
           ++jv;
           prog = true;
         }
-        // rank 0: dK += dS^T Q and dQ^T once dS^T has arrived and the last dQ^T has been
-        // drained; rank 1: dQ^T once its elementwise warps have written dS^T
-        if (rank == 0 ? (jk < jx && (jk == 0 || ready(kBDQE, (jk - 1) & 1)))
+        // rank 0: dK += dS^T Q as soon as dS^T has arrived (it frees the Q stage); it does
+        // not wait for the single dQ^T buffer to be drained
+        if (rank == 0 && jd < jx) {
+          tc_fence_after();
+          const uint32_t xt = sbase + kOffX0 + (jd % kNX) * kTile;
+          const uint64_t xk = sw128_desc(xt, 16, 1024);  // exchange tile, K-major A
+          const uint64_t bmn = sw128_desc(sbase + off_stage + (jd % ns) * kStageBytes, kQPanel, 1024);
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < BM / 16; ++kk)
+              umma_ss(tmem + col_acc, xk + ((kk * 32) >> 4), bmn + ((kk * 2048) >> 4), idesc_acc,
+                      (jd > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(BAR(kBQE + jd % ns));  // Q stage free
+          }
+          __syncwarp();
+          ++jd;
+          prog = true;
+        }
+        // dQ^T: rank 0 once its dK is issued (the tensor pipe runs in order, so that dK has
+        // read the tile before the drain stages into it) and the last dQ^T has been
+        // drained; rank 1 once its elementwise warps have written dS^T
+        if (rank == 0 ? (jk < jd && (jk == 0 || ready(kBDQE, (jk - 1) & 1)))
                       : (jk < jv && ready(kBEW + jk % ns, (jk / ns) & 1))) {
           tc_fence_after();
           // rank 0: the dS^T that arrived in its tile; rank 1: its own dS^T tile
           const uint32_t xt = rank == 0 ? sbase + kOffX0 + (jk % kNX) * kTile
                                         : sbase + kOffDO1 + (jk % kNDO) * kTile;
           const uint64_t xmn = sw128_desc(xt, kKPanel, 1024);  // exchange tile, MN-major B
-          if (rank == 0) {
-            const uint64_t xk = sw128_desc(xt, 16, 1024);      // exchange tile, K-major A
-            const uint64_t bmn = sw128_desc(sbase + off_stage + (jk % ns) * kStageBytes, kQPanel, 1024);
-            if (elect_one()) {
-#pragma unroll
-              for (int kk = 0; kk < BM / 16; ++kk)
-                umma_ss(tmem + col_acc, xk + ((kk * 32) >> 4), bmn + ((kk * 2048) >> 4), idesc_acc,
-                        (jk > 0 || kk > 0) ? 1u : 0u);
-              umma_commit(BAR(kBQE + jk % ns));  // Q stage free
-            }
-            __syncwarp();
-          }
           const uint32_t dq_col = rank == 0 ? kColDQ0 : kColP1 + 64 * (jk & 1);
           if (elect_one()) {
 #pragma unroll
@@ -422,7 +430,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         // S^T (rank 0) / dP^T (rank 1) of the next step: stage loaded, TMEM buffer free
         // (rank 0: loaded by the elementwise warps; rank 1: its dQ^T drained), not too far
         // ahead of the dK / dV stream
-        if (js < n_iter && js <= (rank == 0 ? jk + kLookS0 : jv + kLookS1) &&
+        if (js < n_iter && js <= (rank == 0 ? jd + kLookS0 : jv + kLookS1) &&
             ready(kBQF + js % ns, (js / ns) & 1) &&
             (rank == 0 ? (js == 0 || ready(kBSR, (js - 1) & 1))
                        : (js < 2 || ready(kBDQE + (js & 1), ((js - 2) >> 1) & 1)))) {
@@ -451,10 +459,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         } else {
           if (__shfl_sync(0xFFFFFFFFu, abort_flag->abort, 0) != 0) break;
           if (globaltimer_ns() - t_last > abort_flag->limit_ns) {
-            if (lane == 0) {
-              abort_flag->abort = 1;
-              report_status(a.status, kStatusTimeout);
-            }
+            if (lane == 0) wait_timed_out(abort_flag, a.status);
             __syncwarp();
             break;
           }

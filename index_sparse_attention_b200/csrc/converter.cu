@@ -18,36 +18,86 @@ namespace sa {
 
 constexpr int kAbsent = 0, kPartial = 1, kFull = 2;
 
-// One CTA per (b, i, g): the W-word presence row of query i under KV head g.
-__global__ void scatter_bits_kernel(const int32_t* __restrict__ idx, uint32_t* __restrict__ bitmap,
-                                    int64_t Sq, int64_t Sk, int HK, int topk, int W,
-                                    int32_t* status) {
+// One CTA of kScatterThreads per (b, i, g): the W-word presence row of query i under KV
+// head g.  Every thread's index loads are issued before any of their bits is set (16-byte
+// loads when the rows allow), so a row costs one memory latency, not one per index.
+constexpr int kScatterThreads = 128;
+constexpr int kScatterUnroll = 4;
+
+__device__ __forceinline__ void set_presence_bit(uint32_t* words, int32_t j, int64_t Sk,
+                                                 int32_t* status) {
+  if (j == -1) return;
+  if (j < -1 || j >= Sk) {
+    report_status(status, kStatusIndex);
+    return;
+  }
+  atomicOr(&words[j >> 5], 1u << (j & 31));
+}
+
+__global__ void __launch_bounds__(kScatterThreads)
+    scatter_bits_kernel(const int32_t* __restrict__ idx, uint32_t* __restrict__ bitmap,
+                        int64_t Sq, int64_t Sk, int HK, int topk, int W, int vec,
+                        int32_t* status) {
   extern __shared__ uint32_t words[];
   const int64_t row = blockIdx.x;  // ((b * Sq) + i) * HK + g, the order of idx
   const int g = static_cast<int>(row % HK);
   const int64_t bi = row / HK;  // b * Sq + i
   const int64_t b = bi / Sq, i = bi % Sq;
-  for (int w = threadIdx.x; w < W; w += blockDim.x) words[w] = 0u;
+  for (int w = threadIdx.x; w < W; w += kScatterThreads) words[w] = 0u;
   __syncthreads();
   const int32_t* src = idx + row * topk;
-  for (int t = threadIdx.x; t < topk; t += blockDim.x) {
-    const int32_t j = __ldg(src + t);
-    if (j == -1) continue;
-    if (j < -1 || j >= Sk) {
-      report_status(status, kStatusIndex);
-      continue;
+  if (vec) {  // topk % 4 == 0 and a 16-byte aligned base: rows of int4
+    const int4* s4 = reinterpret_cast<const int4*>(src);
+    const int n4 = topk >> 2;
+    for (int base = 0; base < n4; base += kScatterUnroll * kScatterThreads) {
+      int4 v[kScatterUnroll];
+#pragma unroll
+      for (int u = 0; u < kScatterUnroll; ++u) {
+        const int e = base + u * kScatterThreads + threadIdx.x;
+        v[u] = e < n4 ? __ldg(s4 + e) : make_int4(-1, -1, -1, -1);
+      }
+#pragma unroll
+      for (int u = 0; u < kScatterUnroll; ++u) {
+        set_presence_bit(words, v[u].x, Sk, status);
+        set_presence_bit(words, v[u].y, Sk, status);
+        set_presence_bit(words, v[u].z, Sk, status);
+        set_presence_bit(words, v[u].w, Sk, status);
+      }
     }
-    atomicOr(&words[j >> 5], 1u << (j & 31));
+  } else {
+    for (int base = 0; base < topk; base += kScatterUnroll * kScatterThreads) {
+      int32_t v[kScatterUnroll];
+#pragma unroll
+      for (int u = 0; u < kScatterUnroll; ++u) {
+        const int t = base + u * kScatterThreads + threadIdx.x;
+        v[u] = t < topk ? __ldg(src + t) : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < kScatterUnroll; ++u) set_presence_bit(words, v[u], Sk, status);
+    }
   }
   __syncthreads();
   uint32_t* dst = bitmap + (((b * HK + g) * Sq) + i) * static_cast<int64_t>(W);
-  for (int w = threadIdx.x; w < W; w += blockDim.x) dst[w] = words[w];
+  for (int w = threadIdx.x; w < W; w += kScatterThreads) dst[w] = words[w];
 }
 
-// One CTA per (b, g, mt): classify every key tile of the query tile from the bitmap.
+// Bits of the 32 keys [j0, j0 + 32) of query i that are allowed: set in the presence
+// word, below Sk and, when causal, at most i.  `in_range` receives the bits below Sk.
+__device__ __forceinline__ uint32_t allowed_bits(uint32_t bits, int64_t i, int64_t j0, int64_t Sk,
+                                                 int causal, uint32_t& in_range) {
+  const int64_t n_in = min64(32, Sk - j0);
+  in_range = n_in >= 32 ? 0xFFFFFFFFu : (n_in <= 0 ? 0u : ((1u << n_in) - 1u));
+  const int64_t n_c = causal ? min64(32, max64(0, i + 1 - j0)) : 32;
+  const uint32_t causal_ok = n_c >= 32 ? 0xFFFFFFFFu : ((1u << n_c) - 1u);
+  return bits & in_range & causal_ok;
+}
+
+// One CTA per (b, g, mt): classify every key tile of the query tile from the bitmap.  A
+// key tile is 4 words of a row: with W % 4 == 0 each thread reads one (row, key tile)
+// as a 16-byte load.
 __global__ void classify_index_kernel(const uint32_t* __restrict__ bitmap, int32_t* __restrict__ cls,
                                       int64_t Sq, int64_t Sk, int HK, int Tm, int Tn, int W,
-                                      int causal) {
+                                      int causal, int vec) {
   extern __shared__ int32_t flags[];  // any[Tn], all[Tn]
   int32_t* any_f = flags;
   int32_t* all_f = flags + Tn;
@@ -60,21 +110,40 @@ __global__ void classify_index_kernel(const uint32_t* __restrict__ bitmap, int32
   __syncthreads();
   const int64_t i0 = static_cast<int64_t>(mt) * kTile;
   const int rows = static_cast<int>(min64(kTile, Sq - i0));
-  for (int e = threadIdx.x; e < rows * W; e += blockDim.x) {
-    const int r = e / W, w = e % W;
-    const int64_t i = i0 + r;
-    const uint32_t bits = __ldg(bitmap + (bg * Sq + i) * W + w);
-    const int64_t j0 = 32 * static_cast<int64_t>(w);
-    // in-range bits: j in [j0, j0 + 32) with j < Sk; allowed bits: also set and,
-    // when causal, j <= i.  FULL needs every in-range bit allowed.
-    const int64_t n_in = min64(32, Sk - j0);
-    const uint32_t in_range = n_in >= 32 ? 0xFFFFFFFFu : ((1u << n_in) - 1u);
-    const int64_t n_c = causal ? min64(32, max64(0, i + 1 - j0)) : 32;
-    const uint32_t causal_ok = n_c >= 32 ? 0xFFFFFFFFu : ((1u << n_c) - 1u);
-    const uint32_t allowed = bits & in_range & causal_ok;
-    const int nt = w / (kTile / 32);
-    if (allowed) any_f[nt] = 1;
-    if (allowed != in_range) all_f[nt] = 0;
+  constexpr int kWordsPerTile = kTile / 32;
+  if (vec) {
+    // one (row, key tile) per element; rows are W words apart (W % 4 == 0 and a 16-byte
+    // aligned bitmap keep every load aligned)
+    for (int e = threadIdx.x; e < rows * Tn; e += blockDim.x) {
+      const int r = e / Tn, nt = e - (e / Tn) * Tn;
+      const int64_t i = i0 + r;
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(bitmap + (bg * Sq + i) * W) + nt);
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+      bool any = false, all = true;
+#pragma unroll
+      for (int k = 0; k < kWordsPerTile; ++k) {
+        uint32_t in_range;
+        const uint32_t allowed = allowed_bits(
+            wv[k], i, static_cast<int64_t>(nt) * kTile + 32 * k, Sk, causal, in_range);
+        any |= allowed != 0u;
+        all &= allowed == in_range;
+      }
+      if (any) any_f[nt] = 1;
+      if (!all) all_f[nt] = 0;
+    }
+  } else {
+    for (int e = threadIdx.x; e < rows * W; e += blockDim.x) {
+      const int r = e / W, w = e % W;
+      const int64_t i = i0 + r;
+      const uint32_t bits = __ldg(bitmap + (bg * Sq + i) * W + w);
+      // FULL needs every in-range bit allowed
+      uint32_t in_range;
+      const uint32_t allowed = allowed_bits(bits, i, 32 * static_cast<int64_t>(w), Sk, causal,
+                                            in_range);
+      const int nt = w / kWordsPerTile;
+      if (allowed) any_f[nt] = 1;
+      if (allowed != in_range) all_f[nt] = 0;
+    }
   }
   __syncthreads();
   for (int nt = threadIdx.x; nt < Tn; nt += blockDim.x) {
@@ -201,11 +270,13 @@ extern "C" int index_to_block_sparse(const int32_t* idx, int32_t topk, sa_block_
       cudaFuncSetAttribute(scatter_bits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem_bits)) != cudaSuccess)
     return SA_ERR_CUDA;
-  scatter_bits_kernel<<<static_cast<unsigned>(rows), 256, smem_bits, st>>>(
-      idx, out->bitmap, out->Sq, out->Sk, out->HK, topk, static_cast<int>(W), dev_status);
+  const int vec = (topk % 4 == 0) && (reinterpret_cast<uintptr_t>(idx) % 16 == 0);
+  scatter_bits_kernel<<<static_cast<unsigned>(rows), kScatterThreads, smem_bits, st>>>(
+      idx, out->bitmap, out->Sq, out->Sk, out->HK, topk, static_cast<int>(W), vec, dev_status);
   const int64_t BG = static_cast<int64_t>(out->B) * out->HK;
   classify_index_kernel<<<static_cast<unsigned>(BG * Tm), 256, 2 * Tn * sizeof(int32_t), st>>>(
-      out->bitmap, out->idx, out->Sq, out->Sk, out->HK, Tm, Tn, static_cast<int>(W), out->causal);
+      out->bitmap, out->idx, out->Sq, out->Sk, out->HK, Tm, Tn, static_cast<int>(W), out->causal,
+      static_cast<int>(W % 4 == 0 && reinterpret_cast<uintptr_t>(out->bitmap) % 16 == 0));
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   return launch_lists(out, Tm, Tn, st);
 }

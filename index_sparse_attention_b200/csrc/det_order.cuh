@@ -66,9 +66,8 @@ __device__ __forceinline__ bool det_wait_turn(const int32_t* slot, int rank, vol
   const uint64_t limit = ctl->limit_ns;
   while (ld_acquire_gpu(slot) != rank) {
     if (ctl->abort) return false;
-    if (globaltimer_ns() - t0 > limit) {
-      ctl->abort = 1;
-      report_status(status, kStatusTimeout);
+    if (limit < kShortLimitNs || globaltimer_ns() - t0 > limit) {
+      wait_timed_out(ctl, status);
       return false;
     }
     __nanosleep(128);

@@ -97,21 +97,40 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Limits below this make every wait give up at its first test if the phase has not
+// completed (instrumentation: try_wait may suspend in hardware for longer than a short
+// hint, so a sub-microsecond limit would not make ordinary waits run out reliably).
+constexpr uint64_t kShortLimitNs = 1000;
+
+// Records a timeout (once per CTA) and makes every other wait of the CTA give up.
+__device__ __forceinline__ void wait_timed_out(volatile WaitCtl* ctl, int32_t* status) {
+  if (!ctl->abort) {
+    ctl->abort = 1;
+    report_status(status, kStatusTimeout);
+  }
+}
+
 // Waits until the phase of parity `parity` of the barrier has completed.  Gives up
 // (returns false) when ctl->abort becomes non-zero or after ctl->limit_ns; on a timeout
-// it sets ctl->abort and reports SA_ERR_TIMEOUT through `status`.  The hardware suspend
-// hint never exceeds the limit, so a wait gives up within about twice the limit.
+// it sets ctl->abort and reports SA_ERR_TIMEOUT through `status`.  A limit below
+// kShortLimitNs means a single non-blocking test.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile WaitCtl* ctl,
                                           int32_t* status) {
+  // fast path: the phase has completed already (nothing else is read)
+  if (mbar_test(bar, parity)) return true;
   const uint64_t limit = ctl->limit_ns;
+  if (limit < kShortLimitNs) {
+    wait_timed_out(ctl, status);
+    return false;
+  }
   const uint32_t hint = limit < kSuspendHintNs ? static_cast<uint32_t>(limit) : kSuspendHintNs;
+  if (mbar_try_wait(bar, parity, hint)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity, hint)) return true;
     if (ctl->abort) return false;
     if (globaltimer_ns() - t0 > limit) {
-      ctl->abort = 1;
-      report_status(status, kStatusTimeout);
+      wait_timed_out(ctl, status);
       return false;
     }
   }

@@ -3,11 +3,11 @@
 Every mbarrier wait of the attention kernels gives up after a limit (2 s by default),
 sets bit 2 of the device status word, and its CTA drains the copies and tensor-core
 operations it has in flight before it releases its resources and leaves.  These tests
-shorten the limit to a few hundred nanoseconds through the C ABI
-(sparse_attn_set_wait_limit_ns), so that ordinary waits (a TMA load from HBM, the first
-MMA) run out, and check for each kernel family (forward, backward at D=128 and at
-(192,128), the 2-CTA backward at (256,256), and the deterministic backward) that the
-call returns, that the status word carries the timeout bit, and that the next call at
+set a limit below 1 us through the C ABI (sparse_attn_set_wait_limit_ns), which makes a
+wait give up at its first test when its phase has not completed, so that ordinary
+waits (a TMA load just issued, the first MMA) run out.  For each kernel family
+(forward, backward at D=128 and at (192,128), the 2-CTA backward at (256,256), and the
+deterministic backward) they check that the call returns, that the status word carries the timeout bit, and that the next call at
 the default limit matches the oracle: the CUDA context is still usable.  No GPU fault,
 trap or endless wait is involved: the waits end by themselves.
 """

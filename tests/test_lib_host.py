@@ -92,3 +92,9 @@ def test_block_mask_validation(lib):
     assert lib.block_mask_to_block_sparse(ctypes.byref(s), None) == _lib.SA_ERR_UNSUPPORTED
     s.bs, s.Mb, s.Nb = 64, 2, 4  # Mb * bs < Sq
     assert lib.block_mask_to_block_sparse(ctypes.byref(s), None) == _lib.SA_ERR_INVALID
+
+
+def test_instrumentation_setters(lib):
+    """The test-only knob: the wait limit of the bounded pipeline waits."""
+    assert lib.sparse_attn_set_wait_limit_ns(1000) == _lib.SA_OK
+    assert lib.sparse_attn_set_wait_limit_ns(0) == _lib.SA_OK
