@@ -648,6 +648,71 @@ def run_topk(args):
     print(json.dumps(line), flush=True)
 
 
+# -----------------------------------------------------------------------------------
+# Index-workload statistics (CPU): what finer-grained or gathering designs could skip
+# -----------------------------------------------------------------------------------
+def run_index_stats(args):
+    """Counts on the seeded index workload, per KV head, from the indices alone:
+    - active 128 x 128 tiles (the block path's unit) and their block-counted FLOP against
+      the token-level FLOP of the selected (query, key) pairs;
+    - among the 128-query x 32-key sub-blocks of active tiles, the share holding at least
+      one selected pair (a kernel that skipped empty 32-key sub-blocks could save the rest);
+    - per 128-query tile, the union of its rows' key sets against the tile's causal key
+      range (what a kernel gathering that union for the whole tile would still do);
+    - the K/V rows a per-(token, KV head) gather would move per forward, and how many
+      query heads share each gathered row (its reuse)."""
+    w = I.WORKLOADS[args.workload]
+    if w.mode != "index":
+        raise SystemExit("--op index_stats needs an index workload")
+    if args.seq:
+        w = I.scaled(w, Sq=args.seq, Sk=args.seq, name=f"{w.name}@S{args.seq}")
+    t0 = time.perf_counter()
+    idx = I.topk_indices(w)
+    G = w.HQ // w.HK
+    Tm, Tn = -(-w.Sq // 128), -(-w.Sk // 128)
+    sel = tiles = sub_nonempty = sub_total = 0
+    union_keys = range_keys = 0
+    for b in range(w.B):
+        for g in range(w.HK):
+            present = np.zeros((w.Sq, Tn * 128), dtype=bool)
+            rows = np.repeat(np.arange(w.Sq), w.topk)
+            keys = idx[b, :, g, :].reshape(-1)
+            ok = keys >= 0
+            if w.causal:
+                ok &= keys <= rows
+            present[rows[ok], keys[ok]] = True
+            sel += int(present.sum())
+            pad = np.zeros((Tm * 128, Tn * 128), dtype=bool)
+            pad[:w.Sq] = present
+            sub = pad.reshape(Tm, 128, Tn * 4, 32).any(axis=(1, 3))  # [Tm, Tn*4]
+            act = sub.reshape(Tm, Tn, 4).any(axis=2)                   # [Tm, Tn]
+            tiles += int(act.sum())
+            sub_total += int(act.sum()) * 4
+            sub_nonempty += int(sub.reshape(Tm, Tn, 4)[act].sum())
+            union = pad.reshape(Tm, 128, Tn * 128).any(axis=1)        # [Tm, keys]
+            union_keys += int(union.sum())
+            for mt in range(Tm):
+                hi = min((mt + 1) * 128, w.Sk) if w.causal else w.Sk
+                range_keys += hi
+    flop_block = tiles * G * 2 * 128 * 128 * (w.Dqk + w.Dv)
+    flop_token = sel * G * 2 * (w.Dqk + w.Dv)
+    gather_bytes = sel * 2 * (w.Dqk + w.Dv)  # one K and one V row per selected pair
+    line = {
+        "op": "index_stats", "workload": w.name, "seconds": time.perf_counter() - t0,
+        "selected_pairs_per_kv_head": sel / (w.B * w.HK),
+        "active_tiles": tiles, "forward_flop_block_counted": flop_block,
+        "forward_flop_token_level": flop_token,
+        "block_over_token": flop_block / max(1, flop_token),
+        "nonempty_32key_subblocks_of_active_tiles": sub_nonempty / max(1, sub_total),
+        "tile_union_keys_over_causal_range": union_keys / max(1, range_keys),
+        "token_gather_forward_bytes": gather_bytes,
+        "token_gather_row_reuse_query_heads": G,
+        "block_path_forward_bytes_per_tile_visit": 128 * 2 * (w.Dqk + w.Dv),
+        "block_path_row_reuse_query_heads": 128 * G,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -663,14 +728,18 @@ def main():
                     help="override Sq = Sk (smaller profiling captures of the same kernels)")
     ap.add_argument("--deterministic", action="store_true",
                     help="use the deterministic backward (fixed-order dQ accumulation)")
-    ap.add_argument("--op", default="attention", choices=["attention", "topk"],
-                    help="topk: time the top-k selector alone on one packed sequence")
+    ap.add_argument("--op", default="attention", choices=["attention", "topk", "index_stats"],
+                    help="topk: time the top-k selector alone on one packed sequence; "
+                         "index_stats: counts on an index workload (CPU only)")
     ap.add_argument("--pack", type=int, default=16384, help="--op topk: packed sequence length")
     ap.add_argument("--k", type=int, default=2048, help="--op topk: k")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.op == "topk":
         run_topk(args)
+        return
+    if args.op == "index_stats":
+        run_index_stats(args)
         return
     if args.impl == "reference":
         run_reference(args)

@@ -243,7 +243,6 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(BAR(kBDrainB), 1);
     mbar_init(BAR(kBVT), 256);
     abort_flag->abort = 0;
-    abort_flag->limit_ns = a.wait_limit_ns;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -297,9 +296,9 @@ __global__ void __launch_bounds__(448, 1)
         m0 = __shfl_sync(0xFFFFFFFFu, m0, 0);  // warp-uniform TMA coordinate
         const int st = it % C::kStages, u = it / C::kStages;
         const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
-        if (!warp_wait(BAR(kBQE + st), (u & 1) ^ 1, abort_flag, a.status)) break;
+        if (!warp_wait(BAR(kBQE + st), (u & 1) ^ 1, abort_flag, a.status, a.wait_limit_ns)) break;
         // (192,128): V occupies the last stage until it has been copied into TMEM
-        if (C::kVT && it == C::kStages - 1 && !warp_wait(BAR(kBVT), 0, abort_flag, a.status))
+        if (C::kVT && it == C::kStages - 1 && !warp_wait(BAR(kBVT), 0, abort_flag, a.status, a.wait_limit_ns))
           break;
         if (elect_one()) {
           mbar_arrive_expect_tx(BAR(kBQF + st), C::kQBytes + C::kOBytes);
@@ -351,14 +350,14 @@ __global__ void __launch_bounds__(448, 1)
       // start-address field (no carry: shared addresses stay below 2^18)
       const uint64_t kd = sw128_desc(kbase, 16, 1024), vd = sw128_desc(vbase, 16, 1024);
       const uint64_t kwd = sw128_desc(kbase + (qw0 / 64) * C::kKPanel, C::kKPanel, 1024);
-      bool ok = warp_wait(BAR(kBKV), 0, abort_flag, a.status);
-      if (C::kVT) ok = ok && warp_wait(BAR(kBVT), 0, abort_flag, a.status);
+      bool ok = warp_wait(BAR(kBKV), 0, abort_flag, a.status, a.wait_limit_ns);
+      if (C::kVT) ok = ok && warp_wait(BAR(kBVT), 0, abort_flag, a.status, a.wait_limit_ns);
       // S^T(j) and dP^T(j) into TMEM buffer j & 1
       auto issue_sdp = [&](int j) -> bool {
         const int st = j % C::kStages, u = j / C::kStages, bj = j & 1;
-        if (!warp_wait(BAR(kBQF + st), u & 1, abort_flag, a.status)) return false;
+        if (!warp_wait(BAR(kBQF + st), u & 1, abort_flag, a.status, a.wait_limit_ns)) return false;
         // the dQ^T of step j-2 lives in this buffer until it has been drained
-        if (j >= 2 && !warp_wait(BAR(kBDQE + bj), ((j - 2) >> 1) & 1, abort_flag, a.status))
+        if (j >= 2 && !warp_wait(BAR(kBDQE + bj), ((j - 2) >> 1) & 1, abort_flag, a.status, a.wait_limit_ns))
           return false;
         tc_fence_after();
         const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
@@ -394,7 +393,7 @@ __global__ void __launch_bounds__(448, 1)
         const int st = it % C::kStages, bi = it & 1;
         // the next S^T / dP^T overlap this step's elementwise work
         if (it + 1 < n_iter && !issue_sdp(it + 1)) break;
-        if (!warp_wait(BAR(kBPF + bi), (it >> 1) & 1, abort_flag, a.status)) break;
+        if (!warp_wait(BAR(kBPF + bi), (it >> 1) & 1, abort_flag, a.status, a.wait_limit_ns)) break;
         tc_fence_after();
         const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
         const uint64_t qmn = sw128_desc(qs + (kc0 / 64) * C::kQPanel, C::kQPanel, 1024);
@@ -437,7 +436,7 @@ __global__ void __launch_bounds__(448, 1)
     if (C::kVT && n_iter > 0) {
       // V row r into TMEM (row r in lane r, head dims 2e, 2e+1 in column e): this half of
       // the warps copies the 64-column panel hc from the swizzled smem tile
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(BAR(kBKV), 0, abort_flag, a.status));
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(BAR(kBKV), 0, abort_flag, a.status, a.wait_limit_ns));
       if (ok) {
         const uint8_t* prow = smem + C::kVOff + hc * C::kKPanel + r * 128;
         uint32_t w[32];
@@ -462,11 +461,11 @@ __global__ void __launch_bounds__(448, 1)
       bool partial;
       decode(it, h, m0, partial);
       const int st = it % C::kStages, u = it / C::kStages, bi = it & 1;
-      bool w_ok = mbar_wait(BAR(kBLF + st), u & 1, abort_flag, a.status);
-      w_ok = w_ok && mbar_wait(BAR(kBSF + bi), (it >> 1) & 1, abort_flag, a.status);
+      bool w_ok = mbar_wait(BAR(kBLF + st), u & 1, abort_flag, a.status, a.wait_limit_ns);
+      w_ok = w_ok && mbar_wait(BAR(kBSF + bi), (it >> 1) & 1, abort_flag, a.status, a.wait_limit_ns);
       // the dS^T buffer is free once dQ^T of step it-2 has read it
       if (it >= 2)
-        w_ok = w_ok && mbar_wait(BAR(kBDQF + bi), ((it - 2) >> 1) & 1, abort_flag, a.status);
+        w_ok = w_ok && mbar_wait(BAR(kBDQF + bi), ((it - 2) >> 1) & 1, abort_flag, a.status, a.wait_limit_ns);
       if (!__all_sync(0xFFFFFFFFu, w_ok)) {
         ok = false;
         break;
@@ -557,7 +556,7 @@ __global__ void __launch_bounds__(448, 1)
     // ----------------------------------------------------------- dK / dV epilogue
     bool have = n_iter > 0 && ok;
     if (have) {
-      const bool w_ok = mbar_wait(BAR(kBFin), 0, abort_flag, a.status);
+      const bool w_ok = mbar_wait(BAR(kBFin), 0, abort_flag, a.status, a.wait_limit_ns);
       have = __all_sync(0xFFFFFFFFu, w_ok);
       tc_fence_after();
     }
@@ -628,7 +627,7 @@ __global__ void __launch_bounds__(448, 1)
       decode(it, h, m0, partial);
       const int bi = it & 1;
       // the four drain warps leave together (they share named barrier 1 below)
-      const bool w_ok = mbar_wait(BAR(kBDQF + bi), (it >> 1) & 1, abort_flag, a.status);
+      const bool w_ok = mbar_wait(BAR(kBDQF + bi), (it >> 1) & 1, abort_flag, a.status, a.wait_limit_ns);
       if (!named_bar_and(1, 128, w_ok)) {
         ok = false;
         break;
@@ -648,7 +647,7 @@ __global__ void __launch_bounds__(448, 1)
       bool turn_ok = true;
       if (DET && qhalf == 0 && dtid == 0)
         turn_ok = det_wait_turn(det_slot(a, b, h, mt, split), key_tile_rank(a, bg, mt, nt), abort_flag,
-                                a.status);
+                                a.status, a.wait_limit_ns);
       if (DET && !named_bar_and(1, 128, turn_ok)) {
         ok = false;
         break;

@@ -215,7 +215,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     mbar_init(BAR(kBDrain), 1);
     abort_flag->abort = 0;
     abort_flag->peer_abort = 0;
-    abort_flag->limit_ns = a.wait_limit_ns;
     // the first exchange tiles may arrive from the peer at any time
     for (int s = 0; s < (rank == 0 ? kNX : kNPI) && s < n_iter; ++s)
       mbar_arrive_expect_tx(BAR(kBXF + s), kTile);
@@ -300,9 +299,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         decode(it, h, m0, partial);
         m0 = __shfl_sync(0xFFFFFFFFu, m0, 0);  // warp-uniform TMA coordinate
         const int s = it % ns, u = it / ns;
-        if (!warp_wait(BAR(kBQE + s), (u & 1) ^ 1, abort_flag, a.status)) break;
+        if (!warp_wait(BAR(kBQE + s), (u & 1) ^ 1, abort_flag, a.status, a.wait_limit_ns)) break;
         // rank 1: V occupies stages 1 and 2 until it has been copied into TMEM
-        if (rank == 1 && (it == 1 || it == 2) && !warp_wait(BAR(kBVT), 0, abort_flag, a.status))
+        if (rank == 1 && (it == 1 || it == 2) && !warp_wait(BAR(kBVT), 0, abort_flag, a.status, a.wait_limit_ns))
           break;
         const uint32_t qs = sbase + off_stage + s * kStageBytes;
         if (elect_one()) {
@@ -314,7 +313,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         // rank 1 frees a stage when dV is done, which can precede the elementwise warps'
         // read of the step's Delta: wait for them before overwriting it
         if (rank == 1 && it >= ns &&
-            !warp_wait(BAR(kBEW + s), ((it - ns) / ns) & 1, abort_flag, a.status))
+            !warp_wait(BAR(kBEW + s), ((it - ns) / ns) & 1, abort_flag, a.status, a.wait_limit_ns))
           break;
         float* ls = lbuf + s * BM;
         ls[lane] = rows[0];
@@ -336,8 +335,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       auto ready = [&](int k, int parity) {
         return __shfl_sync(0xFFFFFFFFu, mbar_test(BAR(k), parity) ? 1 : 0, 0) != 0;
       };
-      bool ok = warp_wait(BAR(kBKV), 0, abort_flag, a.status);
-      ok = ok && warp_wait(BAR(kBVT), 0, abort_flag, a.status);
+      bool ok = warp_wait(BAR(kBKV), 0, abort_flag, a.status, a.wait_limit_ns);
+      ok = ok && warp_wait(BAR(kBVT), 0, abort_flag, a.status, a.wait_limit_ns);
       int js = 0;  // next S^T (rank 0) / dP^T (rank 1)
       int jv = 0;  // rank 1: next dV
       int jk = 0;  // next dQ^T
@@ -458,7 +457,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
           t_last = globaltimer_ns();
         } else {
           if (__shfl_sync(0xFFFFFFFFu, abort_flag->abort, 0) != 0) break;
-          if (globaltimer_ns() - t_last > abort_flag->limit_ns) {
+          if (globaltimer_ns() - t_last > a.wait_limit_ns) {
             if (lane == 0) wait_timed_out(abort_flag, a.status);
             __syncwarp();
             break;
@@ -483,7 +482,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       // K (rank 0) / V (rank 1) row r into TMEM (row r in lane r, head dims 2e, 2e+1 in
       // column e): this half of the warps copies head dims [128 hc, 128 hc + 128) from
       // the swizzled panels
-      const bool v_ok = __all_sync(0xFFFFFFFFu, mbar_wait(BAR(kBKV), 0, abort_flag, a.status));
+      const bool v_ok = __all_sync(0xFFFFFFFFu, mbar_wait(BAR(kBKV), 0, abort_flag, a.status, a.wait_limit_ns));
       if (v_ok) {
 #pragma unroll
         for (int pl = 0; pl < 2; ++pl) {
@@ -517,15 +516,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       decode(it, h, m0, partial);
       const int s = it % ns, ph = (it / ns) & 1;
       const int xb = it % kNX, phx = (it / kNX) & 1;
-      bool w_ok = mbar_wait(BAR(kBLF + s), ph, abort_flag, a.status);
-      w_ok = w_ok && mbar_wait(BAR(kBSF + s), ph, abort_flag, a.status);
+      bool w_ok = mbar_wait(BAR(kBLF + s), ph, abort_flag, a.status, a.wait_limit_ns);
+      w_ok = w_ok && mbar_wait(BAR(kBSF + s), ph, abort_flag, a.status, a.wait_limit_ns);
       if (rank == 0) {
         // own tile xb: the dQ drain of step it-4 is done with it
         if (it >= kNX)
-          w_ok = w_ok && mbar_wait(BAR(kBXT + xb), phx ^ 1, abort_flag, a.status);
+          w_ok = w_ok && mbar_wait(BAR(kBXT + xb), phx ^ 1, abort_flag, a.status, a.wait_limit_ns);
       } else {
         w_ok = w_ok && mbar_wait(BAR(kBXF + it % kNPI), (it / kNPI) & 1, abort_flag,
-                                 a.status);  // P^T arrived
+                                 a.status, a.wait_limit_ns);  // P^T arrived
       }
       if (!__all_sync(0xFFFFFFFFu, w_ok)) {
         ok = false;
@@ -603,9 +602,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         // have written them and that tile is free (rank 1 is done with step it-3 there):
         // four copies in flight instead of one
         if (hc == 0 && lane == 0 &&
-            mbar_wait(BAR(kBQH + (it & 1) * 4 + quarter), (it >> 1) & 1, abort_flag, a.status) &&
+            mbar_wait(BAR(kBQH + (it & 1) * 4 + quarter), (it >> 1) & 1, abort_flag, a.status, a.wait_limit_ns) &&
             (it < kNPI ||
-             mbar_wait(BAR(kBXE + it % kNPI), ((it / kNPI) & 1) ^ 1, abort_flag, a.status))) {
+             mbar_wait(BAR(kBXE + it % kNPI), ((it / kNPI) & 1) ^ 1, abort_flag, a.status, a.wait_limit_ns))) {
           bulk_copy_to_cluster(
               mapa_shared(sbase + kOffPI1 + (it % kNPI) * kTile + quarter * (kTile / 4), peer),
               sbase + kOffX0 + xb * kTile + quarter * (kTile / 4), kTile / 4,
@@ -644,7 +643,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         }
         // dS^T tile it % 3: dQ^T of step it-3 has read it and its copy has landed in rank 0
         const bool df_ok =
-            it < kNDO || mbar_wait(BAR(kBDF + it % kNDO), ((it / kNDO) & 1) ^ 1, abort_flag, a.status);
+            it < kNDO || mbar_wait(BAR(kBDF + it % kNDO), ((it / kNDO) & 1) ^ 1, abort_flag, a.status, a.wait_limit_ns);
         if (!__all_sync(0xFFFFFFFFu, df_ok)) {
           ok = false;
           break;
@@ -662,7 +661,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         // each quarter's 32 rows of dS^T go to rank 0's tile xb as soon as they are in
         // (that tile held P^T of this step, which rank 1 has already received)
         if (hc == 0 && lane == 0 &&
-            mbar_wait(BAR(kBQH + (it & 1) * 4 + quarter), (it >> 1) & 1, abort_flag, a.status)) {
+            mbar_wait(BAR(kBQH + (it & 1) * 4 + quarter), (it >> 1) & 1, abort_flag, a.status, a.wait_limit_ns)) {
           bulk_copy_to_cluster(mapa_shared(sbase + kOffX0 + xb * kTile + quarter * (kTile / 4), peer),
                                sbase + kOffDO1 + (it % kNDO) * kTile + quarter * (kTile / 4),
                                kTile / 4, mapa_shared(BAR(kBXF + xb), peer));
@@ -672,7 +671,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     // ----------------------------------------------------------- dK / dV epilogue
     bool have = n_iter > 0 && ok;
     if (have) {
-      const bool w_ok = mbar_wait(BAR(kBFin), 0, abort_flag, a.status);
+      const bool w_ok = mbar_wait(BAR(kBFin), 0, abort_flag, a.status, a.wait_limit_ns);
       have = __all_sync(0xFFFFFFFFu, w_ok);
       tc_fence_after();
     }
@@ -732,7 +731,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       const int qb = rank == 0 ? 0 : (it & 1);
       // the four drain warps leave together (they share named barrier 1 below)
       const bool w_ok = mbar_wait(BAR(kBDQF + qb), rank == 0 ? (it & 1) : ((it >> 1) & 1),
-                                  abort_flag, a.status);
+                                  abort_flag, a.status, a.wait_limit_ns);
       if (!named_bar_and(1, 128, w_ok)) {
         ok = false;
         break;
@@ -755,7 +754,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       bool turn_ok = true;
       if (DET && qhalf == 0 && dtid == 0)
         turn_ok = det_wait_turn(det_slot(a, b, h, mt, static_cast<int>(rank)),
-                                key_tile_rank(a, bg, mt, nt), abort_flag, a.status);
+                                key_tile_rank(a, bg, mt, nt), abort_flag, a.status, a.wait_limit_ns);
       if (DET && !named_bar_and(1, 128, turn_ok)) {
         ok = false;
         break;

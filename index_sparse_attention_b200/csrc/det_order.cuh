@@ -61,9 +61,8 @@ __device__ __forceinline__ int32_t* det_slot(const AttnArgs& a, int b, int h, in
 // Waits until the counter equals `rank` (bounded); then orders the caller's following
 // TMA reduce-adds after the acquire.  False on a timeout or an abort.
 __device__ __forceinline__ bool det_wait_turn(const int32_t* slot, int rank, volatile WaitCtl* ctl,
-                                              int32_t* status) {
+                                              int32_t* status, uint64_t limit) {
   const uint64_t t0 = globaltimer_ns();
-  const uint64_t limit = ctl->limit_ns;
   while (ld_acquire_gpu(slot) != rank) {
     if (ctl->abort) return false;
     if (limit < kShortLimitNs || globaltimer_ns() - t0 > limit) {

@@ -98,7 +98,6 @@ __global__ void __launch_bounds__(224, 1)
     mbar_init(BAR(kBDrain), 1);
     mbar_init(BAR(kBOFin), 1);
     abort_flag->abort = 0;
-    abort_flag->limit_ns = a.wait_limit_ns;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -129,7 +128,7 @@ __global__ void __launch_bounds__(224, 1)
       for (int it = 0; it < n_iter; ++it) {
         const int nt = __shfl_sync(0xFFFFFFFFu, __ldg(list + it), 0);
         const int ks = it % C::kKStages, ku = it / C::kKStages;
-        if (!warp_wait(BAR(kBKE + ks), (ku & 1) ^ 1, abort_flag, a.status)) break;
+        if (!warp_wait(BAR(kBKE + ks), (ku & 1) ^ 1, abort_flag, a.status, a.wait_limit_ns)) break;
         if (elect_one()) {
           mbar_arrive_expect_tx(BAR(kBKF + ks), C::kKBytes);
           for (int c = 0; c < DQK / 64; ++c)
@@ -146,7 +145,7 @@ __global__ void __launch_bounds__(224, 1)
       for (int it = 0; it < n_iter; ++it) {
         const int nt = __shfl_sync(0xFFFFFFFFu, __ldg(list + it), 0);
         const int vs = it % C::kVStages, vu = it / C::kVStages;
-        if (!warp_wait(BAR(kBVE + vs), (vu & 1) ^ 1, abort_flag, a.status)) break;
+        if (!warp_wait(BAR(kBVE + vs), (vu & 1) ^ 1, abort_flag, a.status, a.wait_limit_ns)) break;
         if (elect_one()) {
           mbar_arrive_expect_tx(BAR(kBVF + vs), C::kVBytes);
           for (int c = 0; c < DV / 64; ++c)
@@ -165,10 +164,10 @@ __global__ void __launch_bounds__(224, 1)
       constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(128, DV, 0, 1);
       const uint64_t qdesc = sw128_desc(sbase + C::kQOff, 16, 1024);
-      bool ok = warp_wait(BAR(kBQ), 0, abort_flag, a.status);
+      bool ok = warp_wait(BAR(kBQ), 0, abort_flag, a.status, a.wait_limit_ns);
       auto issue_s = [&](int it) -> bool {
         const int ks = it % C::kKStages, ku = it / C::kKStages;
-        if (!warp_wait(BAR(kBKF + ks), ku & 1, abort_flag, a.status)) return false;
+        if (!warp_wait(BAR(kBKF + ks), ku & 1, abort_flag, a.status, a.wait_limit_ns)) return false;
         tc_fence_after();
         const uint64_t kdesc = sw128_desc(sbase + C::kKOff + ks * C::kKBytes, 16, 1024);
         const uint32_t d = tmem + static_cast<uint32_t>((it & 1) * 128);
@@ -188,8 +187,8 @@ __global__ void __launch_bounds__(224, 1)
       for (int it = 0; ok && it < n_iter; ++it) {
         if (it + 1 < n_iter && !issue_s(it + 1)) break;
         const int vs = it % C::kVStages, vu = it / C::kVStages;
-        if (!warp_wait(BAR(kBPF + (it & 1)), (it >> 1) & 1, abort_flag, a.status)) break;
-        if (!warp_wait(BAR(kBVF + vs), vu & 1, abort_flag, a.status)) break;
+        if (!warp_wait(BAR(kBPF + (it & 1)), (it >> 1) & 1, abort_flag, a.status, a.wait_limit_ns)) break;
+        if (!warp_wait(BAR(kBVF + vs), vu & 1, abort_flag, a.status, a.wait_limit_ns)) break;
         tc_fence_after();
         const uint64_t vdesc = sw128_desc(sbase + C::kVOff + vs * C::kVBytes, C::kPanel, 1024);
         const uint32_t pa = tmem + static_cast<uint32_t>((it & 1) * 128);
@@ -216,7 +215,7 @@ __global__ void __launch_bounds__(224, 1)
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
       const int sb = it & 1;
-      const bool w_ok = mbar_wait(BAR(kBSF + sb), (it >> 1) & 1, abort_flag, a.status);
+      const bool w_ok = mbar_wait(BAR(kBSF + sb), (it >> 1) & 1, abort_flag, a.status, a.wait_limit_ns);
       if (!__all_sync(0xFFFFFFFFu, w_ok)) {
         ok = false;
         break;
@@ -277,7 +276,7 @@ __global__ void __launch_bounds__(224, 1)
         const float alpha = need ? ex2(m_run - m_tile) : 1.f;  // 0 when m_run = -inf
         if (it > 0) {
           // O holds P V up to tile it-1: rescale it in TMEM once that MMA is done.
-          bool w_ok = mbar_wait(BAR(kBOD), (it - 1) & 1, abort_flag, a.status);
+          bool w_ok = mbar_wait(BAR(kBOD), (it - 1) & 1, abort_flag, a.status, a.wait_limit_ns);
           if (!__all_sync(0xFFFFFFFFu, w_ok)) {
             ok = false;
             break;
@@ -321,7 +320,7 @@ __global__ void __launch_bounds__(224, 1)
     }
     // ---------------------------------------------------------------- epilogue
     if (n_iter > 0 && ok) {
-      const bool w_ok = mbar_wait(BAR(kBOFin), 0, abort_flag, a.status);
+      const bool w_ok = mbar_wait(BAR(kBOFin), 0, abort_flag, a.status, a.wait_limit_ns);
       ok = __all_sync(0xFFFFFFFFu, w_ok);
       tc_fence_after();
     }

@@ -23,11 +23,10 @@ constexpr int kTile = 128;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // Per-CTA wait control, kept in shared memory: the abort flag every bounded wait of
-// the CTA watches, and this launch's wait limit.
+// the CTA watches.
 struct WaitCtl {
   int abort;
   int peer_abort;  // 2-CTA kernels: the other CTA's final abort flag, stored there by it
-  uint64_t limit_ns;
 };
 
 // Device status bits (OR-ed into the caller's int32 status word).
@@ -110,21 +109,16 @@ __device__ __forceinline__ void wait_timed_out(volatile WaitCtl* ctl, int32_t* s
   }
 }
 
-// Waits until the phase of parity `parity` of the barrier has completed.  Gives up
-// (returns false) when ctl->abort becomes non-zero or after ctl->limit_ns; on a timeout
-// it sets ctl->abort and reports SA_ERR_TIMEOUT through `status`.  A limit below
-// kShortLimitNs means a single non-blocking test.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile WaitCtl* ctl,
-                                          int32_t* status) {
-  // fast path: the phase has completed already (nothing else is read)
-  if (mbar_test(bar, parity)) return true;
-  const uint64_t limit = ctl->limit_ns;
+// The part of mbar_wait past its first try_wait (kept out of line: the kernels wait in
+// dozens of places and the instruction cache is a shared resource of the SM).
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile WaitCtl* ctl,
+                                            int32_t* status, uint64_t limit) {
   if (limit < kShortLimitNs) {
+    if (mbar_test(bar, parity)) return true;
     wait_timed_out(ctl, status);
     return false;
   }
   const uint32_t hint = limit < kSuspendHintNs ? static_cast<uint32_t>(limit) : kSuspendHintNs;
-  if (mbar_try_wait(bar, parity, hint)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity, hint)) return true;
@@ -134,6 +128,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       return false;
     }
   }
+}
+
+// Waits until the phase of parity `parity` of the barrier has completed.  Gives up
+// (returns false) when ctl->abort becomes non-zero or after `limit` ns (the launch's
+// AttnArgs::wait_limit_ns, read from the kernel parameters: no memory access on the
+// fast path); on a timeout it sets ctl->abort and reports SA_ERR_TIMEOUT through
+// `status`.  A limit below kShortLimitNs means a single non-blocking test.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile WaitCtl* ctl,
+                                          int32_t* status, uint64_t limit) {
+  if (limit >= kShortLimitNs && mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, ctl, status, limit);
 }
 
 // Time-limited wait used only on the abort path (drains copies and MMAs in flight
@@ -148,8 +153,8 @@ __device__ __forceinline__ bool mbar_wait_limited(uint32_t bar, uint32_t parity)
 
 // Warp-collective form: every lane waits; the result is the same on every lane.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile WaitCtl* ctl,
-                                          int32_t* status) {
-  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, ctl, status));
+                                          int32_t* status, uint64_t limit) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, ctl, status, limit));
 }
 
 // Picks one active lane of a converged warp (true on that lane only).

@@ -57,3 +57,18 @@ def test_converter_bytes_index_workload():
     bitmap = 4 * 16384 * 512 * 4        # 128 MiB, written and read back once
     lists = 4 * 4 * (128 * 130 + 128 * 130)
     assert bench.converter_bytes(w) == idx + 2 * bitmap + 2 * lists
+
+
+def test_index_stats_leg_on_a_small_index_workload(capsys):
+    """bench.py --op index_stats: counts on the seeded indices (no GPU)."""
+    import types
+    args = types.SimpleNamespace(workload="indexsparse_gqa_q16384_hq32_hk4_d192_128_top2048",
+                                 seq=1024)
+    bench.run_index_stats(args)
+    d = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert d["block_over_token"] >= 1.0
+    assert 0.0 < d["nonempty_32key_subblocks_of_active_tiles"] <= 1.0
+    assert 0.0 < d["tile_union_keys_over_causal_range"] <= 1.0
+    # causal, 1024 tokens, top-2048: every (q, k <= q) pair is selected
+    assert d["selected_pairs_per_kv_head"] == 1024 * 1025 // 2
+    assert d["token_gather_forward_bytes"] == 4 * 1024 * 1025 // 2 * 2 * (192 + 128)
