@@ -10,19 +10,22 @@
 //   warp 0     TMA producer: Q once, then the K tiles of the ACTIVE key tiles only
 //              (the forward list), 128-byte swizzled, double-buffered when shared
 //              memory allows;
-//   warp 6     TMA producer of the V tiles, so that a K load (which S waits for)
+//   warp 10    TMA producer of the V tiles, so that a K load (which S waits for)
 //              never queues behind a V load that waits for the previous P V.
 //   warp 1     allocates 512 TMEM columns and issues the tcgen05 MMAs (one elected
 //              lane per batch): S = Q K^T into one of two TMEM S buffers (so the next S is
 //              computed while the softmax works on the current one), and
 //              O += P V with P read from TMEM (A operand in tensor memory).
-//   warps 2-5  softmax, one query row per thread (thread = TMEM lane): tcgen05.ld the
-//              S row, apply the element mask on partial tiles (range, causal, 64-block
-//              mask or index bitmap), update the running max lazily (O is rescaled in
-//              TMEM only when the max grows by more than 2^8), exponentiate with
-//              ex2, write bf16 P back over the S buffer, and at the end normalise O
-//              into the idle Q buffer (the output map's swizzled box layout, sent by
-//              TMA tensor stores) and write LSE (fp32, natural log).
+//   warps 2-9  softmax, two warps per TMEM lane quarter: a thread holds one query row
+//              (thread = TMEM lane) and one half of its 128 columns.  It tcgen05.ld's
+//              its half of the S row, applies the element mask on partial tiles (range,
+//              causal, 64-block mask or index bitmap), takes the row max with its
+//              partner (shared memory), updates the running max lazily (O is rescaled
+//              in TMEM only when the max grows by more than 2^8), exponentiates with
+//              ex2 and writes bf16 P back over the S buffer.  At the end the pair adds
+//              its row-sum halves, normalises O into the idle Q buffer (the output map's
+//              swizzled box layout, sent by TMA tensor stores) and writes LSE (fp32,
+//              natural log).  One softmax warp per SM sub-partition was issue bound.
 // TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+Dv).
 // Every mbarrier wait is bounded; a timeout sets SA_ERR_TIMEOUT in the status word and
 // the CTA leaves after releasing its tensor memory.
@@ -31,7 +34,7 @@
 
 namespace sa {
 
-template <int DQK, int DV>
+template <int DQK, int DV, bool PAIRED>
 struct FwdCfg {
   static constexpr int kPanel = 128 * 128;  // one 64-column x 128-row swizzled panel
   static constexpr int kQBytes = 128 * DQK * 2;
@@ -43,25 +46,37 @@ struct FwdCfg {
   static constexpr int kKOff = kQOff + kQBytes;
   static constexpr int kVOff = kKOff + kKStages * kKBytes;
   static constexpr int kBarOff = kVOff + kVStages * kVBytes;
-  static constexpr int kSmem = kBarOff + 256 + 1024;  // barriers + alignment slack
-  static constexpr int kThreads = 224;
+  // softmax exchange: row max [2 tile parities][2 column halves][128 rows] and row sum
+  // [2 halves][128 rows], fp32
+  static constexpr int kXOff = kBarOff + 256;
+  static constexpr int kSmem = kXOff + 3 * 1024 + 1024;  // + alignment slack
+  // softmax warps per TMEM lane quarter (PAIRED: two, each with half of every row)
+  static constexpr int kHalves = PAIRED ? 2 : 1;
+  static constexpr int kThreads = PAIRED ? 352 : 224;
+  static constexpr int kVWarp = PAIRED ? 10 : 6;  // V producer
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kOCol = 256;
+  // Dqk <= 192: Q is held in TMEM after O (bf16 pairs) and S = Q K^T reads it from there,
+  // so that only K is read from shared memory (an operand pair from shared memory costs
+  // 8 KB per 64-cycle k-step, the whole port, before the TMA writes of K and V)
+  static constexpr bool kQT = DQK <= 192;
+  static constexpr uint32_t kColQ = kOCol + DV;
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
   static_assert(kOCol + DV <= kTmemCols, "tensor memory budget");
+  static_assert(!kQT || kColQ + DQK / 2 <= kTmemCols, "tensor memory budget (Q)");
 };
 
 // barrier slots
 enum : int { kBQ = 0, kBKF = 1, kBKE = 3, kBVF = 5, kBVE = 7, kBSF = 9, kBPF = 11, kBOD = 13,
-             kBDrain = 14, kBOFin = 15, kNumBars = 16 };
+             kBDrain = 14, kBOFin = 15, kBQT = 16, kNumBars = 17 };
 
-template <int DQK, int DV>
-__global__ void __launch_bounds__(224, 1)
+template <int DQK, int DV, bool PAIRED>
+__global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
     sparse_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_o, const AttnArgs a) {
-  using C = FwdCfg<DQK, DV>;
+  using C = FwdCfg<DQK, DV, PAIRED>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -92,11 +107,12 @@ __global__ void __launch_bounds__(224, 1)
       mbar_init(BAR(kBVF + s), 1);
       mbar_init(BAR(kBVE + s), 1);
       mbar_init(BAR(kBSF + s), 1);
-      mbar_init(BAR(kBPF + s), 128);
+      mbar_init(BAR(kBPF + s), 128 * C::kHalves);
     }
     mbar_init(BAR(kBOD), 1);
     mbar_init(BAR(kBDrain), 1);
     mbar_init(BAR(kBOFin), 1);
+    mbar_init(BAR(kBQT), 128 * C::kHalves);
     abort_flag->abort = 0;
     fence_mbar_init();
   }
@@ -139,7 +155,7 @@ __global__ void __launch_bounds__(224, 1)
         issued_k = it + 1;
       }
     }
-  } else if (warp == 6) {
+  } else if (warp == C::kVWarp) {
     // ------------------------------------------------------------------ V producer
     if (n_iter > 0) {
       for (int it = 0; it < n_iter; ++it) {
@@ -164,7 +180,8 @@ __global__ void __launch_bounds__(224, 1)
       constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(128, DV, 0, 1);
       const uint64_t qdesc = sw128_desc(sbase + C::kQOff, 16, 1024);
-      bool ok = warp_wait(BAR(kBQ), 0, abort_flag, a.status, a.wait_limit_ns);
+      // Q in TMEM (kQT): the softmax warps have copied it there
+      bool ok = warp_wait(BAR(C::kQT ? kBQT : kBQ), 0, abort_flag, a.status, a.wait_limit_ns);
       auto issue_s = [&](int it) -> bool {
         const int ks = it % C::kKStages, ku = it / C::kKStages;
         if (!warp_wait(BAR(kBKF + ks), ku & 1, abort_flag, a.status, a.wait_limit_ns)) return false;
@@ -175,7 +192,10 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
           for (int kk = 0; kk < DQK / 16; ++kk) {
             const uint32_t off = ((kk >> 2) * C::kPanel + (kk & 3) * 32) >> 4;
-            umma_ss(d, qdesc + off, kdesc + off, idesc_qk, kk > 0 ? 1u : 0u);
+            if constexpr (C::kQT)  // A = Q from TMEM: 16 head dims = 8 columns per k-step
+              umma_ts(d, tmem + C::kColQ + kk * 8, kdesc + off, idesc_qk, kk > 0 ? 1u : 0u);
+            else
+              umma_ss(d, qdesc + off, kdesc + off, idesc_qk, kk > 0 ? 1u : 0u);
           }
           umma_commit(BAR(kBSF + (it & 1)));
           umma_commit(BAR(kBKE + ks));
@@ -206,39 +226,80 @@ __global__ void __launch_bounds__(224, 1)
     }
   } else {
     // ------------------------------------------------------------------ softmax
+    // kHalves warps per TMEM lane quarter.  A thread holds one query row (thread = TMEM
+    // lane) and 128 / kHalves of its columns.  PAIRED (index mode, whose partial-tile
+    // masks make one warp per SM sub-partition issue bound): warp pair p (warps 2+p and
+    // 6+p) splits every row's columns in halves (hc) and exchanges its row maxima per
+    // tile (shared memory, double-buffered by tile parity, behind the pair's named
+    // barrier) and its row sums at the end.  Every wait result is AND-ed over the pair
+    // before either warp acts on it, so the two warps always take the same branch and
+    // never leave one another waiting at the pair's barrier.
+    constexpr int kH = C::kHalves;
+    constexpr int kCols = 128 / kH;                  // S columns per thread
+    constexpr int kOCols = DV / kH;                  // O columns rescaled / stored per thread
     const int quarter = warp & 3;
+    const int hc = kH == 2 ? (warp - 2) >> 2 : 0;   // column part of this warp
+    const int pair_bar = 1 + ((warp - 2) & 3);       // named barrier of a pair (64 threads)
+    auto pair_all = [&](bool v) {                    // v: already uniform over the warp
+      if constexpr (kH == 2) return named_bar_and(pair_bar, 64, v);
+      return v;
+    };
     const int r = quarter * 32 + lane;
     const int64_t i = static_cast<int64_t>(mt) * 128 + r;
     const bool row_ok = i < a.Sq;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    float m_run = -INFINITY, l_run = 0.f;
+    float* xmax = reinterpret_cast<float*>(smem + C::kXOff);          // [2][2][128]
+    float* xsum = reinterpret_cast<float*>(smem + C::kXOff + 2048);   // [2][128]
+    float m_run = -INFINITY, l_run = 0.f;            // l_run: this thread's part of the sum
     bool ok = true;
-    for (int it = 0; it < n_iter; ++it) {
+    if (C::kQT && n_iter > 0) {
+      // Q row r into TMEM (row r in lane r, head dims 2e, 2e+1 in column e); the warps
+      // of a quarter share the 64-column panels
+      ok = pair_all(__all_sync(0xFFFFFFFFu, mbar_wait(BAR(kBQ), 0, abort_flag, a.status, a.wait_limit_ns)));
+      if (ok) {
+        for (int pnl = hc; pnl < DQK / 64; pnl += kH) {
+          const uint8_t* prow = smem + C::kQOff + pnl * C::kPanel + r * 128;
+          uint32_t w[32];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint4 v = *reinterpret_cast<const uint4*>(prow + ((k ^ (r & 7)) << 4));
+            w[4 * k] = v.x;
+            w[4 * k + 1] = v.y;
+            w[4 * k + 2] = v.z;
+            w[4 * k + 3] = v.w;
+          }
+          tmem_st32(tl + C::kColQ + pnl * 32, w);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      mbar_arrive(BAR(kBQT));
+    }
+    for (int it = 0; ok && it < n_iter; ++it) {
       const int sb = it & 1;
-      const bool w_ok = mbar_wait(BAR(kBSF + sb), (it >> 1) & 1, abort_flag, a.status, a.wait_limit_ns);
-      if (!__all_sync(0xFFFFFFFFu, w_ok)) {
+      const bool w_ok = __all_sync(
+          0xFFFFFFFFu, mbar_wait(BAR(kBSF + sb), (it >> 1) & 1, abort_flag, a.status, a.wait_limit_ns));
+      if (!pair_all(w_ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t u[128];
-      tmem_ld32(tl + sb * 128 + 0, u + 0);
-      tmem_ld32(tl + sb * 128 + 32, u + 32);
-      tmem_ld32(tl + sb * 128 + 64, u + 64);
-      tmem_ld32(tl + sb * 128 + 96, u + 96);
-      tmem_wait_ld();
-      float x[128];
+      uint32_t u[kCols];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(u[c]);
+      for (int j = 0; j < kCols / 32; ++j) tmem_ld32(tl + sb * 128 + kCols * hc + 32 * j, u + 32 * j);
+      tmem_wait_ld();
+      float x[kCols];
+#pragma unroll
+      for (int c = 0; c < kCols; ++c) x[c] = __uint_as_float(u[c]);
       if (it >= n_full) {
-        // partial tile: element mask
+        // partial tile: element mask (tile columns kCols hc + c)
         const int nt = __ldg(list + it);
         const int64_t n0 = static_cast<int64_t>(nt) * 128;
         int64_t lim = a.Sk;
         if (a.causal) lim = min64(lim, i + 1);
-        const int lim_c = static_cast<int>(max64(0, min64(128, lim - n0)));
+        const int lim_c = static_cast<int>(max64(0, min64(128, lim - n0))) - kCols * hc;
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
+        for (int c = 0; c < kCols; ++c)
           if (c >= lim_c) x[c] = -INFINITY;
         if (row_ok && a.mode == SA_MODE_BLOCK && a.bs == 64) {
           const uint8_t* mrow = a.mask + (bg * a.Mb + i / 64) * a.Nb;
@@ -246,44 +307,55 @@ __global__ void __launch_bounds__(224, 1)
           const bool m0 = __ldg(mrow + c0) != 0;
           const bool m1 = (c0 + 1 < a.Nb) ? (__ldg(mrow + c0 + 1) != 0) : false;
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (!(c < 64 ? m0 : m1)) x[c] = -INFINITY;
+          for (int c = 0; c < kCols; ++c)
+            if (!(((kCols * hc + c) < 64) ? m0 : m1)) x[c] = -INFINITY;
         } else if (row_ok && a.mode == SA_MODE_INDEX) {
           const uint32_t* brow = a.bitmap + (bg * a.Sq + i) * a.W;
-          const int w0 = static_cast<int>(n0 / 32);
-          uint32_t wd[4];
+          const int w0 = static_cast<int>(n0 / 32) + (kCols / 32) * hc;
+          uint32_t wd[kCols / 32];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) wd[k] = (w0 + k < a.W) ? __ldg(brow + w0 + k) : 0u;
+          for (int k = 0; k < kCols / 32; ++k) wd[k] = (w0 + k < a.W) ? __ldg(brow + w0 + k) : 0u;
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
+          for (int c = 0; c < kCols; ++c)
             if (!((wd[c >> 5] >> (c & 31)) & 1u)) x[c] = -INFINITY;
         }
       }
-      // row max with eight independent chains (a single chain of 127 dependent fmaxf
-      // is latency bound: one softmax warp per SM sub-partition has nothing to hide it)
+      // row max over eight independent chains (a single chain of dependent fmaxf is
+      // latency bound), then the pair's
       float mx8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx8[k] = x[k];
 #pragma unroll
-      for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
+      for (int c = 8; c < kCols; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
       float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                        fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      if constexpr (kH == 2) {
+        float* xm = xmax + sb * 256;
+        xm[hc * 128 + r] = mx;
+        // both halves have loaded their S columns past this barrier, so P may now be
+        // written over them
+        named_bar_sync(pair_bar, 64);
+        mx = fmaxf(xm[r], xm[128 + r]);
+      }
       const float m_tile = mx * a.scale_log2;
       // Lazy rescale: only when this row's max grows by more than 2^8; the decision is
-      // taken per warp so that the warp-collective TMEM accesses stay converged.
+      // taken per warp (the warps of a pair hold the same rows and decide alike) so that
+      // the warp-collective TMEM accesses stay converged.
       const bool need = m_tile > m_run + 8.0f;
       if (__any_sync(0xFFFFFFFFu, need)) {
         const float alpha = need ? ex2(m_run - m_tile) : 1.f;  // 0 when m_run = -inf
         if (it > 0) {
-          // O holds P V up to tile it-1: rescale it in TMEM once that MMA is done.
-          bool w_ok = mbar_wait(BAR(kBOD), (it - 1) & 1, abort_flag, a.status, a.wait_limit_ns);
-          if (!__all_sync(0xFFFFFFFFu, w_ok)) {
+          // O holds P V up to tile it-1: rescale this thread's O columns in TMEM once
+          // that MMA is done
+          const bool o_ok = __all_sync(
+              0xFFFFFFFFu, mbar_wait(BAR(kBOD), (it - 1) & 1, abort_flag, a.status, a.wait_limit_ns));
+          if (!pair_all(o_ok)) {
             ok = false;
             break;
           }
           tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < DV; c += 32) {
+          for (int c = hc * kOCols; c < (hc + 1) * kOCols; c += 32) {
             uint32_t ov[32];
             tmem_ld32(tl + C::kOCol + c, ov);
             tmem_wait_ld();
@@ -302,7 +374,7 @@ __global__ void __launch_bounds__(224, 1)
       const float sc = a.scale_log2;
       float ps[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
+      for (int c0 = 0; c0 < kCols; c0 += 32) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -311,7 +383,8 @@ __global__ void __launch_bounds__(224, 1)
           ps[e & 3] += p0 + p1;
           pk[e] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(tl + sb * 128 + c0 / 2, pk);
+        // bf16 P of tile columns [kCols hc + c0, +32) over the S buffer
+        tmem_st16(tl + sb * 128 + (kCols / 2) * hc + c0 / 2, pk);
       }
       l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
       tmem_wait_st();
@@ -320,17 +393,24 @@ __global__ void __launch_bounds__(224, 1)
     }
     // ---------------------------------------------------------------- epilogue
     if (n_iter > 0 && ok) {
-      const bool w_ok = mbar_wait(BAR(kBOFin), 0, abort_flag, a.status, a.wait_limit_ns);
-      ok = __all_sync(0xFFFFFFFFu, w_ok);
+      const bool w_ok = __all_sync(
+          0xFFFFFFFFu, mbar_wait(BAR(kBOFin), 0, abort_flag, a.status, a.wait_limit_ns));
+      ok = pair_all(w_ok);
       tc_fence_after();
     }
-    const bool have_o = n_iter > 0 && ok;  // warp-uniform
-    const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+    const bool have_o = n_iter > 0 && ok;  // the same on both warps of a pair
+    float l_row = l_run;
+    if constexpr (kH == 2) {  // the row sum is the sum of the two halves'
+      xsum[hc * 128 + r] = l_run;
+      named_bar_sync(pair_bar, 64);
+      l_row = xsum[r] + xsum[128 + r];
+    }
+    const float inv = (l_row > 0.f) ? 1.f / l_row : 0.f;
     // O rows go to the Q buffer (idle once the last P V is done: every S MMA came
     // before it) as [128 rows][64 cols] 128-byte-swizzled panels, the output map's box,
-    // and leave by TMA stores, which drop rows past Sq
+    // and leave by TMA stores, which drop rows past Sq; each thread writes its columns
 #pragma unroll 1
-    for (int c = 0; c < DV; c += 32) {
+    for (int c = hc * kOCols; c < (hc + 1) * kOCols; c += 32) {
       uint32_t ov[32];
       if (have_o) {
         tmem_ld32(tl + C::kOCol + c, ov);
@@ -352,7 +432,7 @@ __global__ void __launch_bounds__(224, 1)
             make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
     }
     fence_proxy_async_smem();
-    named_bar_sync(1, 128);
+    named_bar_sync(5, 128 * kH);  // every softmax warp
     if (threadIdx.x == 64) {
 #pragma unroll
       for (int p = 0; p < DV / 64; ++p)
@@ -360,10 +440,10 @@ __global__ void __launch_bounds__(224, 1)
       bulk_commit_group();
       bulk_wait_group_read0();  // the Q buffer is read before the CTA may leave
     }
-    if (row_ok) {
+    if (row_ok && hc == 0) {
       const float m_eff = (m_run == -INFINITY) ? 0.f : m_run;
       a.lse[(static_cast<int64_t>(b) * a.HQ + h) * a.Sq + i] =
-          (l_run > 0.f) ? (m_eff + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+          (l_row > 0.f) ? (m_eff + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
     }
   }
 
@@ -381,7 +461,7 @@ __global__ void __launch_bounds__(224, 1)
         mbar_wait_limited(BAR(kBQ), 0);
         for (int it = max(0, issued_k - C::kKStages); it < issued_k; ++it)
           mbar_wait_limited(BAR(kBKF + it % C::kKStages), (it / C::kKStages) & 1);
-      } else if (warp == 6) {
+      } else if (warp == C::kVWarp) {
         for (int it = max(0, issued_v - C::kVStages); it < issued_v; ++it)
           mbar_wait_limited(BAR(kBVF + it % C::kVStages), (it / C::kVStages) & 1);
       }
@@ -403,28 +483,36 @@ __global__ void __launch_bounds__(224, 1)
   }
 }
 
-template <int DQK, int DV>
+template <int DQK, int DV, bool PAIRED>
 static int launch_fwd_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
-  using C = FwdCfg<DQK, DV>;
+  using C = FwdCfg<DQK, DV, PAIRED>;
   static PerDeviceOnce attr;
   const int rc = once_per_device(attr, [] {
-    return cuda_error(cudaFuncSetAttribute(sparse_fwd_kernel<DQK, DV>,
+    return cuda_error(cudaFuncSetAttribute(sparse_fwd_kernel<DQK, DV, PAIRED>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem),
                       "forward smem attribute");
   });
   if (rc) return rc;
   dim3 grid(a.Tm, a.HQ, a.B);
   record_event(0, st);
-  sparse_fwd_kernel<DQK, DV><<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.v, m.o, a);
+  sparse_fwd_kernel<DQK, DV, PAIRED><<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.v, m.o, a);
   record_event(1, st);
   return check_launch("forward kernel launch");
 }
 
+// Index mode pairs the softmax warps (its partial-tile bitmap masks make one softmax warp
+// per SM sub-partition issue bound); block and dense modes keep one (measured faster).
+template <int DQK, int DV>
+static int launch_fwd_dims(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
+  return a.mode == SA_MODE_INDEX ? launch_fwd_t<DQK, DV, true>(a, m, st)
+                                 : launch_fwd_t<DQK, DV, false>(a, m, st);
+}
+
 int launch_fwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
-  if (a.Dqk == 64 && a.Dv == 64) return launch_fwd_t<64, 64>(a, m, st);
-  if (a.Dqk == 128 && a.Dv == 128) return launch_fwd_t<128, 128>(a, m, st);
-  if (a.Dqk == 192 && a.Dv == 128) return launch_fwd_t<192, 128>(a, m, st);
-  if (a.Dqk == 256 && a.Dv == 256) return launch_fwd_t<256, 256>(a, m, st);
+  if (a.Dqk == 64 && a.Dv == 64) return launch_fwd_dims<64, 64>(a, m, st);
+  if (a.Dqk == 128 && a.Dv == 128) return launch_fwd_dims<128, 128>(a, m, st);
+  if (a.Dqk == 192 && a.Dv == 128) return launch_fwd_dims<192, 128>(a, m, st);
+  if (a.Dqk == 256 && a.Dv == 256) return launch_fwd_dims<256, 256>(a, m, st);
   return SA_ERR_UNSUPPORTED;
 }
 
