@@ -100,20 +100,6 @@ __global__ void bwd_post_kernel(const float* __restrict__ dq_acc, __nv_bfloat16*
 // DQK, DV: the head dims the kernel is built for (64-wide inputs run through the
 // 128 instance with zero-filled loads); NSPLIT: CTAs sharing one key tile, each owning
 // one head-dim chunk of dK / dV / dQ.
-// 32 x 32 bit-matrix transpose across a converged warp: on entry lane L holds row L
-// (bit c = column c), on exit column L (bit r = row r).  Five butterfly stages: at
-// stage j, lanes whose bit j is clear keep the low half of each 2j-bit group and take
-// the partner's low halves into their high halves, the others the reverse.
-__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
-  uint32_t m = 0x0000FFFFu;
-#pragma unroll
-  for (int j = 16; j != 0; j >>= 1, m ^= (m << j)) {
-    const uint32_t y = __shfl_xor_sync(0xFFFFFFFFu, x, j);
-    x = (lane & j) ? ((x & ~m) | ((y >> j) & m)) : ((x & m) | ((y << j) & ~m));
-  }
-  return x;
-}
-
 template <int DQK, int DV, int NSPLIT>
 struct BwdCfg {
   static constexpr int kBM = 64;                     // queries per inner step

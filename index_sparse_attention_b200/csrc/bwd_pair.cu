@@ -553,18 +553,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                            __ldg(a.mask + (bg * a.Mb + mb) * static_cast<int64_t>(a.Nb) + j / 64) != 0;
             if (!m) cm = 0u;
           } else if (a.mode == SA_MODE_INDEX) {
-            // presence word of this key row's 32-key group for each of the 32 queries
-            // (the same address across the warp: one broadcast load per query)
+            // lane L loads the presence word of query q0 + L over this warp's 32 key rows
+            // (one word: key rows 32 quarter .. +31); a bit transpose across the warp
+            // leaves in lane L the word of key row r over the 32 queries (the branch is
+            // warp-uniform)
             const int w = nt * 4 + (r >> 5);
-            uint32_t bits = 0u;
-#pragma unroll 8
-            for (int q = 0; q < 32; ++q) {
-              const int64_t i = q0 + q;
-              const uint32_t word =
-                  (i < a.Sq && w < a.W) ? __ldg(a.bitmap + (bg * a.Sq + i) * a.W + w) : 0u;
-              bits |= ((word >> lane) & 1u) << q;
-            }
-            cm &= bits;
+            const int64_t i = q0 + lane;
+            const uint32_t word =
+                (i < a.Sq && w < a.W) ? __ldg(a.bitmap + (bg * a.Sq + i) * a.W + w) : 0u;
+            cm &= warp_transpose32(word, lane);
           }
         }
         tmem_wait_ld();

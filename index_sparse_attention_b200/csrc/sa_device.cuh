@@ -425,6 +425,19 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
 // ---------------------------------------------------------------------------------
 // Small numeric helpers
 // ---------------------------------------------------------------------------------
+// 32 x 32 bit-matrix transpose across a converged warp: on entry lane L holds row L
+// (bit c = column c), on exit column L (bit r = row r).  Five butterfly stages: at
+// stage j, lanes whose bit j is clear keep the low half of each 2j-bit group and take
+// the partner's low halves into their high halves, the others the reverse.
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
+  uint32_t m = 0x0000FFFFu;
+#pragma unroll
+  for (int j = 16; j != 0; j >>= 1, m ^= (m << j)) {
+    const uint32_t y = __shfl_xor_sync(0xFFFFFFFFu, x, j);
+    x = (lane & j) ? ((x & ~m) | ((y >> j) & m)) : ((x & m) | ((y << j) & ~m));
+  }
+  return x;
+}
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
