@@ -263,6 +263,11 @@ def get_workload(args):
     w = I.WORKLOADS[args.workload]
     if args.seq:
         w = I.scaled(w, Sq=args.seq, Sk=args.seq, name=f"{w.name}@S{args.seq}")
+    if getattr(args, "heads", ""):
+        hq, hk = (int(x) for x in args.heads.split(","))
+        if hq <= 0 or hk <= 0 or hq % hk:
+            raise SystemExit("--heads wants HQ,HK with HQ a multiple of HK")
+        w = I.scaled(w, HQ=hq, HK=hk, name=f"{w.name}@H{hq}x{hk}")
     return w
 
 
@@ -335,6 +340,7 @@ def run_gpu(args):
     from index_sparse_attention_b200 import _lib
 
     L = _lib.load()
+    sa.sparse_attn_set_forward_pairs(args.fwd_pairs)
     w = get_workload(args)
     inp = I.make_inputs(w)
     dev = torch.device("cuda", local)
@@ -513,7 +519,9 @@ def run_gpu(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": dict(workload_config(w, active),
-                           **({"backward": "deterministic"} if args.deterministic else {})),
+                           **({"backward": "deterministic"} if args.deterministic else {}),
+                           **({"forward_pairs": args.fwd_pairs} if args.fwd_pairs != "auto"
+                              else {})),
             "pct_of_bf16_peak": 100.0 * (value / world) / peak,
             "pct_basis": (f"{peak_kind} {peak:.1f} TFLOP/s ({of}); burst unless the clock record "
                           "of the timed region shows sw_power_cap"),
@@ -728,6 +736,11 @@ def main():
                     help="override Sq = Sk (smaller profiling captures of the same kernels)")
     ap.add_argument("--deterministic", action="store_true",
                     help="use the deterministic backward (fixed-order dQ accumulation)")
+    ap.add_argument("--heads", default="",
+                    help="override the head counts as HQ,HK (e.g. 16,8: GQA on the D=256 workload)")
+    ap.add_argument("--fwd-pairs", default="auto", choices=["auto", "on", "off"],
+                    help="forward form for GQA: CTA pairs with cta_group::2 MMAs (on), one "
+                         "CTA per query tile and head (off), or the library's choice (auto)")
     ap.add_argument("--op", default="attention", choices=["attention", "topk", "index_stats"],
                     help="topk: time the top-k selector alone on one packed sequence; "
                          "index_stats: counts on an index workload (CPU only)")

@@ -232,6 +232,28 @@ int sparse_attn_set_timing_events(void *const *events);
  */
 int sparse_attn_set_wait_limit_ns(uint64_t ns);
 
+/* Policies of sparse_attn_set_forward_pairs. */
+#define SA_FWD_PAIRS_AUTO 0
+#define SA_FWD_PAIRS_ON 1
+#define SA_FWD_PAIRS_OFF 2
+
+/*
+ * sparse_attn_set_forward_pairs -- selects the form of the forward for GQA.  The pages
+ * have 256-row tiles on SM100 (MagiAttention PR #331, "CSR Tile Mapping") and a switch
+ * that turns the 2-CTA mode off (MagiAttention PR #334, section 3, disable_2cta); the
+ * pair form here is this library's own.  The query heads of one GQA group walk the same tile
+ * list, so with an even group size and Dv >= 128 the forward can run two of them (same
+ * query tile) on a pair of CTAs: a 2-CTA cluster whose tensor-core MMAs span both CTAs
+ * (tcgen05 cta_group::2, M = 256) and which split every K and V tile between them.
+ *   SA_FWD_PAIRS_AUTO  the pair form where it is measured faster (Dqk = Dv = 256);
+ *   SA_FWD_PAIRS_ON    the pair form wherever it applies;
+ *   SA_FWD_PAIRS_OFF   one CTA per (query tile, query head) always.
+ * Both forms compute the same O and LSE up to fp32 rounding.  Applies to the forward
+ * calls enqueued after it; process-wide.  Returns SA_OK, or SA_ERR_INVALID for another
+ * value (the setting is then unchanged).
+ */
+int sparse_attn_set_forward_pairs(int policy);
+
 
 /* Largest k that topk_select supports. */
 #define SA_TOPK_MAX_K 4096

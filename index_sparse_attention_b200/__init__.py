@@ -17,6 +17,7 @@ from ._lib import SA_MODE_BLOCK, SA_MODE_DENSE, SA_MODE_INDEX, SA_TILE, SparseAt
 __all__ = ["BlockSparse", "block_mask_to_block_sparse", "index_to_block_sparse",
            "sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_bwd_workspace_size",
            "sparse_attn_bwd_noalloc", "topk_select", "sparse_attn_set_wait_limit_ns",
+           "sparse_attn_set_forward_pairs",
            "SparseAttnError", "SA_TILE"]
 
 
@@ -301,3 +302,18 @@ def sparse_attn_set_wait_limit_ns(ns):
     out sets bit 2 of the device status word and its CTA leaves; see
     include/sparse_attn.h."""
     _lib.check("sparse_attn_set_wait_limit_ns", _lib.load().sparse_attn_set_wait_limit_ns(int(ns)))
+
+
+_FWD_PAIRS = {"auto": _lib.SA_FWD_PAIRS_AUTO, "on": _lib.SA_FWD_PAIRS_ON,
+              "off": _lib.SA_FWD_PAIRS_OFF}
+
+
+def sparse_attn_set_forward_pairs(policy):
+    """The forward's form for GQA: "auto" (the library's choice: CTA pairs sharing K/V
+    tiles through cta_group::2 MMAs at head dims 256), "on" (pairs wherever the group
+    size is even and Dv >= 128) or "off" (one CTA per query tile and head).  Applies to
+    the forward calls made after it, process-wide; see include/sparse_attn.h."""
+    code = _FWD_PAIRS.get(policy, policy) if isinstance(policy, str) else int(policy)
+    if isinstance(code, str):
+        raise ValueError(f"policy must be one of {sorted(_FWD_PAIRS)}, got {policy!r}")
+    _lib.check("sparse_attn_set_forward_pairs", _lib.load().sparse_attn_set_forward_pairs(code))

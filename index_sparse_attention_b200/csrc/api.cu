@@ -22,6 +22,7 @@ int cuda_error(cudaError_t e, const char* what) {
 cudaEvent_t* g_timing_events = nullptr;
 static cudaEvent_t g_events_copy[6];
 std::atomic<uint64_t> g_wait_limit_ns{0};
+std::atomic<int> g_fwd_pairs{SA_FWD_PAIRS_AUTO};
 }  // namespace sa
 
 namespace {
@@ -142,8 +143,9 @@ int fill_args(const sparse_attn_params* p, AttnArgs* a, bool backward) {
   return SA_OK;
 }
 
-// Forward: Q in 128-row boxes.  Backward: Q and dO in 64-row boxes (the backward
-// consumes query tiles in 64-row halves).  K and V: 128-row boxes.
+// Forward: Q in 128-row boxes, K also in 64-row boxes (CTA pairs load half tiles).
+// Backward: Q and dO in 64-row boxes (the backward consumes query tiles in 64-row
+// halves).  K and V: 128-row boxes.
 int fill_maps(const sparse_attn_params* p, TensorMaps* m, bool backward) {
   const int qrows = backward ? 64 : 128;
   if (!make_map(&m->q, p->q, p->Dqk, p->Sq, p->HQ, p->B, qrows)) return SA_ERR_CUDA;
@@ -151,6 +153,8 @@ int fill_maps(const sparse_attn_params* p, TensorMaps* m, bool backward) {
   if (!make_map(&m->v, p->v, p->Dv, p->Sk, p->HK, p->B, 128)) return SA_ERR_CUDA;
   // O output of the forward (written by TMA stores in 128-row boxes)
   if (!backward && !make_map(&m->o, p->o, p->Dv, p->Sq, p->HQ, p->B, 128)) return SA_ERR_CUDA;
+  // K half tiles of the forward's CTA pairs (64-row boxes)
+  if (!backward && !make_map(&m->kh, p->k, p->Dqk, p->Sk, p->HK, p->B, 64)) return SA_ERR_CUDA;
   if (backward && !make_map(&m->dout, p->dout, p->Dv, p->Sq, p->HQ, p->B, qrows))
     return SA_ERR_CUDA;
   // dK / dV outputs (written by TMA stores in 128-row boxes)
@@ -192,6 +196,13 @@ extern "C" int sparse_attn_set_timing_events(void* const* events) {
 
 extern "C" int sparse_attn_set_wait_limit_ns(uint64_t ns) {
   g_wait_limit_ns.store(ns, std::memory_order_relaxed);
+  return SA_OK;
+}
+
+extern "C" int sparse_attn_set_forward_pairs(int policy) {
+  if (policy != SA_FWD_PAIRS_AUTO && policy != SA_FWD_PAIRS_ON && policy != SA_FWD_PAIRS_OFF)
+    return SA_ERR_INVALID;
+  g_fwd_pairs.store(policy, std::memory_order_relaxed);
   return SA_OK;
 }
 

@@ -27,21 +27,37 @@
 //              swizzled box layout, sent by TMA tensor stores) and writes LSE (fp32,
 //              natural log).  One softmax warp per SM sub-partition was issue bound.
 // TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+Dv).
+//
+// GQA pair form (CG2): the query heads of one GQA group walk the same tile list, so two
+// of them (heads 2j and 2j+1, same query tile) run on a 2-CTA cluster whose MMAs are
+// pair MMAs (tcgen05 cta_group::2, M = 256: each CTA's 128 query rows).  The pair shares
+// every K and V tile: each CTA loads and holds half of it (keys [64 r, 64 r + 64) of K,
+// head-dim columns [Dv/2 r, Dv/2 r + Dv/2) of V, r = cluster rank), which halves the
+// per-CTA copy volume and shared-memory operand reads of B.  The even CTA (the leader)
+// issues every MMA; its commits arrive on the barriers of both CTAs; both CTAs' loads
+// complete on the leader's full barriers; the odd CTA's softmax warps report P (and Q
+// in TMEM) to the leader with one remote arrival per warp.  Softmax, masks, epilogue
+// and LSE are per CTA, as in the single-CTA form.
 // Every mbarrier wait is bounded; a timeout sets SA_ERR_TIMEOUT in the status word and
 // the CTA leaves after releasing its tensor memory.
 #include "sa_device.cuh"
 #include "sa_kernels.h"
+#include "sa_pair2.cuh"
 
 namespace sa {
 
-template <int DQK, int DV, bool PAIRED>
+template <int DQK, int DV, bool PAIRED, bool CG2>
 struct FwdCfg {
   static constexpr int kPanel = 128 * 128;  // one 64-column x 128-row swizzled panel
+  // K rows and V columns one CTA holds per tile (a pair splits both in halves)
+  static constexpr int kKRows = CG2 ? 64 : 128;
+  static constexpr int kKPanel = kKRows * 128;  // one 64-column panel of K
+  static constexpr int kVCols = CG2 ? DV / 2 : DV;
   static constexpr int kQBytes = 128 * DQK * 2;
-  static constexpr int kKBytes = 128 * DQK * 2;
-  static constexpr int kVBytes = 128 * DV * 2;
-  static constexpr int kKStages = (DQK == 256) ? 1 : 2;
-  static constexpr int kVStages = (DV == 256) ? 1 : 2;
+  static constexpr int kKBytes = kKRows * DQK * 2;
+  static constexpr int kVBytes = 128 * kVCols * 2;
+  static constexpr int kKStages = CG2 ? (DQK == 256 ? 2 : 3) : (DQK == 256 ? 1 : 2);
+  static constexpr int kVStages = CG2 ? (DV == 256 ? 2 : 3) : (DV == 256 ? 1 : 2);
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kQBytes;
   static constexpr int kVOff = kKOff + kKStages * kKBytes;
@@ -64,19 +80,24 @@ struct FwdCfg {
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
   static_assert(kOCol + DV <= kTmemCols, "tensor memory budget");
   static_assert(!kQT || kColQ + DQK / 2 <= kTmemCols, "tensor memory budget (Q)");
+  static_assert(!CG2 || DV >= 128, "a CTA pair splits V into 64-column panels");
+  static_assert(kKStages <= 4 && kVStages <= 4, "barrier slots");
 };
 
-// barrier slots
-enum : int { kBQ = 0, kBKF = 1, kBKE = 3, kBVF = 5, kBVE = 7, kBSF = 9, kBPF = 11, kBOD = 13,
-             kBDrain = 14, kBOFin = 15, kBQT = 16, kNumBars = 17 };
+// barrier slots (up to four K and four V stages)
+enum : int { kBQ = 0, kBKF = 1, kBKE = 5, kBVF = 9, kBVE = 13, kBSF = 17, kBPF = 19, kBOD = 21,
+             kBDrain = 22, kBOFin = 23, kBQT = 24, kNumBars = 25 };
 
-template <int DQK, int DV, bool PAIRED>
+// tm_kh: K in 64-row boxes (the half tile a CTA of a pair loads); unused by the
+// single-CTA form.
+template <int DQK, int DV, bool PAIRED, bool CG2>
 __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
     sparse_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_kh,
                       const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_o, const AttnArgs a) {
-  using C = FwdCfg<DQK, DV, PAIRED>;
+  using C = FwdCfg<DQK, DV, PAIRED, CG2>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -88,8 +109,16 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
   auto BAR = [&](int k) { return bar0 + 8u * static_cast<uint32_t>(k); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = a.Tm - 1 - static_cast<int>(blockIdx.x);  // longest lists first under causal
-  const int h = blockIdx.y, b = blockIdx.z;
+  // pair: the two CTAs of a cluster are blockIdx.x = 2c, 2c + 1 (rank 0 leads)
+  const uint32_t rank = CG2 ? cluster_ctarank() : 0u;
+  const int xt = CG2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int mt = a.Tm - 1 - xt;  // longest lists first under causal
+  const int h = CG2 ? 2 * static_cast<int>(blockIdx.y) + static_cast<int>(rank)
+                    : static_cast<int>(blockIdx.y);
+  const int b = blockIdx.z;
+  // the leader's barriers as seen from this CTA (remote arrivals and pair loads)
+  const uint32_t lbar0 = CG2 ? mapa_shared(bar0, 0) : bar0;
+  auto LBAR = [&](int k) { return lbar0 + 8u * static_cast<uint32_t>(k); };
   const int g = h / (a.HQ / a.HK);
   const int64_t bg = static_cast<int64_t>(b) * a.HK + g;
   const int64_t lrow = bg * a.Tm + mt;
@@ -99,29 +128,41 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
   // loads issued by the two producers (the abort path drains the last ones in flight)
   int issued_k = 0, issued_v = 0;
 
+  // P / Q-in-TMEM ready: one arrival per softmax thread; in a pair, one per softmax
+  // warp of either CTA on the leader's barrier
+  constexpr uint32_t kReadyCount = CG2 ? 2 * 4 * C::kHalves : 128 * C::kHalves;
   if (threadIdx.x == 0) {
     mbar_init(BAR(kBQ), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < 4; ++s) {
       mbar_init(BAR(kBKF + s), 1);
       mbar_init(BAR(kBKE + s), 1);
       mbar_init(BAR(kBVF + s), 1);
       mbar_init(BAR(kBVE + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(kBSF + s), 1);
-      mbar_init(BAR(kBPF + s), 128 * C::kHalves);
+      mbar_init(BAR(kBPF + s), kReadyCount);
     }
     mbar_init(BAR(kBOD), 1);
     mbar_init(BAR(kBDrain), 1);
     mbar_init(BAR(kBOFin), 1);
-    mbar_init(BAR(kBQT), 128 * C::kHalves);
+    mbar_init(BAR(kBQT), kReadyCount);
     abort_flag->abort = 0;
+    abort_flag->peer_abort = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
-    tmem_relinquish();
+    if constexpr (CG2) {
+      tmem_alloc_pair(smem_u32(tmem_slot), C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (CG2) cluster_sync_all();  // both CTAs' barriers exist before any remote use
   tc_fence_after();
   // broadcast from lane 0 so that the compiler can treat it as warp-uniform
   const uint32_t tmem = __shfl_sync(0xFFFFFFFFu, *tmem_slot, 0);
@@ -134,9 +175,18 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
-        mbar_arrive_expect_tx(BAR(kBQ), C::kQBytes);
-        for (int c = 0; c < DQK / 64; ++c)
-          tma_load_4d(sbase + C::kQOff + c * C::kPanel, &tm_q, BAR(kBQ), c * 64, mt * 128, h, b);
+        if (CG2 && !C::kQT) {
+          // the leader's S MMAs read Q from both CTAs' shared memory: both Q loads
+          // complete on the leader's barrier
+          if (rank == 0) mbar_arrive_expect_tx(BAR(kBQ), 2 * C::kQBytes);
+          for (int c = 0; c < DQK / 64; ++c)
+            tma_load_4d_pair(sbase + C::kQOff + c * C::kPanel, &tm_q, LBAR(kBQ), c * 64, mt * 128,
+                             h, b);
+        } else {
+          mbar_arrive_expect_tx(BAR(kBQ), C::kQBytes);
+          for (int c = 0; c < DQK / 64; ++c)
+            tma_load_4d(sbase + C::kQOff + c * C::kPanel, &tm_q, BAR(kBQ), c * 64, mt * 128, h, b);
+        }
       }
       __syncwarp();
       // K tiles: each one as soon as S of the tile that last used its buffer is done (V
@@ -146,14 +196,28 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
         const int ks = it % C::kKStages, ku = it / C::kKStages;
         if (!warp_wait(BAR(kBKE + ks), (ku & 1) ^ 1, abort_flag, a.status, a.wait_limit_ns)) break;
         if (elect_one()) {
-          mbar_arrive_expect_tx(BAR(kBKF + ks), C::kKBytes);
-          for (int c = 0; c < DQK / 64; ++c)
-            tma_load_4d(sbase + C::kKOff + ks * C::kKBytes + c * C::kPanel, &tm_k, BAR(kBKF + ks),
-                        c * 64, nt * 128, g, b);
+          if constexpr (CG2) {  // keys [64 rank, +64) of the tile, on the leader's barrier
+            if (rank == 0) mbar_arrive_expect_tx(BAR(kBKF + ks), 2 * C::kKBytes);
+            for (int c = 0; c < DQK / 64; ++c)
+              tma_load_4d_pair(sbase + C::kKOff + ks * C::kKBytes + c * C::kKPanel, &tm_kh,
+                               LBAR(kBKF + ks), c * 64, nt * 128 + 64 * static_cast<int>(rank), g, b);
+          } else {
+            mbar_arrive_expect_tx(BAR(kBKF + ks), C::kKBytes);
+            for (int c = 0; c < DQK / 64; ++c)
+              tma_load_4d(sbase + C::kKOff + ks * C::kKBytes + c * C::kPanel, &tm_k,
+                          BAR(kBKF + ks), c * 64, nt * 128, g, b);
+          }
         }
         __syncwarp();
         issued_k = it + 1;
       }
+      // pair: the leader's commits arrive on this CTA's barriers too; wait for the ones
+      // that free the last stages so that none is in flight when the CTA leaves
+      if (CG2 && issued_k == n_iter)
+        for (int it = n_iter; it < n_iter + C::kKStages; ++it)
+          if (!warp_wait(BAR(kBKE + it % C::kKStages), ((it / C::kKStages) & 1) ^ 1, abort_flag,
+                         a.status, a.wait_limit_ns))
+            break;
     }
   } else if (warp == C::kVWarp) {
     // ------------------------------------------------------------------ V producer
@@ -163,23 +227,42 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
         const int vs = it % C::kVStages, vu = it / C::kVStages;
         if (!warp_wait(BAR(kBVE + vs), (vu & 1) ^ 1, abort_flag, a.status, a.wait_limit_ns)) break;
         if (elect_one()) {
-          mbar_arrive_expect_tx(BAR(kBVF + vs), C::kVBytes);
-          for (int c = 0; c < DV / 64; ++c)
-            tma_load_4d(sbase + C::kVOff + vs * C::kVBytes + c * C::kPanel, &tm_v, BAR(kBVF + vs),
-                        c * 64, nt * 128, g, b);
+          if constexpr (CG2) {  // head-dim columns [Dv/2 rank, +Dv/2), on the leader's barrier
+            if (rank == 0) mbar_arrive_expect_tx(BAR(kBVF + vs), 2 * C::kVBytes);
+            for (int c = 0; c < C::kVCols / 64; ++c)
+              tma_load_4d_pair(sbase + C::kVOff + vs * C::kVBytes + c * C::kPanel, &tm_v,
+                               LBAR(kBVF + vs), static_cast<int>(rank) * C::kVCols + c * 64,
+                               nt * 128, g, b);
+          } else {
+            mbar_arrive_expect_tx(BAR(kBVF + vs), C::kVBytes);
+            for (int c = 0; c < DV / 64; ++c)
+              tma_load_4d(sbase + C::kVOff + vs * C::kVBytes + c * C::kPanel, &tm_v,
+                          BAR(kBVF + vs), c * 64, nt * 128, g, b);
+          }
         }
         __syncwarp();
         issued_v = it + 1;
       }
+      if (CG2 && issued_v == n_iter)
+        for (int it = n_iter; it < n_iter + C::kVStages; ++it)
+          if (!warp_wait(BAR(kBVE + it % C::kVStages), ((it / C::kVStages) & 1) ^ 1, abort_flag,
+                         a.status, a.wait_limit_ns))
+            break;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     // The whole warp runs this loop (converged, warp-uniform operands); one elected
-    // lane issues each batch of tcgen05 instructions.
-    if (n_iter > 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16(128, DV, 0, 1);
+    // lane issues each batch of tcgen05 instructions.  In a pair only the leader issues
+    // (M = 256: both CTAs' rows), and every commit arrives on both CTAs' barriers.
+    if (n_iter > 0 && rank == 0) {
+      constexpr int kM = CG2 ? 256 : 128;
+      constexpr uint32_t idesc_qk = idesc_bf16(kM, 128, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16(kM, DV, 0, 1);
       const uint64_t qdesc = sw128_desc(sbase + C::kQOff, 16, 1024);
+      auto commit = [&](int bar) {
+        if constexpr (CG2) umma_commit_pair(BAR(bar), 3);
+        else umma_commit(BAR(bar));
+      };
       // Q in TMEM (kQT): the softmax warps have copied it there
       bool ok = warp_wait(BAR(C::kQT ? kBQT : kBQ), 0, abort_flag, a.status, a.wait_limit_ns);
       auto issue_s = [&](int it) -> bool {
@@ -191,14 +274,22 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < DQK / 16; ++kk) {
-            const uint32_t off = ((kk >> 2) * C::kPanel + (kk & 3) * 32) >> 4;
-            if constexpr (C::kQT)  // A = Q from TMEM: 16 head dims = 8 columns per k-step
-              umma_ts(d, tmem + C::kColQ + kk * 8, kdesc + off, idesc_qk, kk > 0 ? 1u : 0u);
-            else
-              umma_ss(d, qdesc + off, kdesc + off, idesc_qk, kk > 0 ? 1u : 0u);
+            const uint32_t qoff = ((kk >> 2) * C::kPanel + (kk & 3) * 32) >> 4;
+            const uint32_t koff = ((kk >> 2) * C::kKPanel + (kk & 3) * 32) >> 4;
+            if constexpr (C::kQT) {  // A = Q from TMEM: 16 head dims = 8 columns per k-step
+              if constexpr (CG2)
+                umma_ts_pair(d, tmem + C::kColQ + kk * 8, kdesc + koff, idesc_qk, kk > 0 ? 1u : 0u);
+              else
+                umma_ts(d, tmem + C::kColQ + kk * 8, kdesc + koff, idesc_qk, kk > 0 ? 1u : 0u);
+            } else {
+              if constexpr (CG2)
+                umma_ss_pair(d, qdesc + qoff, kdesc + koff, idesc_qk, kk > 0 ? 1u : 0u);
+              else
+                umma_ss(d, qdesc + qoff, kdesc + koff, idesc_qk, kk > 0 ? 1u : 0u);
+            }
           }
-          umma_commit(BAR(kBSF + (it & 1)));
-          umma_commit(BAR(kBKE + ks));
+          commit(kBSF + (it & 1));
+          commit(kBKE + ks);
         }
         __syncwarp();
         return true;
@@ -214,12 +305,19 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
         const uint32_t pa = tmem + static_cast<uint32_t>((it & 1) * 128);
         if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk)
-            umma_ts(tmem + C::kOCol, pa + kk * 8, vdesc + ((kk * 2048) >> 4), idesc_pv,
-                    (it > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(BAR(kBOD));
-          umma_commit(BAR(kBVE + vs));
-          if (it == n_iter - 1) umma_commit(BAR(kBOFin));  // the final O is complete
+          for (int kk = 0; kk < 128 / 16; ++kk) {
+            if constexpr (CG2)
+              umma_ts_pair(tmem + C::kOCol, pa + kk * 8, vdesc + ((kk * 2048) >> 4), idesc_pv,
+                           (it > 0 || kk > 0) ? 1u : 0u);
+            else
+              umma_ts(tmem + C::kOCol, pa + kk * 8, vdesc + ((kk * 2048) >> 4), idesc_pv,
+                      (it > 0 || kk > 0) ? 1u : 0u);
+          }
+          // (pair: no O-done arrival after the last P V, which nobody waits for: every
+          // arrival on the other CTA's barriers is observed before it leaves)
+          if (!CG2 || it < n_iter - 1) commit(kBOD);
+          commit(kBVE + vs);
+          if (it == n_iter - 1) commit(kBOFin);  // the final O is complete
         }
         __syncwarp();
       }
@@ -252,6 +350,20 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
     float* xsum = reinterpret_cast<float*>(smem + C::kXOff + 2048);   // [2][128]
     float m_run = -INFINITY, l_run = 0.f;            // l_run: this thread's part of the sum
     bool ok = true;
+    // Tell the MMA issuer that this warp's TMEM stores are done (the caller has waited
+    // for them and fenced): per thread on this CTA's barrier, or in a pair per warp on
+    // the leader's (a relaxed remote arrival: the stores have completed before it)
+    auto ready = [&](int bar) {
+      if constexpr (CG2) {
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0) mbar_arrive(BAR(bar));
+          else mbar_arrive_remote_relaxed(LBAR(bar));
+        }
+      } else {
+        mbar_arrive(BAR(bar));
+      }
+    };
     if (C::kQT && n_iter > 0) {
       // Q row r into TMEM (row r in lane r, head dims 2e, 2e+1 in column e); the warps
       // of a quarter share the 64-column panels
@@ -273,7 +385,7 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
         tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive(BAR(kBQT));
+      ready(kBQT);
     }
     for (int it = 0; ok && it < n_iter; ++it) {
       const int sb = it & 1;
@@ -389,7 +501,7 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
       l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(BAR(kBPF + sb));
+      ready(kBPF + sb);
     }
     // ---------------------------------------------------------------- epilogue
     if (n_iter > 0 && ok) {
@@ -449,15 +561,33 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
 
   tc_fence_before();
   __syncthreads();
+  bool any_abort = abort_flag->abort != 0;
+  if constexpr (CG2) {
+    // This CTA's abort flag no longer changes: hand it to the peer (a store into the
+    // peer's shared memory while both CTAs are certainly resident), then meet.  Past the
+    // meeting neither CTA issues an MMA, a copy or an arrival to the other, and neither
+    // touches the pair's tensor memory: in the normal path every commit, remote arrival
+    // and load of the pair has been observed by a wait of its receiver.
+    if (threadIdx.x == 0)
+      st_shared_cluster_u32(
+          mapa_shared(smem_u32(const_cast<int*>(&abort_flag->peer_abort)), rank ^ 1u),
+          static_cast<uint32_t>(abort_flag->abort));
+    cluster_sync_all();
+    any_abort = abort_flag->abort != 0 || abort_flag->peer_abort != 0;
+  }
   // Abort path.  Past the barrier above no warp issues another copy or MMA, and the
-  // abort flag no longer changes (the branch is uniform).  A K or V buffer is reloaded
+  // abort flags no longer change (the branch is uniform).  A K or V buffer is reloaded
   // only after the MMA that read its previous tile has completed, so at most the last
   // kKStages K loads and kVStages V loads can still be in flight: wait for them, and for
   // every MMA this CTA issued, before shared memory and TMEM are released
-  // (time-limited waits).
-  if (abort_flag->abort) {
+  // (time-limited waits).  A pair's loads complete on the leader's barriers, whose
+  // phases an abort leaves unknown: there both CTAs wait for the leader's MMAs, stay
+  // resident for 50 us (against a few microseconds per load) and meet once more.
+  if (any_abort) {
     if (n_iter > 0 && lane == 0) {
-      if (warp == 0) {
+      if constexpr (CG2) {
+        if (warp == 0 && (C::kQT || rank == 0)) mbar_wait_limited(BAR(kBQ), 0);
+      } else if (warp == 0) {
         mbar_wait_limited(BAR(kBQ), 0);
         for (int it = max(0, issued_k - C::kKStages); it < issued_k; ++it)
           mbar_wait_limited(BAR(kBKF + it % C::kKStages), (it / C::kKStages) & 1);
@@ -466,46 +596,85 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
           mbar_wait_limited(BAR(kBVF + it % C::kVStages), (it / C::kVStages) & 1);
       }
     }
-    if (warp == 1 && n_iter > 0) {
+    if (warp == 1 && n_iter > 0 && rank == 0) {
       tc_fence_after();
       if (elect_one()) {
-        umma_commit(BAR(kBDrain));
+        if constexpr (CG2) umma_commit_pair(BAR(kBDrain), 1);  // this CTA's barrier only
+        else umma_commit(BAR(kBDrain));
         mbar_wait_limited(BAR(kBDrain), 0);
       }
       __syncwarp();
     }
+    if (CG2 && threadIdx.x == 0) {
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 50000) __nanosleep(1000);
+    }
     tc_fence_before();
     __syncthreads();
+    if constexpr (CG2) cluster_sync_all();
   }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
+    if constexpr (CG2) tmem_dealloc_pair(tmem, C::kTmemCols);
+    else tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
-template <int DQK, int DV, bool PAIRED>
+template <int DQK, int DV, bool PAIRED, bool CG2>
 static int launch_fwd_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
-  using C = FwdCfg<DQK, DV, PAIRED>;
+  using C = FwdCfg<DQK, DV, PAIRED, CG2>;
+  auto kern = sparse_fwd_kernel<DQK, DV, PAIRED, CG2>;
   static PerDeviceOnce attr;
-  const int rc = once_per_device(attr, [] {
-    return cuda_error(cudaFuncSetAttribute(sparse_fwd_kernel<DQK, DV, PAIRED>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem),
+  const int rc = once_per_device(attr, [&] {
+    return cuda_error(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           C::kSmem),
                       "forward smem attribute");
   });
   if (rc) return rc;
-  dim3 grid(a.Tm, a.HQ, a.B);
   record_event(0, st);
-  sparse_fwd_kernel<DQK, DV, PAIRED><<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.v, m.o, a);
-  record_event(1, st);
-  return check_launch("forward kernel launch");
+  if constexpr (CG2) {
+    // one 2-CTA cluster per (query tile, pair of query heads of one GQA group)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * a.Tm, a.HQ / 2, a.B);
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, m.q, m.k, m.kh, m.v, m.o, a);
+    record_event(1, st);
+    return cuda_error(e, "forward (CTA pair) kernel launch");
+  } else {
+    dim3 grid(a.Tm, a.HQ, a.B);
+    kern<<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.kh, m.v, m.o, a);
+    record_event(1, st);
+    return check_launch("forward kernel launch");
+  }
 }
 
 // Index mode pairs the softmax warps (its partial-tile bitmap masks make one softmax warp
 // per SM sub-partition issue bound); block and dense modes keep one (measured faster).
+// GQA with an even group size and Dv >= 128 can run on CTA pairs that share K and V:
+// by default only at head dims 256, where one CTA's forward is bound by shared-memory
+// operand reads that the pair halves; at 128 and 192/128 the softmax binds and the
+// pair's coupling made the forward slower (measured).
 template <int DQK, int DV>
 static int launch_fwd_dims(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
-  return a.mode == SA_MODE_INDEX ? launch_fwd_t<DQK, DV, true>(a, m, st)
-                                 : launch_fwd_t<DQK, DV, false>(a, m, st);
+  constexpr bool kPairable = DV >= 128;
+  constexpr bool kPairByDefault = DQK == 256;
+  const int pol = g_fwd_pairs.load(std::memory_order_relaxed);
+  const bool cg2 = kPairable && (a.HQ / a.HK) % 2 == 0 &&
+                   (pol == SA_FWD_PAIRS_ON || (pol == SA_FWD_PAIRS_AUTO && kPairByDefault));
+  if (a.mode == SA_MODE_INDEX)
+    return cg2 ? launch_fwd_t<DQK, DV, true, kPairable>(a, m, st)
+               : launch_fwd_t<DQK, DV, true, false>(a, m, st);
+  return cg2 ? launch_fwd_t<DQK, DV, false, kPairable>(a, m, st)
+             : launch_fwd_t<DQK, DV, false, false>(a, m, st);
 }
 
 int launch_fwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {

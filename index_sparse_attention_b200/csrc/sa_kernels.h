@@ -47,9 +47,12 @@ struct AttnArgs {
 
 // Wait limit for the next launches (0: the default); see sparse_attn_set_wait_limit_ns.
 extern std::atomic<uint64_t> g_wait_limit_ns;
+// Forward form for GQA (SA_FWD_PAIRS_*); see sparse_attn_set_forward_pairs.
+extern std::atomic<int> g_fwd_pairs;
 
 struct TensorMaps {
   CUtensorMap q, k, v, dout, dq_acc, dk, dv, o;
+  CUtensorMap kh;  // forward: K in 64-row boxes (the half tile of a CTA pair)
 };
 
 // Caller-owned events recorded around the launches (see sparse_attn_set_timing_events);

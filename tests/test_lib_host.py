@@ -98,3 +98,17 @@ def test_instrumentation_setters(lib):
     """The test-only knob: the wait limit of the bounded pipeline waits."""
     assert lib.sparse_attn_set_wait_limit_ns(1000) == _lib.SA_OK
     assert lib.sparse_attn_set_wait_limit_ns(0) == _lib.SA_OK
+
+
+def test_forward_pair_policy_setter(lib):
+    """The forward's GQA form: AUTO / ON / OFF are accepted, anything else is refused
+    with SA_ERR_INVALID; the binding maps the names and refuses unknown ones."""
+    import index_sparse_attention_b200 as sa
+    for code in (_lib.SA_FWD_PAIRS_ON, _lib.SA_FWD_PAIRS_OFF, _lib.SA_FWD_PAIRS_AUTO):
+        assert lib.sparse_attn_set_forward_pairs(code) == _lib.SA_OK
+    for bad in (-1, 3, 1 << 20):
+        assert lib.sparse_attn_set_forward_pairs(bad) == _lib.SA_ERR_INVALID
+    for name in ("on", "off", "auto"):
+        sa.sparse_attn_set_forward_pairs(name)
+    with pytest.raises(ValueError):
+        sa.sparse_attn_set_forward_pairs("sometimes")
