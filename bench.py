@@ -340,7 +340,7 @@ def run_gpu(args):
     from index_sparse_attention_b200 import _lib
 
     L = _lib.load()
-    sa.sparse_attn_set_forward_pairs(args.fwd_pairs)
+    sa.sparse_attn_set_forward_form(args.fwd_form)
     w = get_workload(args)
     inp = I.make_inputs(w)
     dev = torch.device("cuda", local)
@@ -520,7 +520,7 @@ def run_gpu(args):
             "data": "synthetic",
             "config": dict(workload_config(w, active),
                            **({"backward": "deterministic"} if args.deterministic else {}),
-                           **({"forward_pairs": args.fwd_pairs} if args.fwd_pairs != "auto"
+                           **({"forward_form": args.fwd_form} if args.fwd_form != "auto"
                               else {})),
             "pct_of_bf16_peak": 100.0 * (value / world) / peak,
             "pct_basis": (f"{peak_kind} {peak:.1f} TFLOP/s ({of}); burst unless the clock record "
@@ -738,9 +738,11 @@ def main():
                     help="use the deterministic backward (fixed-order dQ accumulation)")
     ap.add_argument("--heads", default="",
                     help="override the head counts as HQ,HK (e.g. 16,8: GQA on the D=256 workload)")
-    ap.add_argument("--fwd-pairs", default="auto", choices=["auto", "on", "off"],
-                    help="forward form for GQA: CTA pairs with cta_group::2 MMAs (on), one "
-                         "CTA per query tile and head (off), or the library's choice (auto)")
+    ap.add_argument("--fwd-form", default="auto",
+                    choices=["auto", "one_head", "cta_pair", "two_heads"],
+                    help="forward head-to-CTA form for GQA: one CTA per query tile and head, "
+                         "two heads on a 2-CTA pair with cta_group::2 MMAs, two heads per "
+                         "CTA, or the library's choice (auto)")
     ap.add_argument("--op", default="attention", choices=["attention", "topk", "index_stats"],
                     help="topk: time the top-k selector alone on one packed sequence; "
                          "index_stats: counts on an index workload (CPU only)")

@@ -232,27 +232,36 @@ int sparse_attn_set_timing_events(void *const *events);
  */
 int sparse_attn_set_wait_limit_ns(uint64_t ns);
 
-/* Policies of sparse_attn_set_forward_pairs. */
-#define SA_FWD_PAIRS_AUTO 0
-#define SA_FWD_PAIRS_ON 1
-#define SA_FWD_PAIRS_OFF 2
+/* Forms of sparse_attn_set_forward_form. */
+#define SA_FWD_FORM_AUTO 0
+#define SA_FWD_FORM_ONE_HEAD 1
+#define SA_FWD_FORM_CTA_PAIR 2
+#define SA_FWD_FORM_TWO_HEADS 3
 
 /*
- * sparse_attn_set_forward_pairs -- selects the form of the forward for GQA.  The pages
- * have 256-row tiles on SM100 (MagiAttention PR #331, "CSR Tile Mapping") and a switch
- * that turns the 2-CTA mode off (MagiAttention PR #334, section 3, disable_2cta); the
- * pair form here is this library's own.  The query heads of one GQA group walk the same tile
- * list, so with an even group size and Dv >= 128 the forward can run two of them (same
- * query tile) on a pair of CTAs: a 2-CTA cluster whose tensor-core MMAs span both CTAs
- * (tcgen05 cta_group::2, M = 256) and which split every K and V tile between them.
- *   SA_FWD_PAIRS_AUTO  the pair form where it is measured faster (Dqk = Dv = 256);
- *   SA_FWD_PAIRS_ON    the pair form wherever it applies;
- *   SA_FWD_PAIRS_OFF   one CTA per (query tile, query head) always.
- * Both forms compute the same O and LSE up to fp32 rounding.  Applies to the forward
- * calls enqueued after it; process-wide.  Returns SA_OK, or SA_ERR_INVALID for another
- * value (the setting is then unchanged).
+ * sparse_attn_set_forward_form -- selects how the forward maps query heads to CTAs.  The
+ * pages pick the number of query tiles per CTA ("q_stage", sgl-flash-attn PR #28, "determine
+ * q_stage via seqlen_q for sm100"), have 256-row tiles on SM100 (MagiAttention PR #331,
+ * "CSR Tile Mapping") and a switch that turns the 2-CTA mode off (MagiAttention PR #334,
+ * section 3, disable_2cta); the forms here are this library's own.  The query heads of
+ * one GQA group walk the same tile list, so with an even group size two of them (same
+ * query tile) can share every K and V tile:
+ *   SA_FWD_FORM_ONE_HEAD   one CTA per (query tile, query head);
+ *   SA_FWD_FORM_CTA_PAIR   two heads on a 2-CTA cluster whose tensor-core MMAs span both
+ *                          CTAs (tcgen05 cta_group::2, M = 256); each CTA holds half of
+ *                          every K and V tile (needs Dv >= 128);
+ *   SA_FWD_FORM_TWO_HEADS  two heads in one CTA, each with its own S and O in tensor
+ *                          memory and its own softmax warps, so that one head's softmax
+ *                          overlaps the other head's MMAs (needs Dqk <= 192, Dv <= 128);
+ *   SA_FWD_FORM_AUTO       the library's choice (measured): CTA pairs at head dims 256,
+ *                          two heads per CTA in block and dense modes at Dqk <= 128, one
+ *                          head per CTA otherwise (MHA, an odd group size, index mode).
+ * A form that does not apply to a call falls back to one head per CTA.  All forms compute
+ * the same O and LSE up to fp32 rounding.  Applies to the forward calls enqueued after it;
+ * process-wide.  Returns SA_OK, or SA_ERR_INVALID for another value (the setting is then
+ * unchanged).
  */
-int sparse_attn_set_forward_pairs(int policy);
+int sparse_attn_set_forward_form(int form);
 
 
 /* Largest k that topk_select supports. */

@@ -17,7 +17,7 @@ from ._lib import SA_MODE_BLOCK, SA_MODE_DENSE, SA_MODE_INDEX, SA_TILE, SparseAt
 __all__ = ["BlockSparse", "block_mask_to_block_sparse", "index_to_block_sparse",
            "sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_bwd_workspace_size",
            "sparse_attn_bwd_noalloc", "topk_select", "sparse_attn_set_wait_limit_ns",
-           "sparse_attn_set_forward_pairs",
+           "sparse_attn_set_forward_form",
            "SparseAttnError", "SA_TILE"]
 
 
@@ -304,16 +304,18 @@ def sparse_attn_set_wait_limit_ns(ns):
     _lib.check("sparse_attn_set_wait_limit_ns", _lib.load().sparse_attn_set_wait_limit_ns(int(ns)))
 
 
-_FWD_PAIRS = {"auto": _lib.SA_FWD_PAIRS_AUTO, "on": _lib.SA_FWD_PAIRS_ON,
-              "off": _lib.SA_FWD_PAIRS_OFF}
+_FWD_FORMS = {"auto": _lib.SA_FWD_FORM_AUTO, "one_head": _lib.SA_FWD_FORM_ONE_HEAD,
+              "cta_pair": _lib.SA_FWD_FORM_CTA_PAIR, "two_heads": _lib.SA_FWD_FORM_TWO_HEADS}
 
 
-def sparse_attn_set_forward_pairs(policy):
-    """The forward's form for GQA: "auto" (the library's choice: CTA pairs sharing K/V
-    tiles through cta_group::2 MMAs at head dims 256), "on" (pairs wherever the group
-    size is even and Dv >= 128) or "off" (one CTA per query tile and head).  Applies to
-    the forward calls made after it, process-wide; see include/sparse_attn.h."""
-    code = _FWD_PAIRS.get(policy, policy) if isinstance(policy, str) else int(policy)
+def sparse_attn_set_forward_form(form):
+    """How the forward maps query heads to CTAs: "auto" (the library's choice), "one_head"
+    (one CTA per query tile and head), "cta_pair" (two heads of a GQA group on a 2-CTA
+    cluster with cta_group::2 MMAs sharing each K/V tile) or "two_heads" (two heads of a
+    group in one CTA, one softmax warpgroup each).  A form that does not apply to a call
+    falls back to one head per CTA.  Applies to the forward calls made after it,
+    process-wide; see include/sparse_attn.h."""
+    code = _FWD_FORMS.get(form, form) if isinstance(form, str) else int(form)
     if isinstance(code, str):
-        raise ValueError(f"policy must be one of {sorted(_FWD_PAIRS)}, got {policy!r}")
-    _lib.check("sparse_attn_set_forward_pairs", _lib.load().sparse_attn_set_forward_pairs(code))
+        raise ValueError(f"form must be one of {sorted(_FWD_FORMS)}, got {form!r}")
+    _lib.check("sparse_attn_set_forward_form", _lib.load().sparse_attn_set_forward_form(code))

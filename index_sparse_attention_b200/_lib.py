@@ -24,7 +24,7 @@ SA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 SA_TOPK_MAX_K = 4096
 
 SA_MODE_DENSE, SA_MODE_BLOCK, SA_MODE_INDEX = 0, 1, 2
-SA_FWD_PAIRS_AUTO, SA_FWD_PAIRS_ON, SA_FWD_PAIRS_OFF = 0, 1, 2
+SA_FWD_FORM_AUTO, SA_FWD_FORM_ONE_HEAD, SA_FWD_FORM_CTA_PAIR, SA_FWD_FORM_TWO_HEADS = 0, 1, 2, 3
 SA_TILE = 128
 
 STATUS_INDEX = 1
@@ -41,7 +41,7 @@ EXPORTS = (
     "sparse_attn_bwd_noalloc",
     "sparse_attn_set_timing_events",
     "sparse_attn_set_wait_limit_ns",
-    "sparse_attn_set_forward_pairs",
+    "sparse_attn_set_forward_form",
     "sparse_attn_error_string",
     "topk_select",
 )
@@ -100,8 +100,8 @@ def load():
     L.sparse_attn_set_timing_events.restype = ctypes.c_int
     L.sparse_attn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     L.sparse_attn_set_wait_limit_ns.restype = ctypes.c_int
-    L.sparse_attn_set_forward_pairs.argtypes = [ctypes.c_int]
-    L.sparse_attn_set_forward_pairs.restype = ctypes.c_int
+    L.sparse_attn_set_forward_form.argtypes = [ctypes.c_int]
+    L.sparse_attn_set_forward_form.restype = ctypes.c_int
     i64 = ctypes.c_int64
     L.topk_select.argtypes = [vp, i64, i64, i64, vp, vp, ctypes.c_int32, vp, vp, vp, vp]
     L.topk_select.restype = ctypes.c_int

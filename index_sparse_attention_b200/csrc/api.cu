@@ -22,7 +22,7 @@ int cuda_error(cudaError_t e, const char* what) {
 cudaEvent_t* g_timing_events = nullptr;
 static cudaEvent_t g_events_copy[6];
 std::atomic<uint64_t> g_wait_limit_ns{0};
-std::atomic<int> g_fwd_pairs{SA_FWD_PAIRS_AUTO};
+std::atomic<int> g_fwd_form{SA_FWD_FORM_AUTO};
 }  // namespace sa
 
 namespace {
@@ -199,10 +199,9 @@ extern "C" int sparse_attn_set_wait_limit_ns(uint64_t ns) {
   return SA_OK;
 }
 
-extern "C" int sparse_attn_set_forward_pairs(int policy) {
-  if (policy != SA_FWD_PAIRS_AUTO && policy != SA_FWD_PAIRS_ON && policy != SA_FWD_PAIRS_OFF)
-    return SA_ERR_INVALID;
-  g_fwd_pairs.store(policy, std::memory_order_relaxed);
+extern "C" int sparse_attn_set_forward_form(int form) {
+  if (form < SA_FWD_FORM_AUTO || form > SA_FWD_FORM_TWO_HEADS) return SA_ERR_INVALID;
+  g_fwd_form.store(form, std::memory_order_relaxed);
   return SA_OK;
 }
 

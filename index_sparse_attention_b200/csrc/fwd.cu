@@ -46,9 +46,10 @@
 
 namespace sa {
 
-template <int DQK, int DV, bool PAIRED, bool CG2>
+template <int DQK, int DV, bool PAIRED, bool CG2, bool QS2>
 struct FwdCfg {
   static constexpr int kPanel = 128 * 128;  // one 64-column x 128-row swizzled panel
+  static constexpr int kHeads = QS2 ? 2 : 1;  // query heads per CTA
   // K rows and V columns one CTA holds per tile (a pair splits both in halves)
   static constexpr int kKRows = CG2 ? 64 : 128;
   static constexpr int kKPanel = kKRows * 128;  // one 64-column panel of K
@@ -56,48 +57,51 @@ struct FwdCfg {
   static constexpr int kQBytes = 128 * DQK * 2;
   static constexpr int kKBytes = kKRows * DQK * 2;
   static constexpr int kVBytes = 128 * kVCols * 2;
-  static constexpr int kKStages = CG2 ? (DQK == 256 ? 2 : 3) : (DQK == 256 ? 1 : 2);
-  static constexpr int kVStages = CG2 ? (DV == 256 ? 2 : 3) : (DV == 256 ? 1 : 2);
-  static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kQBytes;
+  static constexpr int kKStages = QS2 ? 2 : CG2 ? (DQK == 256 ? 2 : 3) : (DQK == 256 ? 1 : 2);
+  static constexpr int kVStages =
+      QS2 ? (DQK == 192 ? 1 : 2) : CG2 ? (DV == 256 ? 2 : 3) : (DV == 256 ? 1 : 2);
+  static constexpr int kQOff = 0;  // kHeads Q tiles
+  static constexpr int kKOff = kQOff + kHeads * kQBytes;
   static constexpr int kVOff = kKOff + kKStages * kKBytes;
   static constexpr int kBarOff = kVOff + kVStages * kVBytes;
-  // softmax exchange: row max [2 tile parities][2 column halves][128 rows] and row sum
-  // [2 halves][128 rows], fp32
+  // softmax exchange of the paired warps: row max [2 tile parities][2 column halves][128
+  // rows] and row sum [2 halves][128 rows], fp32
   static constexpr int kXOff = kBarOff + 256;
-  static constexpr int kSmem = kXOff + 3 * 1024 + 1024;  // + alignment slack
+  static constexpr int kSmem = kXOff + (PAIRED ? 3 * 1024 : 0) + 1024;  // + alignment slack
   // softmax warps per TMEM lane quarter (PAIRED: two, each with half of every row)
   static constexpr int kHalves = PAIRED ? 2 : 1;
-  static constexpr int kThreads = PAIRED ? 352 : 224;
-  static constexpr int kVWarp = PAIRED ? 10 : 6;  // V producer
+  static constexpr int kThreads = QS2 ? 320 : PAIRED ? 352 : 224;
+  static constexpr int kVWarp = QS2 ? -1 : PAIRED ? 10 : 6;  // V producer (QS2: warp 0)
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kOCol = 256;
   // Dqk <= 192: Q is held in TMEM after O (bf16 pairs) and S = Q K^T reads it from there,
   // so that only K is read from shared memory (an operand pair from shared memory costs
   // 8 KB per 64-cycle k-step, the whole port, before the TMA writes of K and V)
-  static constexpr bool kQT = DQK <= 192;
+  static constexpr bool kQT = !QS2 && DQK <= 192;
   static constexpr uint32_t kColQ = kOCol + DV;
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
   static_assert(kOCol + DV <= kTmemCols, "tensor memory budget");
   static_assert(!kQT || kColQ + DQK / 2 <= kTmemCols, "tensor memory budget (Q)");
   static_assert(!CG2 || DV >= 128, "a CTA pair splits V into 64-column panels");
+  static_assert(!QS2 || (!PAIRED && !CG2 && DQK <= 192), "two heads per CTA: full rows, one CTA");
+  static_assert(kOCol + kHeads * DV <= kTmemCols, "tensor memory budget (two heads)");
   static_assert(kKStages <= 4 && kVStages <= 4, "barrier slots");
 };
 
-// barrier slots (up to four K and four V stages)
+// barrier slots (up to four K and four V stages; kBOD2 / kBOFin2: the second head's)
 enum : int { kBQ = 0, kBKF = 1, kBKE = 5, kBVF = 9, kBVE = 13, kBSF = 17, kBPF = 19, kBOD = 21,
-             kBDrain = 22, kBOFin = 23, kBQT = 24, kNumBars = 25 };
+             kBDrain = 22, kBOFin = 23, kBQT = 24, kBOD2 = 25, kBOFin2 = 26, kNumBars = 27 };
 
 // tm_kh: K in 64-row boxes (the half tile a CTA of a pair loads); unused by the
 // single-CTA form.
-template <int DQK, int DV, bool PAIRED, bool CG2>
-__global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
+template <int DQK, int DV, bool PAIRED, bool CG2, bool QS2, bool PREFETCH>
+__global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
     sparse_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_kh,
                       const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_o, const AttnArgs a) {
-  using C = FwdCfg<DQK, DV, PAIRED, CG2>;
+  using C = FwdCfg<DQK, DV, PAIRED, CG2, QS2>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -113,8 +117,9 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
   const uint32_t rank = CG2 ? cluster_ctarank() : 0u;
   const int xt = CG2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int mt = a.Tm - 1 - xt;  // longest lists first under causal
-  const int h = CG2 ? 2 * static_cast<int>(blockIdx.y) + static_cast<int>(rank)
-                    : static_cast<int>(blockIdx.y);
+  // (QS2: h is the first of the CTA's two heads, h + 1 the second)
+  const int h = (CG2 || QS2) ? 2 * static_cast<int>(blockIdx.y) + static_cast<int>(rank)
+                             : static_cast<int>(blockIdx.y);
   const int b = blockIdx.z;
   // the leader's barriers as seen from this CTA (remote arrivals and pair loads)
   const uint32_t lbar0 = CG2 ? mapa_shared(bar0, 0) : bar0;
@@ -147,6 +152,8 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
     mbar_init(BAR(kBDrain), 1);
     mbar_init(BAR(kBOFin), 1);
     mbar_init(BAR(kBQT), kReadyCount);
+    mbar_init(BAR(kBOD2), 1);
+    mbar_init(BAR(kBOFin2), 1);
     abort_flag->abort = 0;
     abort_flag->peer_abort = 0;
     fence_mbar_init();
@@ -183,12 +190,30 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
             tma_load_4d_pair(sbase + C::kQOff + c * C::kPanel, &tm_q, LBAR(kBQ), c * 64, mt * 128,
                              h, b);
         } else {
-          mbar_arrive_expect_tx(BAR(kBQ), C::kQBytes);
-          for (int c = 0; c < DQK / 64; ++c)
-            tma_load_4d(sbase + C::kQOff + c * C::kPanel, &tm_q, BAR(kBQ), c * 64, mt * 128, h, b);
+          // (QS2: the tiles of heads h and h + 1, one after the other)
+          mbar_arrive_expect_tx(BAR(kBQ), C::kHeads * C::kQBytes);
+          for (int hd = 0; hd < C::kHeads; ++hd)
+            for (int c = 0; c < DQK / 64; ++c)
+              tma_load_4d(sbase + C::kQOff + hd * C::kQBytes + c * C::kPanel, &tm_q, BAR(kBQ),
+                          c * 64, mt * 128, h + hd, b);
         }
       }
       __syncwarp();
+      auto load_v = [&](int t) -> bool {  // V tile t (QS2)
+        const int nt = __shfl_sync(0xFFFFFFFFu, __ldg(list + t), 0);
+        const int vs = t % C::kVStages, vu = t / C::kVStages;
+        if (!warp_wait(BAR(kBVE + vs), (vu & 1) ^ 1, abort_flag, a.status, a.wait_limit_ns))
+          return false;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(BAR(kBVF + vs), C::kVBytes);
+          for (int c = 0; c < DV / 64; ++c)
+            tma_load_4d(sbase + C::kVOff + vs * C::kVBytes + c * C::kPanel, &tm_v, BAR(kBVF + vs),
+                        c * 64, nt * 128, g, b);
+        }
+        __syncwarp();
+        issued_v = t + 1;
+        return true;
+      };
       // K tiles: each one as soon as S of the tile that last used its buffer is done (V
       // tiles have a producer warp of their own, so a K load never waits behind P V)
       for (int it = 0; it < n_iter; ++it) {
@@ -210,7 +235,12 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
         }
         __syncwarp();
         issued_k = it + 1;
+        // QS2: V tiles from this warp too, one tile behind K (V(it-1) after K(it)): a K
+        // stage frees when S of the second head is done, a V stage only when its P V is,
+        // later in the tensor pipe's order, so K never waits behind a V stage
+        if (QS2 && it > 0 && !load_v(it - 1)) break;
       }
+      if (QS2 && issued_k == n_iter) load_v(n_iter - 1);
       // pair: the leader's commits arrive on this CTA's barriers too; wait for the ones
       // that free the last stages so that none is in flight when the CTA leaves
       if (CG2 && issued_k == n_iter)
@@ -254,72 +284,129 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
     // The whole warp runs this loop (converged, warp-uniform operands); one elected
     // lane issues each batch of tcgen05 instructions.  In a pair only the leader issues
     // (M = 256: both CTAs' rows), and every commit arrives on both CTAs' barriers.
-    if (n_iter > 0 && rank == 0) {
-      constexpr int kM = CG2 ? 256 : 128;
-      constexpr uint32_t idesc_qk = idesc_bf16(kM, 128, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16(kM, DV, 0, 1);
-      const uint64_t qdesc = sw128_desc(sbase + C::kQOff, 16, 1024);
-      auto commit = [&](int bar) {
-        if constexpr (CG2) umma_commit_pair(BAR(bar), 3);
-        else umma_commit(BAR(bar));
-      };
-      // Q in TMEM (kQT): the softmax warps have copied it there
-      bool ok = warp_wait(BAR(C::kQT ? kBQT : kBQ), 0, abort_flag, a.status, a.wait_limit_ns);
-      auto issue_s = [&](int it) -> bool {
-        const int ks = it % C::kKStages, ku = it / C::kKStages;
-        if (!warp_wait(BAR(kBKF + ks), ku & 1, abort_flag, a.status, a.wait_limit_ns)) return false;
-        tc_fence_after();
-        const uint64_t kdesc = sw128_desc(sbase + C::kKOff + ks * C::kKBytes, 16, 1024);
-        const uint32_t d = tmem + static_cast<uint32_t>((it & 1) * 128);
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < DQK / 16; ++kk) {
-            const uint32_t qoff = ((kk >> 2) * C::kPanel + (kk & 3) * 32) >> 4;
-            const uint32_t koff = ((kk >> 2) * C::kKPanel + (kk & 3) * 32) >> 4;
-            if constexpr (C::kQT) {  // A = Q from TMEM: 16 head dims = 8 columns per k-step
-              if constexpr (CG2)
-                umma_ts_pair(d, tmem + C::kColQ + kk * 8, kdesc + koff, idesc_qk, kk > 0 ? 1u : 0u);
-              else
-                umma_ts(d, tmem + C::kColQ + kk * 8, kdesc + koff, idesc_qk, kk > 0 ? 1u : 0u);
-            } else {
-              if constexpr (CG2)
-                umma_ss_pair(d, qdesc + qoff, kdesc + koff, idesc_qk, kk > 0 ? 1u : 0u);
-              else
-                umma_ss(d, qdesc + qoff, kdesc + koff, idesc_qk, kk > 0 ? 1u : 0u);
+    if constexpr (QS2) {
+      if (n_iter > 0) {
+        // Two heads (A = h, B = h + 1): S_A(j), S_B(j) into each head's 128-column buffer,
+        // P V into O_A, O_B.  Per key tile j: P V of head A once its P is ready, then
+        // S_A(j+1) into the same buffer (the pipe runs in order, so P is read before it is
+        // overwritten), then the same for head B.  While one head's softmax works on its S,
+        // the tensor pipe runs the other head's MMAs.
+        constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0, 0);
+        constexpr uint32_t idesc_pv = idesc_bf16(128, DV, 0, 1);
+        bool ok = warp_wait(BAR(kBQ), 0, abort_flag, a.status, a.wait_limit_ns);
+        auto issue_s2 = [&](int it, int hd) -> bool {
+          const int ks = it % C::kKStages, ku = it / C::kKStages;
+          if (hd == 0 && !warp_wait(BAR(kBKF + ks), ku & 1, abort_flag, a.status, a.wait_limit_ns))
+            return false;
+          tc_fence_after();
+          const uint64_t kdesc = sw128_desc(sbase + C::kKOff + ks * C::kKBytes, 16, 1024);
+          const uint64_t qd = sw128_desc(sbase + C::kQOff + hd * C::kQBytes, 16, 1024);
+          const uint32_t d = tmem + static_cast<uint32_t>(hd * 128);
+          if (elect_one()) {
+  #pragma unroll
+            for (int kk = 0; kk < DQK / 16; ++kk) {
+              const uint32_t off = ((kk >> 2) * C::kPanel + (kk & 3) * 32) >> 4;
+              umma_ss(d, qd + off, kdesc + off, idesc_qk, kk > 0 ? 1u : 0u);
             }
+            umma_commit(BAR(kBSF + hd));
+            if (hd == 1) umma_commit(BAR(kBKE + ks));  // both heads have read the K tile
           }
-          commit(kBSF + (it & 1));
-          commit(kBKE + ks);
-        }
-        __syncwarp();
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      for (int it = 0; ok && it < n_iter; ++it) {
-        if (it + 1 < n_iter && !issue_s(it + 1)) break;
-        const int vs = it % C::kVStages, vu = it / C::kVStages;
-        if (!warp_wait(BAR(kBPF + (it & 1)), (it >> 1) & 1, abort_flag, a.status, a.wait_limit_ns)) break;
-        if (!warp_wait(BAR(kBVF + vs), vu & 1, abort_flag, a.status, a.wait_limit_ns)) break;
-        tc_fence_after();
-        const uint64_t vdesc = sw128_desc(sbase + C::kVOff + vs * C::kVBytes, C::kPanel, 1024);
-        const uint32_t pa = tmem + static_cast<uint32_t>((it & 1) * 128);
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk) {
-            if constexpr (CG2)
-              umma_ts_pair(tmem + C::kOCol, pa + kk * 8, vdesc + ((kk * 2048) >> 4), idesc_pv,
-                           (it > 0 || kk > 0) ? 1u : 0u);
-            else
-              umma_ts(tmem + C::kOCol, pa + kk * 8, vdesc + ((kk * 2048) >> 4), idesc_pv,
+          __syncwarp();
+          return true;
+        };
+        auto issue_pv2 = [&](int it, int hd) -> bool {
+          const int vs = it % C::kVStages, vu = it / C::kVStages;
+          if (!warp_wait(BAR(kBPF + hd), it & 1, abort_flag, a.status, a.wait_limit_ns)) return false;
+          if (hd == 0 && !warp_wait(BAR(kBVF + vs), vu & 1, abort_flag, a.status, a.wait_limit_ns))
+            return false;
+          tc_fence_after();
+          const uint64_t vdesc = sw128_desc(sbase + C::kVOff + vs * C::kVBytes, C::kPanel, 1024);
+          const uint32_t pa = tmem + static_cast<uint32_t>(hd * 128);
+          if (elect_one()) {
+  #pragma unroll
+            for (int kk = 0; kk < 128 / 16; ++kk)
+              umma_ts(tmem + C::kOCol + hd * DV, pa + kk * 8, vdesc + ((kk * 2048) >> 4), idesc_pv,
                       (it > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(BAR(hd ? kBOD2 : kBOD));
+            if (hd == 1) umma_commit(BAR(kBVE + vs));  // both heads have read the V tile
+            if (it == n_iter - 1) umma_commit(BAR(hd ? kBOFin2 : kBOFin));
           }
-          // (pair: no O-done arrival after the last P V, which nobody waits for: every
-          // arrival on the other CTA's barriers is observed before it leaves)
-          if (!CG2 || it < n_iter - 1) commit(kBOD);
-          commit(kBVE + vs);
-          if (it == n_iter - 1) commit(kBOFin);  // the final O is complete
+          __syncwarp();
+          return true;
+        };
+        if (ok) ok = issue_s2(0, 0) && issue_s2(0, 1);
+        for (int it = 0; ok && it < n_iter; ++it)
+          for (int hd = 0; ok && hd < 2; ++hd)
+            ok = issue_pv2(it, hd) && (it + 1 >= n_iter || issue_s2(it + 1, hd));
+      }
+    } else {
+      if (n_iter > 0 && rank == 0) {
+        constexpr int kM = CG2 ? 256 : 128;
+        constexpr uint32_t idesc_qk = idesc_bf16(kM, 128, 0, 0);
+        constexpr uint32_t idesc_pv = idesc_bf16(kM, DV, 0, 1);
+        const uint64_t qdesc = sw128_desc(sbase + C::kQOff, 16, 1024);
+        auto commit = [&](int bar) {
+          if constexpr (CG2) umma_commit_pair(BAR(bar), 3);
+          else umma_commit(BAR(bar));
+        };
+        // Q in TMEM (kQT): the softmax warps have copied it there
+        bool ok = warp_wait(BAR(C::kQT ? kBQT : kBQ), 0, abort_flag, a.status, a.wait_limit_ns);
+        auto issue_s = [&](int it) -> bool {
+          const int ks = it % C::kKStages, ku = it / C::kKStages;
+          if (!warp_wait(BAR(kBKF + ks), ku & 1, abort_flag, a.status, a.wait_limit_ns)) return false;
+          tc_fence_after();
+          const uint64_t kdesc = sw128_desc(sbase + C::kKOff + ks * C::kKBytes, 16, 1024);
+          const uint32_t d = tmem + static_cast<uint32_t>((it & 1) * 128);
+          if (elect_one()) {
+  #pragma unroll
+            for (int kk = 0; kk < DQK / 16; ++kk) {
+              const uint32_t qoff = ((kk >> 2) * C::kPanel + (kk & 3) * 32) >> 4;
+              const uint32_t koff = ((kk >> 2) * C::kKPanel + (kk & 3) * 32) >> 4;
+              if constexpr (C::kQT) {  // A = Q from TMEM: 16 head dims = 8 columns per k-step
+                if constexpr (CG2)
+                  umma_ts_pair(d, tmem + C::kColQ + kk * 8, kdesc + koff, idesc_qk, kk > 0 ? 1u : 0u);
+                else
+                  umma_ts(d, tmem + C::kColQ + kk * 8, kdesc + koff, idesc_qk, kk > 0 ? 1u : 0u);
+              } else {
+                if constexpr (CG2)
+                  umma_ss_pair(d, qdesc + qoff, kdesc + koff, idesc_qk, kk > 0 ? 1u : 0u);
+                else
+                  umma_ss(d, qdesc + qoff, kdesc + koff, idesc_qk, kk > 0 ? 1u : 0u);
+              }
+            }
+            commit(kBSF + (it & 1));
+            commit(kBKE + ks);
+          }
+          __syncwarp();
+          return true;
+        };
+        if (ok) ok = issue_s(0);
+        for (int it = 0; ok && it < n_iter; ++it) {
+          if (it + 1 < n_iter && !issue_s(it + 1)) break;
+          const int vs = it % C::kVStages, vu = it / C::kVStages;
+          if (!warp_wait(BAR(kBPF + (it & 1)), (it >> 1) & 1, abort_flag, a.status, a.wait_limit_ns)) break;
+          if (!warp_wait(BAR(kBVF + vs), vu & 1, abort_flag, a.status, a.wait_limit_ns)) break;
+          tc_fence_after();
+          const uint64_t vdesc = sw128_desc(sbase + C::kVOff + vs * C::kVBytes, C::kPanel, 1024);
+          const uint32_t pa = tmem + static_cast<uint32_t>((it & 1) * 128);
+          if (elect_one()) {
+  #pragma unroll
+            for (int kk = 0; kk < 128 / 16; ++kk) {
+              if constexpr (CG2)
+                umma_ts_pair(tmem + C::kOCol, pa + kk * 8, vdesc + ((kk * 2048) >> 4), idesc_pv,
+                             (it > 0 || kk > 0) ? 1u : 0u);
+              else
+                umma_ts(tmem + C::kOCol, pa + kk * 8, vdesc + ((kk * 2048) >> 4), idesc_pv,
+                        (it > 0 || kk > 0) ? 1u : 0u);
+            }
+            // (pair: no O-done arrival after the last P V, which nobody waits for: every
+            // arrival on the other CTA's barriers is observed before it leaves)
+            if (!CG2 || it < n_iter - 1) commit(kBOD);
+            commit(kBVE + vs);
+            if (it == n_iter - 1) commit(kBOFin);  // the final O is complete
+          }
+          __syncwarp();
         }
-        __syncwarp();
       }
     }
   } else {
@@ -337,6 +424,12 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
     constexpr int kOCols = DV / kH;                  // O columns rescaled / stored per thread
     const int quarter = warp & 3;
     const int hc = kH == 2 ? (warp - 2) >> 2 : 0;   // column part of this warp
+    // QS2: warps 2-5 hold head h, warps 6-9 head h + 1, each with its own S buffer, O
+    // accumulator and barriers
+    const int hd = QS2 ? (warp - 2) >> 2 : 0;
+    const int hh = h + hd;                           // this warp's query head
+    const uint32_t ocol = C::kOCol + static_cast<uint32_t>(hd * DV);
+    const int bar_od = hd ? kBOD2 : kBOD, bar_ofin = hd ? kBOFin2 : kBOFin;
     const int pair_bar = 1 + ((warp - 2) & 3);       // named barrier of a pair (64 threads)
     auto pair_all = [&](bool v) {                    // v: already uniform over the warp
       if constexpr (kH == 2) return named_bar_and(pair_bar, 64, v);
@@ -395,7 +488,7 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
     // Block and dense modes mask only the diagonal tile (or a ragged edge); there the
     // loads stay inline, because the prefetch's per-tile instructions cost the issue-bound
     // softmax warp more than it saves (+3 to +4% measured).
-    constexpr bool kPrefetch = PAIRED;  // the index-mode instance
+    constexpr bool kPrefetch = PREFETCH;  // the index-mode instances
     constexpr int kWords = kCols / 32;
     auto fetch_nt = [&](int t) {
       return (kPrefetch && t < n_iter && t >= n_full) ? __ldg(list + t) : 0;
@@ -427,13 +520,16 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
     bool m0_cur, m1_cur;
     fetch_mask(0, nt_cur, wd_cur, m0_cur, m1_cur);
     for (int it = 0; ok && it < n_iter; ++it) {
-      const int sb = it & 1;
+      // S / P buffer of this tile and the parity of its S-ready phase (QS2: the head's
+      // single buffer, one phase per tile)
+      const int sb = QS2 ? hd : (it & 1);
+      const uint32_t s_par = QS2 ? (it & 1) : ((it >> 1) & 1);
       const int nt_nn = fetch_nt(it + 2);
       uint32_t wd_nxt[kWords];
       bool m0_nxt, m1_nxt;
       fetch_mask(it + 1, nt_nxt, wd_nxt, m0_nxt, m1_nxt);
       const bool w_ok = __all_sync(
-          0xFFFFFFFFu, mbar_wait(BAR(kBSF + sb), (it >> 1) & 1, abort_flag, a.status, a.wait_limit_ns));
+          0xFFFFFFFFu, mbar_wait(BAR(kBSF + sb), s_par, abort_flag, a.status, a.wait_limit_ns));
       if (!pair_all(w_ok)) {
         ok = false;
         break;
@@ -501,7 +597,7 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
           // O holds P V up to tile it-1: rescale this thread's O columns in TMEM once
           // that MMA is done
           const bool o_ok = __all_sync(
-              0xFFFFFFFFu, mbar_wait(BAR(kBOD), (it - 1) & 1, abort_flag, a.status, a.wait_limit_ns));
+              0xFFFFFFFFu, mbar_wait(BAR(bar_od), (it - 1) & 1, abort_flag, a.status, a.wait_limit_ns));
           if (!pair_all(o_ok)) {
             ok = false;
             break;
@@ -510,11 +606,11 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
 #pragma unroll 1
           for (int c = hc * kOCols; c < (hc + 1) * kOCols; c += 32) {
             uint32_t ov[32];
-            tmem_ld32(tl + C::kOCol + c, ov);
+            tmem_ld32(tl + ocol + c, ov);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(tl + C::kOCol + c, ov);
+            tmem_st32(tl + ocol + c, ov);
           }
           tmem_wait_st();
         }
@@ -547,7 +643,7 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
     // ---------------------------------------------------------------- epilogue
     if (n_iter > 0 && ok) {
       const bool w_ok = __all_sync(
-          0xFFFFFFFFu, mbar_wait(BAR(kBOFin), 0, abort_flag, a.status, a.wait_limit_ns));
+          0xFFFFFFFFu, mbar_wait(BAR(bar_ofin), 0, abort_flag, a.status, a.wait_limit_ns));
       ok = pair_all(w_ok);
       tc_fence_after();
     }
@@ -566,7 +662,7 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
     for (int c = hc * kOCols; c < (hc + 1) * kOCols; c += 32) {
       uint32_t ov[32];
       if (have_o) {
-        tmem_ld32(tl + C::kOCol + c, ov);
+        tmem_ld32(tl + ocol + c, ov);
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -577,7 +673,7 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
       for (int e = 0; e < 16; ++e)
         pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
       // columns [c, c+32) = 16-byte chunks (c % 64) / 8 .. +3 of row r in panel c / 64
-      uint8_t* prow = smem + C::kQOff + (c >> 6) * C::kPanel + r * 128;
+      uint8_t* prow = smem + C::kQOff + hd * C::kQBytes + (c >> 6) * C::kPanel + r * 128;
       const int ch0 = (c & 63) >> 3;
 #pragma unroll
       for (int e = 0; e < 4; ++e)
@@ -585,17 +681,18 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
             make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
     }
     fence_proxy_async_smem();
-    named_bar_sync(5, 128 * kH);  // every softmax warp
-    if (threadIdx.x == 64) {
+    named_bar_sync(5 + hd, 128 * kH);  // every softmax warp (of this head)
+    if (threadIdx.x == 64 + 128 * hd) {
 #pragma unroll
       for (int p = 0; p < DV / 64; ++p)
-        tma_store_4d(&tm_o, sbase + C::kQOff + p * C::kPanel, p * 64, mt * 128, h, b);
+        tma_store_4d(&tm_o, sbase + C::kQOff + hd * C::kQBytes + p * C::kPanel, p * 64, mt * 128,
+                     hh, b);
       bulk_commit_group();
       bulk_wait_group_read0();  // the Q buffer is read before the CTA may leave
     }
     if (row_ok && hc == 0) {
       const float m_eff = (m_run == -INFINITY) ? 0.f : m_run;
-      a.lse[(static_cast<int64_t>(b) * a.HQ + h) * a.Sq + i] =
+      a.lse[(static_cast<int64_t>(b) * a.HQ + hh) * a.Sq + i] =
           (l_row > 0.f) ? (m_eff + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
     }
   }
@@ -632,6 +729,9 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
         mbar_wait_limited(BAR(kBQ), 0);
         for (int it = max(0, issued_k - C::kKStages); it < issued_k; ++it)
           mbar_wait_limited(BAR(kBKF + it % C::kKStages), (it / C::kKStages) & 1);
+        if constexpr (QS2)  // this warp loads V too
+          for (int it = max(0, issued_v - C::kVStages); it < issued_v; ++it)
+            mbar_wait_limited(BAR(kBVF + it % C::kVStages), (it / C::kVStages) & 1);
       } else if (warp == C::kVWarp) {
         for (int it = max(0, issued_v - C::kVStages); it < issued_v; ++it)
           mbar_wait_limited(BAR(kBVF + it % C::kVStages), (it / C::kVStages) & 1);
@@ -661,10 +761,10 @@ __global__ void __launch_bounds__(PAIRED ? 352 : 224, 1)
   }
 }
 
-template <int DQK, int DV, bool PAIRED, bool CG2>
+template <int DQK, int DV, bool PAIRED, bool CG2, bool QS2, bool PREFETCH>
 static int launch_fwd_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
-  using C = FwdCfg<DQK, DV, PAIRED, CG2>;
-  auto kern = sparse_fwd_kernel<DQK, DV, PAIRED, CG2>;
+  using C = FwdCfg<DQK, DV, PAIRED, CG2, QS2>;
+  auto kern = sparse_fwd_kernel<DQK, DV, PAIRED, CG2, QS2, PREFETCH>;
   static PerDeviceOnce attr;
   const int rc = once_per_device(attr, [&] {
     return cuda_error(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -691,31 +791,53 @@ static int launch_fwd_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st)
     record_event(1, st);
     return cuda_error(e, "forward (CTA pair) kernel launch");
   } else {
-    dim3 grid(a.Tm, a.HQ, a.B);
+    dim3 grid(a.Tm, QS2 ? a.HQ / 2 : a.HQ, a.B);  // QS2: one CTA per pair of heads
     kern<<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.kh, m.v, m.o, a);
     record_event(1, st);
     return check_launch("forward kernel launch");
   }
 }
 
-// Index mode pairs the softmax warps (its partial-tile bitmap masks make one softmax warp
-// per SM sub-partition issue bound); block and dense modes keep one (measured faster).
-// GQA with an even group size and Dv >= 128 can run on CTA pairs that share K and V:
-// by default only at head dims 256, where one CTA's forward is bound by shared-memory
-// operand reads that the pair halves; at 128 and 192/128 the softmax binds and the
-// pair's coupling made the forward slower (measured).
+// Forms (see sparse_attn_set_forward_form):
+//   one head per CTA: index mode pairs the softmax warps (its partial-tile bitmap masks
+//     make one softmax warp per SM sub-partition issue bound) and fetches the masks ahead;
+//     block and dense modes keep one warp per quarter (measured faster);
+//   CTA pair (GQA, even group, Dv >= 128): two heads on a 2-CTA cluster sharing each K/V
+//     tile through cta_group::2 MMAs; the default at head dims 256, where one CTA's
+//     forward waits on its single K and V stages;
+//   two heads per CTA (GQA, even group, Dqk <= 192, Dv <= 128): S and O of both heads in
+//     TMEM, one softmax warpgroup per head, so that one head's softmax overlaps the
+//     other head's MMAs; the default in block and dense modes at Dqk <= 128 (GQA D=128
+//     forward 0.419 -> 0.386 ms).  Its ten warps cap registers at 168 (three warps on
+//     two SM sub-partitions), so a full-row softmax spills a little; in index mode, with
+//     the bitmap masks on every tile, it measured slower than one head per CTA with
+//     paired softmax warps (3.72 against 3.13 ms at 192/128), which stays the default.
 template <int DQK, int DV>
 static int launch_fwd_dims(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
   constexpr bool kPairable = DV >= 128;
-  constexpr bool kPairByDefault = DQK == 256;
-  const int pol = g_fwd_pairs.load(std::memory_order_relaxed);
-  const bool cg2 = kPairable && (a.HQ / a.HK) % 2 == 0 &&
-                   (pol == SA_FWD_PAIRS_ON || (pol == SA_FWD_PAIRS_AUTO && kPairByDefault));
-  if (a.mode == SA_MODE_INDEX)
-    return cg2 ? launch_fwd_t<DQK, DV, true, kPairable>(a, m, st)
-               : launch_fwd_t<DQK, DV, true, false>(a, m, st);
-  return cg2 ? launch_fwd_t<DQK, DV, false, kPairable>(a, m, st)
-             : launch_fwd_t<DQK, DV, false, false>(a, m, st);
+  constexpr bool kTwoHeadsOk = DV <= 128 && DQK <= 192;
+  const bool even = (a.HQ / a.HK) % 2 == 0;
+  const bool index = a.mode == SA_MODE_INDEX;
+  int form = g_fwd_form.load(std::memory_order_relaxed);
+  if (form == SA_FWD_FORM_AUTO)
+    form = !even                      ? SA_FWD_FORM_ONE_HEAD
+           : DQK == 256               ? SA_FWD_FORM_CTA_PAIR
+           : (DQK <= 128 && !index)   ? SA_FWD_FORM_TWO_HEADS
+                                      : SA_FWD_FORM_ONE_HEAD;
+  if (form == SA_FWD_FORM_CTA_PAIR && !(kPairable && even)) form = SA_FWD_FORM_ONE_HEAD;
+  if (form == SA_FWD_FORM_TWO_HEADS && !(kTwoHeadsOk && even)) form = SA_FWD_FORM_ONE_HEAD;
+  if (form == SA_FWD_FORM_CTA_PAIR) {
+    if constexpr (kPairable)
+      return index ? launch_fwd_t<DQK, DV, true, true, false, true>(a, m, st)
+                   : launch_fwd_t<DQK, DV, false, true, false, false>(a, m, st);
+  }
+  if (form == SA_FWD_FORM_TWO_HEADS) {
+    if constexpr (kTwoHeadsOk)
+      return index ? launch_fwd_t<DQK, DV, false, false, true, true>(a, m, st)
+                   : launch_fwd_t<DQK, DV, false, false, true, false>(a, m, st);
+  }
+  return index ? launch_fwd_t<DQK, DV, true, false, false, true>(a, m, st)
+               : launch_fwd_t<DQK, DV, false, false, false, false>(a, m, st);
 }
 
 int launch_fwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {

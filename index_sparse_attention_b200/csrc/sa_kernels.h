@@ -47,8 +47,8 @@ struct AttnArgs {
 
 // Wait limit for the next launches (0: the default); see sparse_attn_set_wait_limit_ns.
 extern std::atomic<uint64_t> g_wait_limit_ns;
-// Forward form for GQA (SA_FWD_PAIRS_*); see sparse_attn_set_forward_pairs.
-extern std::atomic<int> g_fwd_pairs;
+// Forward form (SA_FWD_FORM_*); see sparse_attn_set_forward_form.
+extern std::atomic<int> g_fwd_form;
 
 struct TensorMaps {
   CUtensorMap q, k, v, dout, dq_acc, dk, dv, o;

@@ -100,15 +100,17 @@ def test_instrumentation_setters(lib):
     assert lib.sparse_attn_set_wait_limit_ns(0) == _lib.SA_OK
 
 
-def test_forward_pair_policy_setter(lib):
-    """The forward's GQA form: AUTO / ON / OFF are accepted, anything else is refused
-    with SA_ERR_INVALID; the binding maps the names and refuses unknown ones."""
+def test_forward_form_setter(lib):
+    """The forward's head-to-CTA form: the four SA_FWD_FORM_* values are accepted,
+    anything else is refused with SA_ERR_INVALID; the binding maps the names and refuses
+    unknown ones."""
     import index_sparse_attention_b200 as sa
-    for code in (_lib.SA_FWD_PAIRS_ON, _lib.SA_FWD_PAIRS_OFF, _lib.SA_FWD_PAIRS_AUTO):
-        assert lib.sparse_attn_set_forward_pairs(code) == _lib.SA_OK
-    for bad in (-1, 3, 1 << 20):
-        assert lib.sparse_attn_set_forward_pairs(bad) == _lib.SA_ERR_INVALID
-    for name in ("on", "off", "auto"):
-        sa.sparse_attn_set_forward_pairs(name)
+    for code in (_lib.SA_FWD_FORM_ONE_HEAD, _lib.SA_FWD_FORM_CTA_PAIR, _lib.SA_FWD_FORM_TWO_HEADS,
+                 _lib.SA_FWD_FORM_AUTO):
+        assert lib.sparse_attn_set_forward_form(code) == _lib.SA_OK
+    for bad in (-1, 4, 1 << 20):
+        assert lib.sparse_attn_set_forward_form(bad) == _lib.SA_ERR_INVALID
+    for name in ("one_head", "cta_pair", "two_heads", "auto"):
+        sa.sparse_attn_set_forward_form(name)
     with pytest.raises(ValueError):
-        sa.sparse_attn_set_forward_pairs("sometimes")
+        sa.sparse_attn_set_forward_form("sometimes")
