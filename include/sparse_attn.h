@@ -253,9 +253,9 @@ int sparse_attn_set_wait_limit_ns(uint64_t ns);
  *   SA_FWD_FORM_TWO_HEADS  two heads in one CTA, each with its own S and O in tensor
  *                          memory and its own softmax warps, so that one head's softmax
  *                          overlaps the other head's MMAs (needs Dqk <= 192, Dv <= 128);
- *   SA_FWD_FORM_AUTO       the library's choice (measured): CTA pairs at head dims 256,
- *                          two heads per CTA in block and dense modes at Dqk <= 128, one
- *                          head per CTA otherwise (MHA, an odd group size, index mode).
+ *   SA_FWD_FORM_AUTO       the library's choice (measured): two heads per CTA where that
+ *                          applies, CTA pairs at head dims 256, one head per CTA for MHA
+ *                          and odd group sizes.
  * A form that does not apply to a call falls back to one head per CTA.  All forms compute
  * the same O and LSE up to fp32 rounding.  Applies to the forward calls enqueued after it;
  * process-wide.  Returns SA_OK, or SA_ERR_INVALID for another value (the setting is then

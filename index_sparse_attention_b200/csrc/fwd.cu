@@ -591,26 +591,35 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
       // taken per warp (the warps of a pair hold the same rows and decide alike) so that
       // the warp-collective TMEM accesses stay converged.
       const bool need = m_tile > m_run + 8.0f;
-      if (__any_sync(0xFFFFFFFFu, need)) {
-        const float alpha = need ? ex2(m_run - m_tile) : 1.f;  // 0 when m_run = -inf
-        if (it > 0) {
-          // O holds P V up to tile it-1: rescale this thread's O columns in TMEM once
-          // that MMA is done
-          const bool o_ok = __all_sync(
-              0xFFFFFFFFu, mbar_wait(BAR(bar_od), (it - 1) & 1, abort_flag, a.status, a.wait_limit_ns));
-          if (!pair_all(o_ok)) {
+      const bool any_need = __any_sync(0xFFFFFFFFu, need);
+      const float alpha = need ? ex2(m_run - m_tile) : 1.f;  // 0 when m_run = -inf
+      // O holds P V up to tile it-1: rescale this thread's O columns in TMEM once that MMA
+      // is done (false: a wait gave up)
+      auto rescale_o = [&]() -> bool {
+        const bool o_ok = __all_sync(
+            0xFFFFFFFFu, mbar_wait(BAR(bar_od), (it - 1) & 1, abort_flag, a.status, a.wait_limit_ns));
+        if (!pair_all(o_ok)) return false;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = hc * kOCols; c < (hc + 1) * kOCols; c += 32) {
+          uint32_t ov[32];
+          tmem_ld32(tl + ocol + c, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st32(tl + ocol + c, ov);
+        }
+        return true;
+      };
+      // QS2 rescales after P is written (still before P V of this tile, which waits for
+      // the P-ready arrival below): the 32 O columns then never share registers with the
+      // 128 S values, and the wait for P V of tile it-1 overlaps the exponentials
+      constexpr bool kLateRescale = QS2;
+      if (any_need) {
+        if (!kLateRescale && it > 0) {
+          if (!rescale_o()) {
             ok = false;
             break;
-          }
-          tc_fence_after();
-#pragma unroll 1
-          for (int c = hc * kOCols; c < (hc + 1) * kOCols; c += 32) {
-            uint32_t ov[32];
-            tmem_ld32(tl + ocol + c, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(tl + ocol + c, ov);
           }
           tmem_wait_st();
         }
@@ -636,6 +645,10 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
         tmem_st16(tl + sb * 128 + (kCols / 2) * hc + c0 / 2, pk);
       }
       l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      if (kLateRescale && any_need && it > 0 && !rescale_o()) {
+        ok = false;
+        break;
+      }
       tmem_wait_st();
       tc_fence_before();
       ready(kBPF + sb);
@@ -807,11 +820,8 @@ static int launch_fwd_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st)
 //     forward waits on its single K and V stages;
 //   two heads per CTA (GQA, even group, Dqk <= 192, Dv <= 128): S and O of both heads in
 //     TMEM, one softmax warpgroup per head, so that one head's softmax overlaps the
-//     other head's MMAs; the default in block and dense modes at Dqk <= 128 (GQA D=128
-//     forward 0.419 -> 0.386 ms).  Its ten warps cap registers at 168 (three warps on
-//     two SM sub-partitions), so a full-row softmax spills a little; in index mode, with
-//     the bitmap masks on every tile, it measured slower than one head per CTA with
-//     paired softmax warps (3.72 against 3.13 ms at 192/128), which stays the default.
+//     other head's MMAs; the default there (forward 0.420 -> 0.368 ms on the D=128 GQA
+//     workload, 3.143 -> 2.786 ms on the 192/128 index workload).
 template <int DQK, int DV>
 static int launch_fwd_dims(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
   constexpr bool kPairable = DV >= 128;
@@ -820,10 +830,9 @@ static int launch_fwd_dims(const AttnArgs& a, const TensorMaps& m, cudaStream_t 
   const bool index = a.mode == SA_MODE_INDEX;
   int form = g_fwd_form.load(std::memory_order_relaxed);
   if (form == SA_FWD_FORM_AUTO)
-    form = !even                      ? SA_FWD_FORM_ONE_HEAD
-           : DQK == 256               ? SA_FWD_FORM_CTA_PAIR
-           : (DQK <= 128 && !index)   ? SA_FWD_FORM_TWO_HEADS
-                                      : SA_FWD_FORM_ONE_HEAD;
+    form = !even ? SA_FWD_FORM_ONE_HEAD
+           : kPairable && !kTwoHeadsOk ? SA_FWD_FORM_CTA_PAIR
+                                       : SA_FWD_FORM_TWO_HEADS;
   if (form == SA_FWD_FORM_CTA_PAIR && !(kPairable && even)) form = SA_FWD_FORM_ONE_HEAD;
   if (form == SA_FWD_FORM_TWO_HEADS && !(kTwoHeadsOk && even)) form = SA_FWD_FORM_ONE_HEAD;
   if (form == SA_FWD_FORM_CTA_PAIR) {
