@@ -1,7 +1,10 @@
 """Host-side helpers of bench.py that need no GPU: the code hash that keeps a committed
-DRAM-traffic measurement tied to the kernel source it was taken on."""
+DRAM-traffic measurement tied to the kernel source it was taken on, the peak basis, the
+converter's byte count, the index-statistics leg and the workload overrides."""
 import json
 import os
+
+import pytest
 
 import bench
 
@@ -72,3 +75,21 @@ def test_index_stats_leg_on_a_small_index_workload(capsys):
     # causal, 1024 tokens, top-2048: every (q, k <= q) pair is selected
     assert d["selected_pairs_per_kv_head"] == 1024 * 1025 // 2
     assert d["token_gather_forward_bytes"] == 4 * 1024 * 1025 // 2 * 2 * (192 + 128)
+
+
+def test_head_count_override_makes_a_gqa_workload():
+    """--heads HQ,HK turns a workload into GQA with those head counts (the mask is then
+    drawn per KV head); invalid counts are refused before any work."""
+    import argparse
+    from index_sparse_attention_b200 import inputs as I
+    ns = argparse.Namespace(workload="long_causal_blocksparse_h16_s32768_d256", seq=0,
+                            heads="16,8")
+    w = bench.get_workload(ns)
+    assert (w.HQ, w.HK, w.Dqk, w.Sq) == (16, 8, 256, 32768)
+    assert w.name.endswith("@H16x8")
+    assert I.block_mask(I.scaled(w, Sq=512, Sk=512)).shape == (1, 8, 4, 4)
+    for bad in ("16,5", "0,4", "8,16"):
+        with pytest.raises(SystemExit):
+            bench.get_workload(argparse.Namespace(workload=ns.workload, seq=0, heads=bad))
+    ns.heads = ""
+    assert bench.get_workload(ns) == I.WORKLOADS[ns.workload]
