@@ -41,6 +41,14 @@ CASES = [
              bs=64, density=0.5, name="bs64_b2_d256"),
     I.scaled(W["long_causal_blocksparse_h16_s32768_d256"], mode="index", Sq=450, Sk=450, HQ=4,
              HK=2, topk=120, name="index_ragged_d256"),
+    # group of six (head pairs (0,1), (2,3), (4,5) inside the group) and of three (odd:
+    # every form falls back to one head per CTA)
+    I.scaled(W["gqa_blocksparse_b2_hq32_hk8_s8192_d128"], B=1, Sq=384, Sk=384, HQ=12, HK=2,
+             name="block_g6_d128"),
+    I.scaled(W["indexsparse_gqa_q16384_hq32_hk4_d192_128_top2048"], Sq=300, Sk=300, HQ=6, HK=2,
+             topk=80, name="index_g3_d192_128"),
+    I.scaled(W["long_causal_blocksparse_h16_s32768_d256"], Sq=256, Sk=256, HQ=6, HK=1,
+             density=0.5, name="block_g6_d256"),
 ]
 FORMS = ("one_head", "cta_pair", "two_heads")
 
