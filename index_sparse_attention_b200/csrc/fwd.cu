@@ -6,38 +6,54 @@
 // out in its multi-row softmax notes: running max and running sum per row,
 // un-normalised P = exp(s - max), accumulate P V, final O = acc / sum.
 //
-// B200 design (one CTA per 128-query tile of one (batch, query head)):
+// B200 design: three forms of one kernel template, chosen per call (see
+// sparse_attn_set_forward_form).
+//
+// One head per CTA (one CTA per 128-query tile of one (batch, query head)):
 //   warp 0     TMA producer: Q once, then the K tiles of the ACTIVE key tiles only
 //              (the forward list), 128-byte swizzled, double-buffered when shared
 //              memory allows;
-//   warp 10    TMA producer of the V tiles, so that a K load (which S waits for)
-//              never queues behind a V load that waits for the previous P V.
+//   warp 6/10  TMA producer of the V tiles, so that a K load (which S waits for)
+//              never queues behind a V load that waits for the previous P V;
 //   warp 1     allocates 512 TMEM columns and issues the tcgen05 MMAs (one elected
 //              lane per batch): S = Q K^T into one of two TMEM S buffers (so the next S is
 //              computed while the softmax works on the current one), and
-//              O += P V with P read from TMEM (A operand in tensor memory).
-//   warps 2-9  softmax, two warps per TMEM lane quarter: a thread holds one query row
-//              (thread = TMEM lane) and one half of its 128 columns.  It tcgen05.ld's
-//              its half of the S row, applies the element mask on partial tiles (range,
-//              causal, 64-block mask or index bitmap), takes the row max with its
-//              partner (shared memory), updates the running max lazily (O is rescaled
-//              in TMEM only when the max grows by more than 2^8), exponentiates with
-//              ex2 and writes bf16 P back over the S buffer.  At the end the pair adds
-//              its row-sum halves, normalises O into the idle Q buffer (the output map's
-//              swizzled box layout, sent by TMA tensor stores) and writes LSE (fp32,
-//              natural log).  One softmax warp per SM sub-partition was issue bound.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+Dv).
+//              O += P V with P read from TMEM (A operand in tensor memory);
+//   softmax    warps 2-5 in block and dense modes (a thread holds one query row, thread
+//              = TMEM lane, all 128 columns); warps 2-9 in index mode, two per TMEM lane
+//              quarter, each with half of every row (they exchange row maxima per tile
+//              and row sums at the end through shared memory; one warp per SM
+//              sub-partition was issue bound by the bitmap masks).  A thread tcgen05.ld's
+//              its S columns, applies the element mask on partial tiles (range, causal,
+//              64-block mask or index bitmap; index-mode inputs fetched a tile ahead),
+//              updates the running max lazily (O is rescaled in TMEM only when the max
+//              grows by more than 2^8), exponentiates with ex2 and writes bf16 P back over
+//              the S buffer.  At the end it normalises O into the idle Q buffer (the output
+//              map's swizzled box layout, sent by TMA tensor stores) and writes LSE (fp32,
+//              natural log).
+//   With Dqk <= 192 the softmax warps first copy Q into TMEM and S reads it from there,
+//   so that only K comes from shared memory.
+//   TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+Dv), Q [256+Dv, 256+Dv+Dqk/2).
 //
-// GQA pair form (CG2): the query heads of one GQA group walk the same tile list, so two
-// of them (heads 2j and 2j+1, same query tile) run on a 2-CTA cluster whose MMAs are
-// pair MMAs (tcgen05 cta_group::2, M = 256: each CTA's 128 query rows).  The pair shares
-// every K and V tile: each CTA loads and holds half of it (keys [64 r, 64 r + 64) of K,
-// head-dim columns [Dv/2 r, Dv/2 r + Dv/2) of V, r = cluster rank), which halves the
-// per-CTA copy volume and shared-memory operand reads of B.  The even CTA (the leader)
-// issues every MMA; its commits arrive on the barriers of both CTAs; both CTAs' loads
-// complete on the leader's full barriers; the odd CTA's softmax warps report P (and Q
-// in TMEM) to the leader with one remote arrival per warp.  Softmax, masks, epilogue
-// and LSE are per CTA, as in the single-CTA form.
+// Two heads per CTA (QS2; GQA with an even group, Dqk <= 192, Dv <= 128): the query heads
+// of one GQA group walk the same tile list, so heads 2j and 2j+1 of one query tile share a
+// CTA, each with its own S buffer, O accumulator (TMEM: S_A, S_B, O_A, O_B), softmax
+// warpgroup (warps 2-5 and 6-9, full rows) and barriers.  Warp 0 loads Q of both heads, K,
+// and V one tile behind K.  Per key tile the MMA warp issues P V of head A, then head A's
+// next S into the same buffer, then the same for head B, so that one head's softmax
+// overlaps the other head's MMAs.  This form rescales O after writing P (ten warps cap
+// registers at 168, and O columns must not be live beside the 128 S values).
+//
+// CTA pair (CG2; GQA with an even group, Dv >= 128): two heads of one group (heads 2j and
+// 2j+1, same query tile) run on a 2-CTA cluster whose MMAs are pair MMAs (tcgen05
+// cta_group::2, M = 256: each CTA's 128 query rows).  The pair shares every K and V tile:
+// each CTA loads and holds half of it (keys [64 r, 64 r + 64) of K, head-dim columns
+// [Dv/2 r, Dv/2 r + Dv/2) of V, r = cluster rank), which halves the per-CTA copy volume and
+// shared-memory operand reads of B.  The even CTA (the leader) issues every MMA; its
+// commits arrive on the barriers of both CTAs; both CTAs' loads complete on the leader's
+// full barriers; the odd CTA's softmax warps report P (and Q in TMEM) to the leader with
+// one remote arrival per warp.  Softmax, masks, epilogue and LSE are per CTA, as in the
+// one-head form.
 // Every mbarrier wait is bounded; a timeout sets SA_ERR_TIMEOUT in the status word and
 // the CTA leaves after releasing its tensor memory.
 #include "sa_device.cuh"
