@@ -574,6 +574,78 @@ TOPK_METRIC = "top-k selector time per packed sequence (ms)"
 TOPK_PAGE_MS = {16384: 2.660752, 32768: 5.570000, 65536: 12.461776, 131072: 30.375248}
 
 
+def run_gather(args):
+    """Token-gather forward (sparse_attn_fwd_gather) against the block forward on an index
+    workload: both timed with CUDA events on the same inputs, and the gather path's
+    volume (the K/V rows it gathers) and token-level rate."""
+    import torch
+
+    import index_sparse_attention_b200 as sa
+
+    w = get_workload(args)
+    if w.mode != "index":
+        raise SystemExit("--op gather needs an index workload")
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    inp = I.make_inputs(w, with_grad=False)
+
+    def bf(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k, v = bf(inp.q), bf(inp.k), bf(inp.v)
+    idx = torch.from_numpy(inp.idx).to(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    bsp = sa.index_to_block_sparse(idx, w.Sk, causal=w.causal, dev_status=status)
+    o = torch.empty((w.B, w.Sq, w.HQ, w.Dv), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.HQ, w.Sq), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    with ClockSampler(dev.index) as clk:
+        g_ms = timed(lambda: sa.sparse_attn_fwd_gather(q, k, v, bsp, w.scale, o=o, lse=lse,
+                                                       dev_status=status))
+        b_ms = timed(lambda: sa.sparse_attn_fwd(q, k, v, bsp, w.scale, o=o, lse=lse,
+                                                dev_status=status))
+    assert int(status.item()) == 0
+    # selected (query, KV head) keys: distinct entries below the causal limit
+    pairs = 0
+    qpos = np.arange(w.Sq)[None, :, None, None]
+    for b in range(w.B):
+        x = np.sort(inp.idx[b:b + 1], axis=-1)
+        ok = x >= 0
+        if w.causal:
+            ok &= x <= qpos
+        ok[..., 1:] &= x[..., 1:] != x[..., :-1]
+        pairs += int(ok.sum())
+    G = w.HQ // w.HK
+    gathered = pairs * (w.Dqk + w.Dv) * 2
+    token_flop = pairs * G * 2 * (w.Dqk + w.Dv)
+    active = int(bsp.cnt.reshape(-1, 2).sum())
+    block_flop = active * w.HQ // w.HK * 2 * 128 * 128 * (w.Dqk + w.Dv)
+    print(json.dumps({
+        "op": "gather_vs_block_forward", "workload": w.name, "steps": args.steps,
+        "warmup": args.warmup, "gather_ms": g_ms, "block_ms": b_ms, "gather_over_block": g_ms / b_ms,
+        "gathered_bytes": gathered, "gather_gbs": gathered / (g_ms * 1e-3) / 1e9,
+        "token_level_tflop": token_flop / 1e12,
+        "token_level_tflops_gather": token_flop / (g_ms * 1e-3) / 1e12,
+        "block_counted_tflop": block_flop / 1e12,
+        "block_tflops_block_path": block_flop / (b_ms * 1e-3) / 1e12,
+        "token_level_tflops_block_path": token_flop / (b_ms * 1e-3) / 1e12,
+        "clocks": clk.summary(), "data": "synthetic",
+    }))
+
+
 def run_topk(args):
     import torch
 
@@ -743,9 +815,11 @@ def main():
                     help="forward head-to-CTA form for GQA: one CTA per query tile and head, "
                          "two heads on a 2-CTA pair with cta_group::2 MMAs, two heads per "
                          "CTA, or the library's choice (auto)")
-    ap.add_argument("--op", default="attention", choices=["attention", "topk", "index_stats"],
+    ap.add_argument("--op", default="attention",
+                    choices=["attention", "topk", "index_stats", "gather"],
                     help="topk: time the top-k selector alone on one packed sequence; "
-                         "index_stats: counts on an index workload (CPU only)")
+                         "index_stats: counts on an index workload (CPU only); gather: the "
+                         "token-gather forward against the block forward (index workload)")
     ap.add_argument("--pack", type=int, default=16384, help="--op topk: packed sequence length")
     ap.add_argument("--k", type=int, default=2048, help="--op topk: k")
     args = ap.parse_args()
@@ -755,6 +829,9 @@ def main():
         return
     if args.op == "index_stats":
         run_index_stats(args)
+        return
+    if args.op == "gather":
+        run_gather(args)
         return
     if args.impl == "reference":
         run_reference(args)

@@ -148,6 +148,20 @@ typedef struct sparse_attn_params {
  */
 int sparse_attn_fwd(const sparse_attn_params *p, sa_stream_t stream);
 
+/*
+ * sparse_attn_fwd_gather -- the same O and LSE in index mode, computed by gathering each
+ * query's selected K/V rows instead of streaming whole key tiles (the token-level
+ * alternative the sparse MLA backends of xtuner PR #2096, Background, stand for).  One
+ * warp per (batch, query, KV head) enumerates the query's keys from the presence bitmap
+ * of `sparse` (so repeated indices count once and the causal limit applies), gathers
+ * their rows 16 at a time and runs S = Q K^T and O += P V for the group's query heads on
+ * the tensor cores (mma.sync, the heads as M).  A comparison path: the benchmark times it
+ * against sparse_attn_fwd.  Needs sparse->mode == SA_MODE_INDEX, HQ / HK <= 8 and
+ * (Dqk, Dv) in {(64,64), (128,128), (192,128)} (SA_ERR_UNSUPPORTED otherwise).  Reads
+ * q, k, v and the bitmap; writes o, lse.
+ */
+int sparse_attn_fwd_gather(const sparse_attn_params *p, sa_stream_t stream);
+
 /* Bytes of device workspace sparse_attn_bwd needs for these shapes (fp32 Delta, the
  * fp32 dQ accumulator and the deterministic mode's int32 turn counters, each rounded
  * up to 256 B). */

@@ -15,9 +15,9 @@ from . import _lib
 from ._lib import SA_MODE_BLOCK, SA_MODE_DENSE, SA_MODE_INDEX, SA_TILE, SparseAttnError
 
 __all__ = ["BlockSparse", "block_mask_to_block_sparse", "index_to_block_sparse",
-           "sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_bwd_workspace_size",
-           "sparse_attn_bwd_noalloc", "topk_select", "sparse_attn_set_wait_limit_ns",
-           "sparse_attn_set_forward_form",
+           "sparse_attn_fwd", "sparse_attn_fwd_gather", "sparse_attn_bwd",
+           "sparse_attn_bwd_workspace_size", "sparse_attn_bwd_noalloc", "topk_select",
+           "sparse_attn_set_wait_limit_ns", "sparse_attn_set_forward_form",
            "SparseAttnError", "SA_TILE"]
 
 
@@ -209,6 +209,25 @@ def sparse_attn_fwd(q, k, v, sparse, softmax_scale=None, o=None, lse=None, dev_s
         lse = torch.empty((B, HQ, Sq), dtype=torch.float32, device=q.device)
     p = _params(q, k, v, o, lse, sparse, softmax_scale, dev_status=dev_status)
     _lib.check("sparse_attn_fwd", L.sparse_attn_fwd(ctypes.byref(p), _stream(q.device)))
+    return o, lse
+
+
+@_on_device("q")
+def sparse_attn_fwd_gather(q, k, v, sparse, softmax_scale=None, o=None, lse=None,
+                           dev_status=None):
+    """The forward of sparse_attn_fwd by per-query gathers of the selected K/V rows
+    (index mode only; HQ / HK <= 8; Dv <= 128): a comparison path, same O and LSE."""
+    L = _lib.load()
+    B, Sq, HQ, Dqk = q.shape
+    Dv = v.shape[3]
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(Dqk)
+    if o is None:
+        o = torch.empty((B, Sq, HQ, Dv), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, HQ, Sq), dtype=torch.float32, device=q.device)
+    p = _params(q, k, v, o, lse, sparse, softmax_scale, dev_status=dev_status)
+    _lib.check("sparse_attn_fwd_gather", L.sparse_attn_fwd_gather(ctypes.byref(p), _stream(q.device)))
     return o, lse
 
 

@@ -35,6 +35,7 @@ EXPORTS = (
     "index_to_block_sparse",
     "block_mask_to_block_sparse",
     "sparse_attn_fwd",
+    "sparse_attn_fwd_gather",
     "sparse_attn_bwd_workspace_size",
     "sparse_attn_bwd",
     "sparse_attn_bwd_deterministic",
@@ -88,6 +89,8 @@ def load():
     L.block_mask_to_block_sparse.restype = ctypes.c_int
     L.sparse_attn_fwd.argtypes = [P_p, vp]
     L.sparse_attn_fwd.restype = ctypes.c_int
+    L.sparse_attn_fwd_gather.argtypes = [P_p, vp]
+    L.sparse_attn_fwd_gather.restype = ctypes.c_int
     L.sparse_attn_bwd_workspace_size.argtypes = [P_p]
     L.sparse_attn_bwd_workspace_size.restype = ctypes.c_size_t
     L.sparse_attn_bwd.argtypes = [P_p, vp, ctypes.c_size_t, vp]

@@ -205,6 +205,21 @@ extern "C" int sparse_attn_set_forward_form(int form) {
   return SA_OK;
 }
 
+namespace sa {
+// token-gather forward (gather_fwd.cu)
+int launch_fwd_gather(const AttnArgs& a, const void* q, const void* k, const void* v,
+                      cudaStream_t st);
+}  // namespace sa
+
+extern "C" int sparse_attn_fwd_gather(const sparse_attn_params* p, sa_stream_t stream) {
+  AttnArgs a;
+  int rc = fill_args(p, &a, false);
+  if (rc) return rc;
+  rc = check_stream_device(reinterpret_cast<cudaStream_t>(stream));
+  if (rc) return rc;
+  return launch_fwd_gather(a, p->q, p->k, p->v, reinterpret_cast<cudaStream_t>(stream));
+}
+
 extern "C" int sparse_attn_fwd(const sparse_attn_params* p, sa_stream_t stream) {
   AttnArgs a;
   int rc = fill_args(p, &a, false);
