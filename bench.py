@@ -811,10 +811,11 @@ def main():
     ap.add_argument("--heads", default="",
                     help="override the head counts as HQ,HK (e.g. 16,8: GQA on the D=256 workload)")
     ap.add_argument("--fwd-form", default="auto",
-                    choices=["auto", "one_head", "cta_pair", "two_heads"],
-                    help="forward head-to-CTA form for GQA: one CTA per query tile and head, "
-                         "two heads on a 2-CTA pair with cta_group::2 MMAs, two heads per "
-                         "CTA, or the library's choice (auto)")
+                    choices=["auto", "one_head", "cta_pair", "two_heads", "two_tiles"],
+                    help="forward form: one CTA per query tile and head, two heads of a "
+                         "GQA group on a 2-CTA pair with cta_group::2 MMAs, two heads per "
+                         "CTA, two query tiles of one head per CTA, or the library's choice "
+                         "(auto)")
     ap.add_argument("--op", default="attention",
                     choices=["attention", "topk", "index_stats", "gather"],
                     help="topk: time the top-k selector alone on one packed sequence; "

@@ -251,11 +251,12 @@ int sparse_attn_set_wait_limit_ns(uint64_t ns);
 #define SA_FWD_FORM_ONE_HEAD 1
 #define SA_FWD_FORM_CTA_PAIR 2
 #define SA_FWD_FORM_TWO_HEADS 3
+#define SA_FWD_FORM_TWO_TILES 4
 
 /*
- * sparse_attn_set_forward_form -- selects how the forward maps query heads to CTAs.  The
- * pages pick the number of query tiles per CTA ("q_stage", sgl-flash-attn PR #28, "determine
- * q_stage via seqlen_q for sm100"), have 256-row tiles on SM100 (MagiAttention PR #331,
+ * sparse_attn_set_forward_form -- selects how the forward maps query heads (and query
+ * tiles) to CTAs.  The pages pick the number of query tiles per CTA ("q_stage",
+ * sgl-flash-attn PR #28, "determine q_stage via seqlen_q for sm100"), have 256-row tiles on SM100 (MagiAttention PR #331,
  * "CSR Tile Mapping") and a switch that turns the 2-CTA mode off (MagiAttention PR #334,
  * section 3, disable_2cta); the forms here are this library's own.  The query heads of
  * one GQA group walk the same tile list, so with an even group size two of them (same
@@ -267,9 +268,18 @@ int sparse_attn_set_wait_limit_ns(uint64_t ns);
  *   SA_FWD_FORM_TWO_HEADS  two heads in one CTA, each with its own S and O in tensor
  *                          memory and its own softmax warps, so that one head's softmax
  *                          overlaps the other head's MMAs (needs Dqk <= 192, Dv <= 128);
+ *   SA_FWD_FORM_TWO_TILES  two consecutive query tiles of one head in one CTA, arranged
+ *                          as the two heads above; the CTA walks the union of the two
+ *                          tiles' lists, and a key tile that one tile's list lacks is
+ *                          masked out for that tile's rows (needs Dqk, Dv <= 128 and at
+ *                          most 2048 key tiles).  Worth it where the two lists nearly
+ *                          agree (dense and causal masks); on lists that share few tiles
+ *                          the union costs up to twice the tensor work;
  *   SA_FWD_FORM_AUTO       the library's choice (measured): two heads per CTA where that
  *                          applies, CTA pairs at head dims 256, one head per CTA for MHA
- *                          and odd group sizes.
+ *                          and odd group sizes (two query tiles per CTA halve the CTA
+ *                          count, which lost more to partial waves than it gained at the
+ *                          sizes measured).
  * A form that does not apply to a call falls back to one head per CTA.  All forms compute
  * the same O and LSE up to fp32 rounding.  Applies to the forward calls enqueued after it;
  * process-wide.  Returns SA_OK, or SA_ERR_INVALID for another value (the setting is then

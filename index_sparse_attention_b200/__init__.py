@@ -324,15 +324,17 @@ def sparse_attn_set_wait_limit_ns(ns):
 
 
 _FWD_FORMS = {"auto": _lib.SA_FWD_FORM_AUTO, "one_head": _lib.SA_FWD_FORM_ONE_HEAD,
-              "cta_pair": _lib.SA_FWD_FORM_CTA_PAIR, "two_heads": _lib.SA_FWD_FORM_TWO_HEADS}
+              "cta_pair": _lib.SA_FWD_FORM_CTA_PAIR, "two_heads": _lib.SA_FWD_FORM_TWO_HEADS,
+              "two_tiles": _lib.SA_FWD_FORM_TWO_TILES}
 
 
 def sparse_attn_set_forward_form(form):
-    """How the forward maps query heads to CTAs: "auto" (the library's choice), "one_head"
-    (one CTA per query tile and head), "cta_pair" (two heads of a GQA group on a 2-CTA
-    cluster with cta_group::2 MMAs sharing each K/V tile) or "two_heads" (two heads of a
-    group in one CTA, one softmax warpgroup each).  A form that does not apply to a call
-    falls back to one head per CTA.  Applies to the forward calls made after it,
+    """How the forward maps query heads and tiles to CTAs: "auto" (the library's
+    choice), "one_head" (one CTA per query tile and head), "cta_pair" (two heads of a GQA
+    group on a 2-CTA cluster with cta_group::2 MMAs sharing each K/V tile), "two_heads"
+    (two heads of a group in one CTA, one softmax warpgroup each) or "two_tiles" (two
+    consecutive query tiles of one head in one CTA, walking the union of their lists).  A
+    form that does not apply to a call falls back to one head per CTA.  Applies to the forward calls made after it,
     process-wide; see include/sparse_attn.h."""
     code = _FWD_FORMS.get(form, form) if isinstance(form, str) else int(form)
     if isinstance(code, str):

@@ -25,6 +25,7 @@ SA_TOPK_MAX_K = 4096
 
 SA_MODE_DENSE, SA_MODE_BLOCK, SA_MODE_INDEX = 0, 1, 2
 SA_FWD_FORM_AUTO, SA_FWD_FORM_ONE_HEAD, SA_FWD_FORM_CTA_PAIR, SA_FWD_FORM_TWO_HEADS = 0, 1, 2, 3
+SA_FWD_FORM_TWO_TILES = 4
 SA_TILE = 128
 
 STATUS_INDEX = 1

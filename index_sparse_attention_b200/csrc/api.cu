@@ -200,7 +200,7 @@ extern "C" int sparse_attn_set_wait_limit_ns(uint64_t ns) {
 }
 
 extern "C" int sparse_attn_set_forward_form(int form) {
-  if (form < SA_FWD_FORM_AUTO || form > SA_FWD_FORM_TWO_HEADS) return SA_ERR_INVALID;
+  if (form < SA_FWD_FORM_AUTO || form > SA_FWD_FORM_TWO_TILES) return SA_ERR_INVALID;
   g_fwd_form.store(form, std::memory_order_relaxed);
   return SA_OK;
 }

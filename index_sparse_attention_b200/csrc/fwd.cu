@@ -44,6 +44,14 @@
 // overlaps the other head's MMAs.  This form rescales O after writing P (ten warps cap
 // registers at 168, and O columns must not be live beside the 128 S values).
 //
+// Two query tiles per CTA (QS2 == 2; Dqk, Dv <= 128, any group size): the same structure
+// for query tiles 2u and 2u + 1 of one head, which share K and V but have lists of their
+// own.  At the start warp 0 merges the two lists into their union in shared memory (the
+// tiles full for both first), each entry flagged per tile as absent, partial or full;
+// the CTA walks the union, and a tile's softmax masks out every key of a union entry
+// that its own list lacks.  Where the lists agree (dense) or differ by the diagonal tile
+// (causal) this costs nothing; where they share few tiles it costs up to twice the MMAs.
+//
 // CTA pair (CG2; GQA with an even group, Dv >= 128): two heads of one group (heads 2j and
 // 2j+1, same query tile) run on a 2-CTA cluster whose MMAs are pair MMAs (tcgen05
 // cta_group::2, M = 256: each CTA's 128 query rows).  The pair shares every K and V tile:
@@ -62,10 +70,16 @@
 
 namespace sa {
 
-template <int DQK, int DV, bool PAIRED, bool CG2, bool QS2>
+// Key tiles the two-query-tile form's union can hold (Sk up to 256K).
+constexpr int kUnionMaxTiles = 2048;
+
+// QS2: 0 one query tile of one head per CTA; 1 two heads of one GQA group (one query
+// tile); 2 two consecutive query tiles of one head.  Both QS2 forms hold two units (A, B),
+// each with its own Q tile, S buffer, O accumulator and softmax warpgroup.
+template <int DQK, int DV, bool PAIRED, bool CG2, int QS2>
 struct FwdCfg {
   static constexpr int kPanel = 128 * 128;  // one 64-column x 128-row swizzled panel
-  static constexpr int kHeads = QS2 ? 2 : 1;  // query heads per CTA
+  static constexpr int kHeads = QS2 ? 2 : 1;  // Q tiles (units) per CTA
   // K rows and V columns one CTA holds per tile (a pair splits both in halves)
   static constexpr int kKRows = CG2 ? 64 : 128;
   static constexpr int kKPanel = kKRows * 128;  // one 64-column panel of K
@@ -83,7 +97,12 @@ struct FwdCfg {
   // softmax exchange of the paired warps: row max [2 tile parities][2 column halves][128
   // rows] and row sum [2 halves][128 rows], fp32
   static constexpr int kXOff = kBarOff + 256;
-  static constexpr int kSmem = kXOff + (PAIRED ? 3 * 1024 : 0) + 1024;  // + alignment slack
+  // two query tiles (QS2 == 2): the union of the two tiles' lists, built in shared memory
+  // at the start: kUnionMax int32 entries, a byte per key tile, two int32 counts
+  static constexpr int kUnionMax = kUnionMaxTiles;
+  static constexpr int kUOff = kXOff + (PAIRED ? 3 * 1024 : 0);
+  static constexpr int kUBytes = QS2 == 2 ? 5 * kUnionMax + 8 : 0;
+  static constexpr int kSmem = kUOff + kUBytes + 1024;  // + alignment slack
   // softmax warps per TMEM lane quarter (PAIRED: two, each with half of every row)
   static constexpr int kHalves = PAIRED ? 2 : 1;
   static constexpr int kThreads = QS2 ? 320 : PAIRED ? 352 : 224;
@@ -99,7 +118,7 @@ struct FwdCfg {
   static_assert(kOCol + DV <= kTmemCols, "tensor memory budget");
   static_assert(!kQT || kColQ + DQK / 2 <= kTmemCols, "tensor memory budget (Q)");
   static_assert(!CG2 || DV >= 128, "a CTA pair splits V into 64-column panels");
-  static_assert(!QS2 || (!PAIRED && !CG2 && DQK <= 192), "two heads per CTA: full rows, one CTA");
+  static_assert(!QS2 || (!PAIRED && !CG2 && DQK <= 192), "two units per CTA: full rows, one CTA");
   static_assert(kOCol + kHeads * DV <= kTmemCols, "tensor memory budget (two heads)");
   static_assert(kKStages <= 4 && kVStages <= 4, "barrier slots");
 };
@@ -110,7 +129,7 @@ enum : int { kBQ = 0, kBKF = 1, kBKE = 5, kBVF = 9, kBVE = 13, kBSF = 17, kBPF =
 
 // tm_kh: K in 64-row boxes (the half tile a CTA of a pair loads); unused by the
 // single-CTA form.
-template <int DQK, int DV, bool PAIRED, bool CG2, bool QS2, bool PREFETCH>
+template <int DQK, int DV, bool PAIRED, bool CG2, int QS2, bool PREFETCH>
 __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
     sparse_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -132,10 +151,13 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
   // pair: the two CTAs of a cluster are blockIdx.x = 2c, 2c + 1 (rank 0 leads)
   const uint32_t rank = CG2 ? cluster_ctarank() : 0u;
   const int xt = CG2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-  const int mt = a.Tm - 1 - xt;  // longest lists first under causal
-  // (QS2: h is the first of the CTA's two heads, h + 1 the second)
-  const int h = (CG2 || QS2) ? 2 * static_cast<int>(blockIdx.y) + static_cast<int>(rank)
-                             : static_cast<int>(blockIdx.y);
+  // longest lists first under causal; two query tiles (kTiles): CTA xt holds tiles mt and
+  // mt + 1 (the second one absent past the last tile)
+  constexpr bool kTiles = QS2 == 2;
+  const int mt = kTiles ? 2 * ((a.Tm + 1) / 2 - 1 - xt) : a.Tm - 1 - xt;
+  // (two heads: h is the first of the CTA's two heads, h + 1 the second)
+  const int h = (CG2 || QS2 == 1) ? 2 * static_cast<int>(blockIdx.y) + static_cast<int>(rank)
+                                  : static_cast<int>(blockIdx.y);
   const int b = blockIdx.z;
   // the leader's barriers as seen from this CTA (remote arrivals and pair loads)
   const uint32_t lbar0 = CG2 ? mapa_shared(bar0, 0) : bar0;
@@ -143,9 +165,19 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
   const int g = h / (a.HQ / a.HK);
   const int64_t bg = static_cast<int64_t>(b) * a.HK + g;
   const int64_t lrow = bg * a.Tm + mt;
-  const int n_full = __ldg(a.cnt + 2 * lrow);
-  const int n_iter = n_full + __ldg(a.cnt + 2 * lrow + 1);
   const int32_t* list = a.idx + lrow * a.Tn;
+  // Two query tiles walk the union of their lists (uni), whose entries carry the key
+  // tile (bits 0-27) and, per unit u, whether the tile is absent from (0), partial in (1)
+  // or full in (2) that unit's own list (bits 28 + 2u, 29 + 2u); the entries full for both
+  // come first.  n_iter is provisional until the union is built (it is > 0 exactly when
+  // the union is not empty).
+  const bool has_b = kTiles && mt + 1 < a.Tm;
+  int32_t* uni = reinterpret_cast<int32_t*>(smem + C::kUOff);
+  int n_full = __ldg(a.cnt + 2 * lrow);
+  int n_iter = n_full + __ldg(a.cnt + 2 * lrow + 1);
+  if (kTiles && has_b) n_iter += __ldg(a.cnt + 2 * lrow + 2) + __ldg(a.cnt + 2 * lrow + 3);
+  auto entry_at = [&](int t) -> int { return kTiles ? uni[t] : __ldg(list + t); };
+  auto tile_of = [](int e) -> int { return kTiles ? (e & 0x0FFFFFFF) : e; };
   // loads issued by the two producers (the abort path drains the last ones in flight)
   int issued_k = 0, issued_v = 0;
 
@@ -173,6 +205,56 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
     abort_flag->abort = 0;
     abort_flag->peer_abort = 0;
     fence_mbar_init();
+    if (kTiles && n_iter > 0) {
+      // two query tiles: their Q loads start now, while warp 0 builds the union below
+      // (past the last query tile, B's box lies beyond Sq and is zero-filled)
+      fence_proxy_async_smem();
+      prefetch_tensormap(&tm_q);
+      mbar_arrive_expect_tx(BAR(kBQ), 2 * C::kQBytes);
+      for (int u = 0; u < 2; ++u)
+        for (int c = 0; c < DQK / 64; ++c)
+          tma_load_4d(sbase + C::kQOff + u * C::kQBytes + c * C::kPanel, &tm_q, BAR(kBQ), c * 64,
+                      (mt + u) * 128, h, b);
+    }
+  }
+  if (kTiles && warp == 0) {
+    // The union of the two query tiles' lists (each: full entries, then partial ones;
+    // every key tile at most once).  cls[t] collects per key tile t: bit 2u + 1 full in
+    // unit u's list, bit 2u partial in it.  Without a second tile, B takes A's flags.
+    uint8_t* cls = smem + C::kUOff + 4 * C::kUnionMax;
+    int32_t* cnts = reinterpret_cast<int32_t*>(cls + C::kUnionMax);
+    const int tn = a.Tn;
+    for (int t = lane; t < tn; t += 32) cls[t] = 0;
+    __syncwarp();
+    for (int u = 0; u < (has_b ? 2 : 1); ++u) {
+      const int64_t lr = lrow + u;
+      const int nf = __ldg(a.cnt + 2 * lr), nl = nf + __ldg(a.cnt + 2 * lr + 1);
+      for (int e = lane; e < nl; e += 32) {
+        const int t = __ldg(a.idx + lr * a.Tn + e);
+        if (t >= 0 && t < tn) cls[t] |= static_cast<uint8_t>((e < nf ? 2 : 1) << (2 * u));
+      }
+      __syncwarp();
+    }
+    int n = 0, nfull = 0;
+    for (int pass = 0; pass < 2; ++pass) {  // full for both, then the rest
+      for (int t0 = 0; t0 < tn; t0 += 32) {
+        const int t = t0 + lane;
+        const uint32_t c = t < tn ? cls[t] : 0u;
+        const uint32_t fa = c & 3u, fb = has_b ? (c >> 2) & 3u : fa;
+        const bool both_full = fa == 2u && fb == 2u;
+        const bool take = c != 0u && (pass == 0) == both_full;
+        const uint32_t bal = __ballot_sync(0xFFFFFFFFu, take);
+        if (take)
+          uni[n + __popc(bal & ((1u << lane) - 1u))] =
+              static_cast<int32_t>(static_cast<uint32_t>(t) | (fa << 28) | (fb << 30));
+        n += __popc(bal);
+      }
+      if (pass == 0) nfull = n;
+    }
+    if (lane == 0) {
+      cnts[0] = nfull;
+      cnts[1] = n;
+    }
   }
   if (warp == 1) {
     if constexpr (CG2) {
@@ -189,6 +271,13 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
   tc_fence_after();
   // broadcast from lane 0 so that the compiler can treat it as warp-uniform
   const uint32_t tmem = __shfl_sync(0xFFFFFFFFu, *tmem_slot, 0);
+  // (the Q loads above were issued on the provisional count)
+  const bool q_issued = kTiles && n_iter > 0;
+  if constexpr (kTiles) {
+    const int32_t* cnts = reinterpret_cast<const int32_t*>(smem + C::kUOff + 5 * C::kUnionMax);
+    n_full = cnts[0];
+    n_iter = cnts[1];
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
@@ -205,8 +294,8 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
           for (int c = 0; c < DQK / 64; ++c)
             tma_load_4d_pair(sbase + C::kQOff + c * C::kPanel, &tm_q, LBAR(kBQ), c * 64, mt * 128,
                              h, b);
-        } else {
-          // (QS2: the tiles of heads h and h + 1, one after the other)
+        } else if (!kTiles) {  // (two query tiles: loaded before the union was built)
+          // (two heads: the tiles of heads h and h + 1, one after the other)
           mbar_arrive_expect_tx(BAR(kBQ), C::kHeads * C::kQBytes);
           for (int hd = 0; hd < C::kHeads; ++hd)
             for (int c = 0; c < DQK / 64; ++c)
@@ -215,8 +304,13 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
         }
       }
       __syncwarp();
+      // key tile of list entry t (read by every lane, the same address)
+      auto tile_at = [&](int t) -> int {
+        if constexpr (kTiles) return tile_of(uni[t]);
+        return __shfl_sync(0xFFFFFFFFu, __ldg(list + t), 0);
+      };
       auto load_v = [&](int t) -> bool {  // V tile t (QS2)
-        const int nt = __shfl_sync(0xFFFFFFFFu, __ldg(list + t), 0);
+        const int nt = tile_at(t);
         const int vs = t % C::kVStages, vu = t / C::kVStages;
         if (!warp_wait(BAR(kBVE + vs), (vu & 1) ^ 1, abort_flag, a.status, a.wait_limit_ns))
           return false;
@@ -233,7 +327,7 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
       // K tiles: each one as soon as S of the tile that last used its buffer is done (V
       // tiles have a producer warp of their own, so a K load never waits behind P V)
       for (int it = 0; it < n_iter; ++it) {
-        const int nt = __shfl_sync(0xFFFFFFFFu, __ldg(list + it), 0);
+        const int nt = tile_at(it);
         const int ks = it % C::kKStages, ku = it / C::kKStages;
         if (!warp_wait(BAR(kBKE + ks), (ku & 1) ^ 1, abort_flag, a.status, a.wait_limit_ns)) break;
         if (elect_one()) {
@@ -440,10 +534,12 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
     constexpr int kOCols = DV / kH;                  // O columns rescaled / stored per thread
     const int quarter = warp & 3;
     const int hc = kH == 2 ? (warp - 2) >> 2 : 0;   // column part of this warp
-    // QS2: warps 2-5 hold head h, warps 6-9 head h + 1, each with its own S buffer, O
-    // accumulator and barriers
+    // QS2: warps 2-5 hold unit A, warps 6-9 unit B (head h + 1 of the same query tile, or
+    // query tile mt + 1 of the same head), each with its own S buffer, O accumulator and
+    // barriers
     const int hd = QS2 ? (warp - 2) >> 2 : 0;
-    const int hh = h + hd;                           // this warp's query head
+    const int hh = QS2 == 1 ? h + hd : h;            // this warp's query head
+    const int mtu = kTiles ? mt + hd : mt;           // and query tile
     const uint32_t ocol = C::kOCol + static_cast<uint32_t>(hd * DV);
     const int bar_od = hd ? kBOD2 : kBOD, bar_ofin = hd ? kBOFin2 : kBOFin;
     const int pair_bar = 1 + ((warp - 2) & 3);       // named barrier of a pair (64 threads)
@@ -452,7 +548,7 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
       return v;
     };
     const int r = quarter * 32 + lane;
-    const int64_t i = static_cast<int64_t>(mt) * 128 + r;
+    const int64_t i = static_cast<int64_t>(mtu) * 128 + r;
     const bool row_ok = i < a.Sq;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     float* xmax = reinterpret_cast<float*>(smem + C::kXOff);          // [2][2][128]
@@ -506,8 +602,8 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
     // softmax warp more than it saves (+3 to +4% measured).
     constexpr bool kPrefetch = PREFETCH;  // the index-mode instances
     constexpr int kWords = kCols / 32;
-    auto fetch_nt = [&](int t) {
-      return (kPrefetch && t < n_iter && t >= n_full) ? __ldg(list + t) : 0;
+    auto fetch_nt = [&](int t) {  // a list entry (two query tiles: with its flags)
+      return (kPrefetch && t < n_iter && t >= n_full) ? entry_at(t) : 0;
     };
     // the mask inputs of key tile nt for this thread's row and columns
     auto load_mask = [&](int nt, uint32_t (&wd)[kWords], bool& m0, bool& m1) {
@@ -529,7 +625,7 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
       m0 = m1 = true;
 #pragma unroll
       for (int k = 0; k < kWords; ++k) wd[k] = ~0u;
-      if (kPrefetch && t < n_iter && t >= n_full) load_mask(nt, wd, m0, m1);
+      if (kPrefetch && t < n_iter && t >= n_full) load_mask(tile_of(nt), wd, m0, m1);
     };
     int nt_cur = fetch_nt(0), nt_nxt = fetch_nt(1);
     uint32_t wd_cur[kWords];
@@ -560,7 +656,8 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
       for (int c = 0; c < kCols; ++c) x[c] = __uint_as_float(u[c]);
       if (it >= n_full) {
         // partial tile: element mask (tile columns kCols hc + c)
-        const int nt = kPrefetch ? nt_cur : __ldg(list + it);
+        const int ent = kPrefetch ? nt_cur : entry_at(it);
+        const int nt = tile_of(ent);
         const int64_t n0 = static_cast<int64_t>(nt) * 128;
         int64_t lim = a.Sk;
         if (a.causal) lim = min64(lim, i + 1);
@@ -577,6 +674,11 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
 #pragma unroll
           for (int c = 0; c < kCols; ++c)
             if (!((wd_cur[c >> 5] >> (c & 31)) & 1u)) x[c] = -INFINITY;
+        }
+        // two query tiles: a tile of the union that this unit's own list lacks
+        if (kTiles && ((static_cast<uint32_t>(ent) >> (28 + 2 * hd)) & 3u) == 0u) {
+#pragma unroll
+          for (int c = 0; c < kCols; ++c) x[c] = -INFINITY;
         }
       }
       nt_cur = nt_nxt;
@@ -711,10 +813,11 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
     }
     fence_proxy_async_smem();
     named_bar_sync(5 + hd, 128 * kH);  // every softmax warp (of this head)
-    if (threadIdx.x == 64 + 128 * hd) {
+    // (no store for a second query tile past the last one)
+    if (threadIdx.x == 64 + 128 * hd && static_cast<int64_t>(mtu) * 128 < a.Sq) {
 #pragma unroll
       for (int p = 0; p < DV / 64; ++p)
-        tma_store_4d(&tm_o, sbase + C::kQOff + hd * C::kQBytes + p * C::kPanel, p * 64, mt * 128,
+        tma_store_4d(&tm_o, sbase + C::kQOff + hd * C::kQBytes + p * C::kPanel, p * 64, mtu * 128,
                      hh, b);
       bulk_commit_group();
       bulk_wait_group_read0();  // the Q buffer is read before the CTA may leave
@@ -783,6 +886,8 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
     __syncthreads();
     if constexpr (CG2) cluster_sync_all();
   }
+  // two query tiles whose lists held no valid key tile: nothing waited for their Q loads
+  if (q_issued && n_iter == 0 && threadIdx.x == 0) mbar_wait_limited(BAR(kBQ), 0);
   if (warp == 1) {
     tc_fence_after();
     if constexpr (CG2) tmem_dealloc_pair(tmem, C::kTmemCols);
@@ -790,7 +895,7 @@ __global__ void __launch_bounds__(QS2 ? 320 : PAIRED ? 352 : 224, 1)
   }
 }
 
-template <int DQK, int DV, bool PAIRED, bool CG2, bool QS2, bool PREFETCH>
+template <int DQK, int DV, bool PAIRED, bool CG2, int QS2, bool PREFETCH>
 static int launch_fwd_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
   using C = FwdCfg<DQK, DV, PAIRED, CG2, QS2>;
   auto kern = sparse_fwd_kernel<DQK, DV, PAIRED, CG2, QS2, PREFETCH>;
@@ -820,7 +925,8 @@ static int launch_fwd_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st)
     record_event(1, st);
     return cuda_error(e, "forward (CTA pair) kernel launch");
   } else {
-    dim3 grid(a.Tm, QS2 ? a.HQ / 2 : a.HQ, a.B);  // QS2: one CTA per pair of heads
+    // two heads: one CTA per pair of heads; two query tiles: per pair of query tiles
+    dim3 grid(QS2 == 2 ? (a.Tm + 1) / 2 : a.Tm, QS2 == 1 ? a.HQ / 2 : a.HQ, a.B);
     kern<<<grid, C::kThreads, C::kSmem, st>>>(m.q, m.k, m.kh, m.v, m.o, a);
     record_event(1, st);
     return check_launch("forward kernel launch");
@@ -837,13 +943,22 @@ static int launch_fwd_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st)
 //   two heads per CTA (GQA, even group, Dqk <= 192, Dv <= 128): S and O of both heads in
 //     TMEM, one softmax warpgroup per head, so that one head's softmax overlaps the
 //     other head's MMAs; the default there (forward 0.420 -> 0.368 ms on the D=128 GQA
-//     workload, 3.143 -> 2.786 ms on the 192/128 index workload).
+//     workload, 3.143 -> 2.786 ms on the 192/128 index workload);
+//   two query tiles per CTA (Dqk, Dv <= 128, at most 2048 key tiles): the same
+//     structure for query tiles 2u and 2u + 1 of one head, walking the union of their
+//     lists; chosen explicitly only.  Per query tile it is ~5% faster than one head per
+//     CTA on dense D=128 lists, but it halves the CTA count (3.5 waves on 148 SMs at
+//     S=4096, B=2, H=16: dense full forward 0.2705 -> 0.293 ms, causal 0.180 -> 0.197),
+//     and on lists that share few tiles the union costs up to twice the tensor work
+//     (random 25% block mask at S=8192: 0.418 -> 0.727 ms).
 template <int DQK, int DV>
 static int launch_fwd_dims(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
   constexpr bool kPairable = DV >= 128;
   constexpr bool kTwoHeadsOk = DV <= 128 && DQK <= 192;
+  constexpr bool kTwoTilesOk = DV <= 128 && DQK <= 128;
   const bool even = (a.HQ / a.HK) % 2 == 0;
   const bool index = a.mode == SA_MODE_INDEX;
+  const bool tiles_fit = a.Tn <= kUnionMaxTiles;
   int form = g_fwd_form.load(std::memory_order_relaxed);
   if (form == SA_FWD_FORM_AUTO)
     form = !even ? SA_FWD_FORM_ONE_HEAD
@@ -851,18 +966,24 @@ static int launch_fwd_dims(const AttnArgs& a, const TensorMaps& m, cudaStream_t 
                                        : SA_FWD_FORM_TWO_HEADS;
   if (form == SA_FWD_FORM_CTA_PAIR && !(kPairable && even)) form = SA_FWD_FORM_ONE_HEAD;
   if (form == SA_FWD_FORM_TWO_HEADS && !(kTwoHeadsOk && even)) form = SA_FWD_FORM_ONE_HEAD;
+  if (form == SA_FWD_FORM_TWO_TILES && !(kTwoTilesOk && tiles_fit)) form = SA_FWD_FORM_ONE_HEAD;
   if (form == SA_FWD_FORM_CTA_PAIR) {
     if constexpr (kPairable)
-      return index ? launch_fwd_t<DQK, DV, true, true, false, true>(a, m, st)
-                   : launch_fwd_t<DQK, DV, false, true, false, false>(a, m, st);
+      return index ? launch_fwd_t<DQK, DV, true, true, 0, true>(a, m, st)
+                   : launch_fwd_t<DQK, DV, false, true, 0, false>(a, m, st);
   }
   if (form == SA_FWD_FORM_TWO_HEADS) {
     if constexpr (kTwoHeadsOk)
-      return index ? launch_fwd_t<DQK, DV, false, false, true, true>(a, m, st)
-                   : launch_fwd_t<DQK, DV, false, false, true, false>(a, m, st);
+      return index ? launch_fwd_t<DQK, DV, false, false, 1, true>(a, m, st)
+                   : launch_fwd_t<DQK, DV, false, false, 1, false>(a, m, st);
   }
-  return index ? launch_fwd_t<DQK, DV, true, false, false, true>(a, m, st)
-               : launch_fwd_t<DQK, DV, false, false, false, false>(a, m, st);
+  if (form == SA_FWD_FORM_TWO_TILES) {
+    if constexpr (kTwoTilesOk)
+      return index ? launch_fwd_t<DQK, DV, false, false, 2, true>(a, m, st)
+                   : launch_fwd_t<DQK, DV, false, false, 2, false>(a, m, st);
+  }
+  return index ? launch_fwd_t<DQK, DV, true, false, 0, true>(a, m, st)
+               : launch_fwd_t<DQK, DV, false, false, 0, false>(a, m, st);
 }
 
 int launch_fwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {

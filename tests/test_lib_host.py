@@ -106,11 +106,11 @@ def test_forward_form_setter(lib):
     unknown ones."""
     import index_sparse_attention_b200 as sa
     for code in (_lib.SA_FWD_FORM_ONE_HEAD, _lib.SA_FWD_FORM_CTA_PAIR, _lib.SA_FWD_FORM_TWO_HEADS,
-                 _lib.SA_FWD_FORM_AUTO):
+                 _lib.SA_FWD_FORM_TWO_TILES, _lib.SA_FWD_FORM_AUTO):
         assert lib.sparse_attn_set_forward_form(code) == _lib.SA_OK
-    for bad in (-1, 4, 1 << 20):
+    for bad in (-1, 5, 1 << 20):
         assert lib.sparse_attn_set_forward_form(bad) == _lib.SA_ERR_INVALID
-    for name in ("one_head", "cta_pair", "two_heads", "auto"):
+    for name in ("one_head", "cta_pair", "two_heads", "two_tiles", "auto"):
         sa.sparse_attn_set_forward_form(name)
     with pytest.raises(ValueError):
         sa.sparse_attn_set_forward_form("sometimes")
