@@ -277,9 +277,9 @@ int sparse_attn_set_wait_limit_ns(uint64_t ns);
  *                          the union costs up to twice the tensor work;
  *   SA_FWD_FORM_AUTO       the library's choice (measured): two heads per CTA where that
  *                          applies, CTA pairs at head dims 256, one head per CTA for MHA
- *                          and odd group sizes (two query tiles per CTA halve the CTA
- *                          count, which lost more to partial waves than it gained at the
- *                          sizes measured).
+ *                          and odd group sizes (two query tiles per CTA measured no
+ *                          faster on dense lists, and slower where halving the CTA count
+ *                          leaves a partial last wave).
  * A form that does not apply to a call falls back to one head per CTA.  All forms compute
  * the same O and LSE up to fp32 rounding.  Applies to the forward calls enqueued after it;
  * process-wide.  Returns SA_OK, or SA_ERR_INVALID for another value (the setting is then

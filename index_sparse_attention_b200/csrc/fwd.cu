@@ -946,11 +946,14 @@ static int launch_fwd_t(const AttnArgs& a, const TensorMaps& m, cudaStream_t st)
 //     workload, 3.143 -> 2.786 ms on the 192/128 index workload);
 //   two query tiles per CTA (Dqk, Dv <= 128, at most 2048 key tiles): the same
 //     structure for query tiles 2u and 2u + 1 of one head, walking the union of their
-//     lists; chosen explicitly only.  Per query tile it is ~5% faster than one head per
-//     CTA on dense D=128 lists, but it halves the CTA count (3.5 waves on 148 SMs at
-//     S=4096, B=2, H=16: dense full forward 0.2705 -> 0.293 ms, causal 0.180 -> 0.197),
-//     and on lists that share few tiles the union costs up to twice the tensor work
-//     (random 25% block mask at S=8192: 0.418 -> 0.727 ms).
+//     lists; chosen explicitly only.  On dense D=128 lists it measured no faster than
+//     one head per CTA even with many waves (S=16384: causal 1.984 -> 2.085 ms, full
+//     3.776 -> 3.75-3.84), and slower where halving the CTA count leaves a partial last
+//     wave (S=4096: full 0.2705 -> 0.293, causal 0.180 -> 0.197): with two S and two O
+//     buffers TMEM has no room for Q, so its S MMAs read both operands from shared
+//     memory, the port the one-head form keeps half free.  On lists that share few
+//     tiles the union costs up to twice the tensor work (random 25% block mask at
+//     S=8192: 0.418 -> 0.727 ms).
 template <int DQK, int DV>
 static int launch_fwd_dims(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
   constexpr bool kPairable = DV >= 128;
