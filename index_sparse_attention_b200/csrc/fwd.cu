@@ -50,7 +50,9 @@
 // tiles full for both first), each entry flagged per tile as absent, partial or full;
 // the CTA walks the union, and a tile's softmax masks out every key of a union entry
 // that its own list lacks.  Where the lists agree (dense) or differ by the diagonal tile
-// (causal) this costs nothing; where they share few tiles it costs up to twice the MMAs.
+// (causal) this adds no MMAs; where they share few tiles it costs up to twice the MMAs.
+// Measured no faster than one head per CTA (see launch_fwd_dims), it is chosen
+// explicitly only.
 //
 // CTA pair (CG2; GQA with an even group, Dv >= 128): two heads of one group (heads 2j and
 // 2j+1, same query tile) run on a 2-CTA cluster whose MMAs are pair MMAs (tcgen05
