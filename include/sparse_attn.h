@@ -138,6 +138,9 @@ typedef struct sparse_attn_params {
   const sa_block_sparse *sparse; /* host pointer; lists built for the same B, HK, Sq, Sk */
   int32_t *dev_status;           /* optional device int32 */
 } sparse_attn_params;
+/* Sizes: B, HQ, HK, Sq and Sk are at least 1 here and in sa_block_sparse; a problem with
+ * a zero extent has nothing to compute and is refused with SA_ERR_INVALID before any
+ * launch (callers skip the call). */
 
 /*
  * sparse_attn_fwd -- forward: O and LSE.  Streams only the listed key tiles of each

@@ -75,6 +75,20 @@ def test_unsupported_and_inconsistent_shapes(lib):
     assert lib.sparse_attn_fwd(ctypes.byref(p), None) == _lib.SA_ERR_INVALID
 
 
+def test_zero_extents_are_refused_on_host(lib):
+    """A problem with a zero extent is refused before any launch, by every entry point."""
+    for field in ("B", "HQ", "HK", "Sq", "Sk"):
+        p, s = _fake_params(**{field: 0})
+        assert lib.sparse_attn_fwd(ctypes.byref(p), None) == _lib.SA_ERR_INVALID, field
+        assert lib.sparse_attn_bwd(ctypes.byref(p), 0x2000, 1 << 30, None) == _lib.SA_ERR_INVALID, field
+        if field in ("B", "HQ", "Sq"):  # the workspace holds per-query-row data only
+            assert lib.sparse_attn_bwd_workspace_size(ctypes.byref(p)) == 0, field
+    for field in ("B", "HK", "Sq", "Sk"):
+        p, s = _fake_params()
+        setattr(s, field, 0)
+        assert lib.block_mask_to_block_sparse(ctypes.byref(s), None) == _lib.SA_ERR_INVALID, field
+
+
 def test_bwd_workspace_is_checked_on_host(lib):
     p, s = _fake_params()
     need = lib.sparse_attn_bwd_workspace_size(ctypes.byref(p))
