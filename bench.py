@@ -89,11 +89,14 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def bwd_kernel_name(w):
-    """The backward main kernel that the library launches for this workload's head dims."""
+def bwd_kernel_name(w, deterministic=False):
+    """The backward main kernel that the library launches for this workload's head dims
+    (at (192,128) one CTA per key tile, or the head-dim split over two in deterministic
+    mode)."""
     if (w.Dqk, w.Dv) == (256, 256):
         return "sparse_bwd_pair_kernel"
-    inst = {(64, 64): "128,128,1", (128, 128): "128,128,1", (192, 128): "192,128,2"}
+    inst = {(64, 64): "128,128,1", (128, 128): "128,128,1",
+            (192, 128): "192,128,2" if deterministic else "192,128,1"}
     return f"sparse_bwd_kernel<{inst.get((w.Dqk, w.Dv), '?')}>"
 
 
@@ -529,7 +532,8 @@ def run_gpu(args):
             "pct_of_bf16_sustained": 100.0 * (value / world) / peak_sust,
             "flop_per_step": flop_step, "kernel_ms": per_kernel,
             "roofline": {
-                "kernel": bwd_kernel_name(w), "bound": "tensor", "achieved": achieved,
+                "kernel": bwd_kernel_name(w, args.deterministic), "bound": "tensor",
+                "achieved": achieved,
                 "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_kind": f"{peak_kind} ({of}); burst {peak_burst:.1f}, sustained {peak_sust:.1f}",
                 "traffic": profiled_traffic(w.name),

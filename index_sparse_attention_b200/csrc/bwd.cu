@@ -29,9 +29,16 @@
 // the block mask, index mode from the presence bitmap (one word per lane and a warp
 // bit transpose give each key row its 32-query word).  dK (scaled by softmax_scale)
 // and dV leave through the idle stages by TMA tensor stores.
-// When Dqk + Dv does not leave room in the 512 TMEM columns (192/128), the head dim of
-// dK/dV/dQ is split over two CTAs, each recomputing S^T and dP^T.  Head dims 256/256
-// run on a 2-CTA cluster that splits the work instead (bwd_pair.cu).
+// Head dims (192,128) also run on one CTA per key tile, with a single S^T and a single
+// dP^T buffer: dK (192 columns), dV (128) and V (64, the TMEM operand of dP^T) leave 128
+// of the 512 TMEM columns.  The next step's S^T / dP^T then follow this step's dQ^T,
+// which comes in two 128-row windows: head dims 0-127 into the consumed S^T buffer (the
+// drain warps read it on its own commit), 64-191 into the consumed dP^T buffer (the
+// elementwise warps of lane quarters 2 and 3 read its rows 64-127, head dims 128-191,
+// and reduce-add them).  Measured on the index workload against a head-dim split over
+// two CTAs that both recompute S^T and dP^T: backward main 13.11 -> 11.78 ms.  The
+// deterministic mode keeps that split (its dQ turns assume one reduce issuer per CTA).
+// Head dims 256/256 run on a 2-CTA cluster that splits the work by role (bwd_pair.cu).
 // Every mbarrier wait is bounded (see sa_device.cuh).
 #include "det_order.cuh"
 #include "sa_device.cuh"
@@ -120,10 +127,21 @@ struct BwdCfg {
   static constexpr int kQOff = kKOff + kKBytes + (kVT ? 0 : kVBytes);  // per stage: Q then dO
   static constexpr int kVOff = kVT ? kQOff + (kStages - 1) * (kQBytes + kOBytes) : kKOff + kKBytes;
   static constexpr int kStageBytes = kQBytes + kOBytes;
-  static constexpr int kDSOff = kQOff + kStages * kStageBytes;     // two dS^T buffers
+  // S^T / dP^T buffers in TMEM (and dS^T buffers in shared memory): two, so that the next
+  // step's S^T and dP^T overlap this step's elementwise work, or one where TMEM must hold
+  // dK and dV over the whole head dim beside V: (192,128) on one CTA per key tile takes
+  // 64 + 64 + 192 + 128 + 64 = 512 columns.  Its dQ^T (192 rows) then comes in two
+  // 128-row windows, head dims 0-127 into the consumed S^T buffer and 64-191 into the
+  // consumed dP^T buffer; the elementwise warps of lane quarters 2 and 3 drain the second
+  // window's rows 64-127 (head dims 128-191), the drain warps the first window.
+  static constexpr bool kWhole = DQK == 192 && NSPLIT == 1;
+  static constexpr int kNB = kWhole ? 1 : 2;
+  static constexpr int kDSOff = kQOff + kStages * kStageBytes;     // kNB dS^T buffers
   // fp32 dQ staging tile [2 panels][32 q][64 d]
-  static constexpr int kDQOff = kDSOff + 2 * kDSBytes;
-  static constexpr int kLOff = kDQOff + 128 * 32 * 4;               // per stage: lse2[64], delta[64]
+  static constexpr int kDQOff = kDSOff + kNB * kDSBytes;
+  // (kWhole) fp32 staging of the second window's head dims 128-191: [2 query halves][32 q][64 d]
+  static constexpr int kDQ2Off = kDQOff + 128 * 32 * 4;
+  static constexpr int kLOff = kDQ2Off + (kWhole ? 64 * 64 * 4 : 0);  // per stage: lse2[64], delta[64]
   static constexpr int kBMOff = kLOff + kStages * 2 * kBM * 4;     // per stage: bitmap words [64][4]
   static constexpr int kBarOff = kBMOff + kStages * kBM * 4 * 4;
   static constexpr int kSmem = kBarOff + 256 + 1024;
@@ -131,10 +149,10 @@ struct BwdCfg {
   // head-dim chunks of this CTA: dK [kc0, kc0 + kcn), dV [vc0, vc0 + vcn)
   static constexpr int kDKMax = NSPLIT == 1 ? DQK : (DQK == 192 ? 128 : DQK / 2);
   static constexpr int kDVMax = DV / NSPLIT;
-  // TMEM columns: S^T / P^T x2, dP^T / dS^T / dQ^T x2, dK, dV
-  static constexpr uint32_t kColS = 0;     // + 64 * buffer
-  static constexpr uint32_t kColDP = 128;  // + 64 * buffer
-  static constexpr uint32_t kColDK = 256;
+  // TMEM columns: S^T / P^T (/ dQ^T window 0) x kNB, dP^T / dS^T / dQ^T x kNB, dK, dV
+  static constexpr uint32_t kColS = 0;                // + 64 * buffer
+  static constexpr uint32_t kColDP = 64 * kNB;        // + 64 * buffer
+  static constexpr uint32_t kColDK = 128 * kNB;
   static constexpr uint32_t kColDV = kColDK + kDKMax;
   static constexpr uint32_t kColV = kColDV + kDVMax;  // V (kVT), DV / 2 columns
   static constexpr uint32_t kTmemCols = 512;
@@ -148,8 +166,10 @@ struct BwdCfg {
 enum : int {
   kBKV = 0, kBQF = 1, kBQE = 4, kBLF = 7, kBSF = 10, kBPF = 12, kBDQF = 14, kBDQE = 16,
   kBFin = 18, kBDrainB = 19,
-  kBVT = 20,  // V copied into TMEM (256 elementwise threads; (192,128) only)
-  kNumBarsB = 21
+  kBVT = 20,   // V copied into TMEM (256 elementwise threads; (192,128) only)
+  kBDQE2 = 21, // (kWhole) dQ^T window 1 read from the dP^T buffer (128 elementwise threads)
+  kBDQF2 = 22, // (kWhole) dQ^T window 1 complete (commit; with window 0 and dV / dK before it)
+  kNumBarsB = 23
 };
 
 // Warp roles: 0 producer, 1 MMA, 2-9 elementwise (one key row and 32 of the 64 query
@@ -170,6 +190,9 @@ __global__ void __launch_bounds__(448, 1)
                       const __grid_constant__ CUtensorMap tm_dv, const AttnArgs a) {
   using C = BwdCfg<DQK, DV, NSPLIT>;
   constexpr int BM = C::kBM;
+  constexpr int NB = C::kNB;
+  // (the deterministic mode's dQ turns assume one issuer of reduce-adds per CTA)
+  static_assert(!(DET && C::kWhole), "deterministic mode keeps the head-dim split");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -228,6 +251,8 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(BAR(kBFin), 1);
     mbar_init(BAR(kBDrainB), 1);
     mbar_init(BAR(kBVT), 256);
+    mbar_init(BAR(kBDQE2), 128);
+    mbar_init(BAR(kBDQF2), 1);
     abort_flag->abort = 0;
     fence_mbar_init();
   }
@@ -336,19 +361,25 @@ __global__ void __launch_bounds__(448, 1)
       // start-address field (no carry: shared addresses stay below 2^18)
       const uint64_t kd = sw128_desc(kbase, 16, 1024), vd = sw128_desc(vbase, 16, 1024);
       const uint64_t kwd = sw128_desc(kbase + (qw0 / 64) * C::kKPanel, C::kKPanel, 1024);
+      // (kWhole) dQ^T window 1: head dims 64-191 (K panels 1 and 2)
+      const uint64_t kwd1 = sw128_desc(kbase + C::kKPanel, C::kKPanel, 1024);
       bool ok = warp_wait(BAR(kBKV), 0, abort_flag, a.status, a.wait_limit_ns);
       if (C::kVT) ok = ok && warp_wait(BAR(kBVT), 0, abort_flag, a.status, a.wait_limit_ns);
-      // S^T(j) and dP^T(j) into TMEM buffer j & 1
+      // S^T(j) and dP^T(j) into TMEM buffer j % NB
       auto issue_sdp = [&](int j) -> bool {
-        const int st = j % C::kStages, u = j / C::kStages, bj = j & 1;
+        const int st = j % C::kStages, u = j / C::kStages, bj = NB == 2 ? (j & 1) : 0;
         if (!warp_wait(BAR(kBQF + st), u & 1, abort_flag, a.status, a.wait_limit_ns)) return false;
-        // the dQ^T of step j-2 lives in this buffer until it has been drained
-        if (j >= 2 && !warp_wait(BAR(kBDQE + bj), ((j - 2) >> 1) & 1, abort_flag, a.status, a.wait_limit_ns))
+        // the dQ^T of step j-NB lives in this buffer until it has been drained (kWhole:
+        // window 0 in the S^T buffer)
+        if (j >= NB && !warp_wait(BAR(kBDQE + bj), ((j - NB) / NB) & 1, abort_flag, a.status, a.wait_limit_ns))
           return false;
         tc_fence_after();
         const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
         const uint64_t qd = sw128_desc(qs, 16, 1024), od = sw128_desc(qs + C::kQBytes, 16, 1024);
-        if (elect_one()) {
+        // one lane issues both MMA batches and the commit (a commit tracks the MMAs of
+        // the thread that executes it)
+        const bool leader = elect_one();
+        if (leader) {
           for (int p = 0; p < DQK / 64; ++p) {
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
@@ -357,6 +388,15 @@ __global__ void __launch_bounds__(448, 1)
                       (p > 0 || k4 > 0) ? 1u : 0u);
             }
           }
+        }
+        __syncwarp();
+        // (kWhole) window 1 of dQ^T(j-1) lives in the dP^T buffer until the elementwise
+        // warps of lane quarters 2 and 3 have read it
+        if (C::kWhole && j >= 1) {
+          if (!warp_wait(BAR(kBDQE2), (j - 1) & 1, abort_flag, a.status, a.wait_limit_ns)) return false;
+          tc_fence_after();
+        }
+        if (leader) {
           for (int p = 0; p < DV / 64; ++p) {
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
@@ -376,10 +416,11 @@ __global__ void __launch_bounds__(448, 1)
       };
       if (ok) ok = issue_sdp(0);
       for (int it = 0; ok && it < n_iter; ++it) {
-        const int st = it % C::kStages, bi = it & 1;
-        // the next S^T / dP^T overlap this step's elementwise work
-        if (it + 1 < n_iter && !issue_sdp(it + 1)) break;
-        if (!warp_wait(BAR(kBPF + bi), (it >> 1) & 1, abort_flag, a.status, a.wait_limit_ns)) break;
+        const int st = it % C::kStages, bi = NB == 2 ? (it & 1) : 0;
+        // the next S^T / dP^T overlap this step's elementwise work (two buffers; with one
+        // they follow this step's dQ^T, once it has been drained)
+        if (NB == 2 && it + 1 < n_iter && !issue_sdp(it + 1)) break;
+        if (!warp_wait(BAR(kBPF + bi), (it / NB) & 1, abort_flag, a.status, a.wait_limit_ns)) break;
         tc_fence_after();
         const uint32_t qs = sbase + C::kQOff + st * C::kStageBytes;
         const uint64_t qmn = sw128_desc(qs + (kc0 / 64) * C::kQPanel, C::kQPanel, 1024);
@@ -397,13 +438,25 @@ __global__ void __launch_bounds__(448, 1)
                     qmn + ((kk * 2048) >> 4), idesc_dk, (it > 0 || kk > 0) ? 1u : 0u);
           umma_commit(BAR(kBQE + st));
           // dQ^T = K^T dS^T over the 128 keys, into the dP^T buffer dK has just consumed
+          // (kWhole: window 0 into the S^T buffer dV has consumed, window 1 into dP^T's)
+          const uint32_t dq0 = (C::kWhole ? C::kColS : C::kColDP) + 64 * bi;
 #pragma unroll
           for (int kk = 0; kk < 128 / 16; ++kk)
-            umma_ss(tmem + C::kColDP + 64 * bi, kwd + ((kk * 2048) >> 4), dsd + ((kk * 2048) >> 4),
-                    idesc_dq, kk > 0 ? 1u : 0u);
+            umma_ss(tmem + dq0, kwd + ((kk * 2048) >> 4), dsd + ((kk * 2048) >> 4), idesc_dq,
+                    kk > 0 ? 1u : 0u);
+          // (kWhole: window 0 completes on its own barrier, so that the drain reads it, and
+          // the next S^T can be queued, while window 1 is computed)
           umma_commit(BAR(kBDQF + bi));
+          if constexpr (C::kWhole) {
+#pragma unroll
+            for (int kk = 0; kk < 128 / 16; ++kk)
+              umma_ss(tmem + C::kColDP, kwd1 + ((kk * 2048) >> 4), dsd + ((kk * 2048) >> 4),
+                      idesc_dq, kk > 0 ? 1u : 0u);
+            umma_commit(BAR(kBDQF2));
+          }
         }
         __syncwarp();
+        if (NB == 1 && it + 1 < n_iter && !issue_sdp(it + 1)) break;
       }
       if (elect_one()) umma_commit(BAR(kBFin));
       __syncwarp();
@@ -413,6 +466,9 @@ __global__ void __launch_bounds__(448, 1)
     const int quarter = warp & 3;
     const int hc = (warp - 2) >> 2;              // which 32 of the 64 query columns
     const int r = quarter * 32 + lane;           // key row of the tile = TMEM lane
+    // (kWhole) warps 2, 3 / 6, 7 (lane quarters 2 and 3, query halves 0 / 1) also drain
+    // dQ^T window 1, whose useful rows 64-127 are their TMEM lanes
+    const bool w1_helper = C::kWhole && quarter >= 2;
     const int64_t j = static_cast<int64_t>(nt) * 128 + r;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float* lbuf = reinterpret_cast<const float*>(smem + C::kLOff);
@@ -441,18 +497,26 @@ __global__ void __launch_bounds__(448, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(BAR(kBVT));
+      // a helper pair enters the step loop together or not at all (its warps' waits above
+      // can end differently when a wait runs out, and the loop meets at named barriers)
+      if (w1_helper) ok = named_bar_and(3 + hc, 64, ok);
     }
     for (int it = 0; ok && it < n_iter; ++it) {
       int h, m0;
       bool partial;
       decode(it, h, m0, partial);
-      const int st = it % C::kStages, u = it / C::kStages, bi = it & 1;
+      const int st = it % C::kStages, u = it / C::kStages, bi = NB == 2 ? (it & 1) : 0;
       bool w_ok = mbar_wait(BAR(kBLF + st), u & 1, abort_flag, a.status, a.wait_limit_ns);
-      w_ok = w_ok && mbar_wait(BAR(kBSF + bi), (it >> 1) & 1, abort_flag, a.status, a.wait_limit_ns);
-      // the dS^T buffer is free once dQ^T of step it-2 has read it
-      if (it >= 2)
-        w_ok = w_ok && mbar_wait(BAR(kBDQF + bi), ((it - 2) >> 1) & 1, abort_flag, a.status, a.wait_limit_ns);
-      if (!__all_sync(0xFFFFFFFFu, w_ok)) {
+      w_ok = w_ok && mbar_wait(BAR(kBSF + bi), (it / NB) & 1, abort_flag, a.status, a.wait_limit_ns);
+      // the dS^T buffer is free once dQ^T of step it-NB has read it (kWhole: both windows)
+      if (it >= NB)
+        w_ok = w_ok && mbar_wait(BAR(C::kWhole ? kBDQF2 : kBDQF + bi), ((it - NB) / NB) & 1,
+                                 abort_flag, a.status, a.wait_limit_ns);
+      w_ok = __all_sync(0xFFFFFFFFu, w_ok);
+      // (the two warps of a dQ^T-window-1 helper pair leave together: they share a named
+      // barrier below)
+      if (w1_helper) w_ok = named_bar_and(3 + hc, 64, w_ok);
+      if (!w_ok) {
         ok = false;
         break;
       }
@@ -538,7 +602,37 @@ __global__ void __launch_bounds__(448, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(BAR(kBPF + bi));
+      if (w1_helper) {
+        // dQ^T window 1 (head dims 64-191 in the dP^T buffer): this thread's row r - 64 of
+        // head dims 128-191 over this pair's 32 queries, read as soon as dQ^T is complete
+        // (S^T / dP^T of the next step wait for that), then staged as a [32 q][64 d] fp32
+        // tile and reduce-added into dQ_acc by one thread of the pair
+        bool d_ok = mbar_wait(BAR(kBDQF2), it & 1, abort_flag, a.status, a.wait_limit_ns);
+        if (!named_bar_and(3 + hc, 64, __all_sync(0xFFFFFFFFu, d_ok))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t w1[32];
+        tmem_ld32(tl + C::kColDP + 32 * hc, w1);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(BAR(kBDQE2));
+        const bool issuer = threadIdx.x == 64 + 128 * hc;  // warp 2 / 6, lane 0
+        float* st2 = reinterpret_cast<float*>(smem + C::kDQ2Off + hc * 32 * 64 * 4);
+        if (issuer) bulk_wait_group_read0();  // the previous reduce has read the tile
+        named_bar_sync(3 + hc, 64);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) st2[q * 64 + (r - 64)] = __uint_as_float(w1[q]);
+        fence_proxy_async_smem();
+        named_bar_sync(3 + hc, 64);
+        if (issuer) {
+          tma_reduce_add_4d(&tm_dq, sbase + C::kDQ2Off + hc * 32 * 64 * 4, 128, m0 + 32 * hc, h, b);
+          bulk_commit_group();
+        }
+      }
     }
+    if (w1_helper && threadIdx.x == 64 + 128 * hc) bulk_wait_group0();  // every reduce landed
     // ----------------------------------------------------------- dK / dV epilogue
     bool have = n_iter > 0 && ok;
     if (have) {
@@ -611,17 +705,19 @@ __global__ void __launch_bounds__(448, 1)
       int h, m0;
       bool partial;
       decode(it, h, m0, partial);
-      const int bi = it & 1;
+      const int bi = NB == 2 ? (it & 1) : 0;
       // the four drain warps leave together (they share named barrier 1 below)
-      const bool w_ok = mbar_wait(BAR(kBDQF + bi), (it >> 1) & 1, abort_flag, a.status, a.wait_limit_ns);
+      const bool w_ok = mbar_wait(BAR(kBDQF + bi), (it / NB) & 1, abort_flag, a.status, a.wait_limit_ns);
       if (!named_bar_and(1, 128, w_ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t q_u[BM];
-      tmem_ld32(tl + C::kColDP + 64 * bi, q_u);
-      tmem_ld32(tl + C::kColDP + 64 * bi + 32, q_u + 32);
+      // dQ^T window 0 (kWhole: in the S^T buffer)
+      const uint32_t dq0 = (C::kWhole ? C::kColS : C::kColDP) + 64 * bi;
+      tmem_ld32(tl + dq0, q_u);
+      tmem_ld32(tl + dq0 + 32, q_u + 32);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(BAR(kBDQE + bi));
@@ -750,7 +846,10 @@ int launch_bwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
   else if (a.Dqk == 128 && a.Dv == 128)
     rc = launch_bwd_main<128, 128, 1>(a, m, st);
   else if (a.Dqk == 192 && a.Dv == 128)
-    rc = launch_bwd_main<192, 128, 2>(a, m, st);
+    // one CTA per key tile (single-buffered S^T / dP^T); the deterministic mode keeps the
+    // head-dim split over two CTAs
+    rc = a.det ? launch_bwd_main_t<192, 128, 2, true>(a, m, st)
+               : launch_bwd_main_t<192, 128, 1, false>(a, m, st);
   else if (a.Dqk == 256 && a.Dv == 256)
     rc = launch_bwd_pair(a, m, st);
   else
