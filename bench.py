@@ -89,14 +89,18 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def bwd_kernel_name(w, deterministic=False):
-    """The backward main kernel that the library launches for this workload's head dims
-    (at (192,128) one CTA per key tile, or the head-dim split over two in deterministic
-    mode)."""
+def bwd_kernel_name(w, deterministic=False, form="auto", sms=148):
+    """The backward main kernel that the library launches for this workload's head dims.
+    At (192,128): one CTA per key tile ("whole") when chosen, or under "auto" when the
+    grid of key tiles is at least twice the SM count; else (and in deterministic mode)
+    the head-dim split over two CTAs (the rule of sparse_attn_set_backward_form)."""
     if (w.Dqk, w.Dv) == (256, 256):
         return "sparse_bwd_pair_kernel"
-    inst = {(64, 64): "128,128,1", (128, 128): "128,128,1",
-            (192, 128): "192,128,2" if deterministic else "192,128,1"}
+    if (w.Dqk, w.Dv) == (192, 128):
+        tiles = -(-w.Sk // 128) * w.HK * w.B
+        whole = not deterministic and (form == "whole" or (form == "auto" and tiles >= 2 * sms))
+        return f"sparse_bwd_kernel<192,128,{1 if whole else 2}>"
+    inst = {(64, 64): "128,128,1", (128, 128): "128,128,1"}
     return f"sparse_bwd_kernel<{inst.get((w.Dqk, w.Dv), '?')}>"
 
 
@@ -344,6 +348,7 @@ def run_gpu(args):
 
     L = _lib.load()
     sa.sparse_attn_set_forward_form(args.fwd_form)
+    sa.sparse_attn_set_backward_form(args.bwd_form)
     w = get_workload(args)
     inp = I.make_inputs(w)
     dev = torch.device("cuda", local)
@@ -524,6 +529,8 @@ def run_gpu(args):
             "config": dict(workload_config(w, active),
                            **({"backward": "deterministic"} if args.deterministic else {}),
                            **({"forward_form": args.fwd_form} if args.fwd_form != "auto"
+                              else {}),
+                           **({"backward_form": args.bwd_form} if args.bwd_form != "auto"
                               else {})),
             "pct_of_bf16_peak": 100.0 * (value / world) / peak,
             "pct_basis": (f"{peak_kind} {peak:.1f} TFLOP/s ({of}); burst unless the clock record "
@@ -532,7 +539,9 @@ def run_gpu(args):
             "pct_of_bf16_sustained": 100.0 * (value / world) / peak_sust,
             "flop_per_step": flop_step, "kernel_ms": per_kernel,
             "roofline": {
-                "kernel": bwd_kernel_name(w, args.deterministic), "bound": "tensor",
+                "kernel": bwd_kernel_name(w, args.deterministic, args.bwd_form,
+                                          torch.cuda.get_device_properties(dev).multi_processor_count),
+                "bound": "tensor",
                 "achieved": achieved,
                 "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_kind": f"{peak_kind} ({of}); burst {peak_burst:.1f}, sustained {peak_sust:.1f}",
@@ -820,6 +829,10 @@ def main():
                          "GQA group on a 2-CTA pair with cta_group::2 MMAs, two heads per "
                          "CTA, two query tiles of one head per CTA, or the library's choice "
                          "(auto)")
+    ap.add_argument("--bwd-form", default="auto", choices=["auto", "split", "whole"],
+                    help="backward form at head dims (192,128): two CTAs per key tile each "
+                         "with part of the head dim, one CTA per key tile, or the library's "
+                         "choice by grid size (auto)")
     ap.add_argument("--op", default="attention",
                     choices=["attention", "topk", "index_stats", "gather"],
                     help="topk: time the top-k selector alone on one packed sequence; "

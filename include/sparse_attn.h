@@ -290,6 +290,31 @@ int sparse_attn_set_wait_limit_ns(uint64_t ns);
  */
 int sparse_attn_set_forward_form(int form);
 
+/* Forms of sparse_attn_set_backward_form. */
+#define SA_BWD_FORM_AUTO 0
+#define SA_BWD_FORM_SPLIT 1
+#define SA_BWD_FORM_WHOLE 2
+
+/*
+ * sparse_attn_set_backward_form -- selects how the backward main kernel covers a 128-key
+ * tile at head dims (192,128), where the fp32 dK and dV of the whole head dim (320 TMEM
+ * columns) leave too little tensor memory for double-buffered S^T / dP^T tiles
+ * (MagiAttention PR #331 builds 192/128 with 2-CTA tiles; the forms here are this
+ * library's own):
+ *   SA_BWD_FORM_SPLIT  two CTAs per key tile, each owning part of the head dim of dK, dV
+ *                      and dQ and each recomputing S^T and dP^T (double-buffered);
+ *   SA_BWD_FORM_WHOLE  one CTA per key tile with single S^T / dP^T buffers: no
+ *                      recompute, but each step's MMAs wait for the previous step;
+ *   SA_BWD_FORM_AUTO   WHOLE when the grid of key tiles (B * HK * ceil(Sk/128)) is at
+ *                      least twice the SM count, else SPLIT (measured: WHOLE is ~10%
+ *                      faster once the SMs are filled, slower while half of them idle).
+ * The deterministic backward always splits.  Other head dims ignore the setting.  All
+ * forms compute the same gradients up to fp32 rounding.  Applies to the backward calls
+ * enqueued after it; process-wide.  Returns SA_OK, or SA_ERR_INVALID for another value
+ * (the setting is then unchanged).
+ */
+int sparse_attn_set_backward_form(int form);
+
 
 /* Largest k that topk_select supports. */
 #define SA_TOPK_MAX_K 4096

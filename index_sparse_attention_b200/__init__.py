@@ -18,7 +18,7 @@ __all__ = ["BlockSparse", "block_mask_to_block_sparse", "index_to_block_sparse",
            "sparse_attn_fwd", "sparse_attn_fwd_gather", "sparse_attn_bwd",
            "sparse_attn_bwd_workspace_size", "sparse_attn_bwd_noalloc", "topk_select",
            "sparse_attn_set_wait_limit_ns", "sparse_attn_set_forward_form",
-           "SparseAttnError", "SA_TILE"]
+           "sparse_attn_set_backward_form", "SparseAttnError", "SA_TILE"]
 
 
 def _stream(device):
@@ -340,3 +340,19 @@ def sparse_attn_set_forward_form(form):
     if isinstance(code, str):
         raise ValueError(f"form must be one of {sorted(_FWD_FORMS)}, got {form!r}")
     _lib.check("sparse_attn_set_forward_form", _lib.load().sparse_attn_set_forward_form(code))
+
+
+_BWD_FORMS = {"auto": _lib.SA_BWD_FORM_AUTO, "split": _lib.SA_BWD_FORM_SPLIT,
+              "whole": _lib.SA_BWD_FORM_WHOLE}
+
+
+def sparse_attn_set_backward_form(form):
+    """How the backward covers a key tile at head dims (192,128): "auto" (the library's
+    choice by grid size), "split" (two CTAs per key tile, each with part of the head dim,
+    both recomputing S^T and dP^T) or "whole" (one CTA per key tile, single-buffered).
+    The deterministic backward always splits.  Applies to the backward calls made after
+    it, process-wide; see include/sparse_attn.h."""
+    code = _BWD_FORMS.get(form, form) if isinstance(form, str) else int(form)
+    if isinstance(code, str):
+        raise ValueError(f"form must be one of {sorted(_BWD_FORMS)}, got {form!r}")
+    _lib.check("sparse_attn_set_backward_form", _lib.load().sparse_attn_set_backward_form(code))

@@ -26,6 +26,7 @@ SA_TOPK_MAX_K = 4096
 SA_MODE_DENSE, SA_MODE_BLOCK, SA_MODE_INDEX = 0, 1, 2
 SA_FWD_FORM_AUTO, SA_FWD_FORM_ONE_HEAD, SA_FWD_FORM_CTA_PAIR, SA_FWD_FORM_TWO_HEADS = 0, 1, 2, 3
 SA_FWD_FORM_TWO_TILES = 4
+SA_BWD_FORM_AUTO, SA_BWD_FORM_SPLIT, SA_BWD_FORM_WHOLE = 0, 1, 2
 SA_TILE = 128
 
 STATUS_INDEX = 1
@@ -44,6 +45,7 @@ EXPORTS = (
     "sparse_attn_set_timing_events",
     "sparse_attn_set_wait_limit_ns",
     "sparse_attn_set_forward_form",
+    "sparse_attn_set_backward_form",
     "sparse_attn_error_string",
     "topk_select",
 )
@@ -106,6 +108,8 @@ def load():
     L.sparse_attn_set_wait_limit_ns.restype = ctypes.c_int
     L.sparse_attn_set_forward_form.argtypes = [ctypes.c_int]
     L.sparse_attn_set_forward_form.restype = ctypes.c_int
+    L.sparse_attn_set_backward_form.argtypes = [ctypes.c_int]
+    L.sparse_attn_set_backward_form.restype = ctypes.c_int
     i64 = ctypes.c_int64
     L.topk_select.argtypes = [vp, i64, i64, i64, vp, vp, ctypes.c_int32, vp, vp, vp, vp]
     L.topk_select.restype = ctypes.c_int

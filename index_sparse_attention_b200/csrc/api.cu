@@ -23,6 +23,7 @@ cudaEvent_t* g_timing_events = nullptr;
 static cudaEvent_t g_events_copy[6];
 std::atomic<uint64_t> g_wait_limit_ns{0};
 std::atomic<int> g_fwd_form{SA_FWD_FORM_AUTO};
+std::atomic<int> g_bwd_form{SA_BWD_FORM_AUTO};  // read by launch_bwd (bwd.cu)
 }  // namespace sa
 
 namespace {
@@ -202,6 +203,12 @@ extern "C" int sparse_attn_set_wait_limit_ns(uint64_t ns) {
 extern "C" int sparse_attn_set_forward_form(int form) {
   if (form < SA_FWD_FORM_AUTO || form > SA_FWD_FORM_TWO_TILES) return SA_ERR_INVALID;
   g_fwd_form.store(form, std::memory_order_relaxed);
+  return SA_OK;
+}
+
+extern "C" int sparse_attn_set_backward_form(int form) {
+  if (form < SA_BWD_FORM_AUTO || form > SA_BWD_FORM_WHOLE) return SA_ERR_INVALID;
+  g_bwd_form.store(form, std::memory_order_relaxed);
   return SA_OK;
 }
 

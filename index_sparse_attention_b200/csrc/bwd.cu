@@ -49,6 +49,9 @@
 
 namespace sa {
 
+// Backward form at head dims (192,128) (SA_BWD_FORM_*, set by sparse_attn_set_backward_form).
+extern std::atomic<int> g_bwd_form;
+
 // ------------------------------------------------------------------------------------
 // preprocess: Delta = rowsum(dO * O) (fp32) and a zeroed dQ accumulator
 // ------------------------------------------------------------------------------------
@@ -845,11 +848,23 @@ int launch_bwd(const AttnArgs& a, const TensorMaps& m, cudaStream_t st) {
     rc = launch_bwd_main<128, 128, 1>(a, m, st);
   else if (a.Dqk == 128 && a.Dv == 128)
     rc = launch_bwd_main<128, 128, 1>(a, m, st);
-  else if (a.Dqk == 192 && a.Dv == 128)
-    // one CTA per key tile (single-buffered S^T / dP^T); the deterministic mode keeps the
-    // head-dim split over two CTAs
-    rc = a.det ? launch_bwd_main_t<192, 128, 2, true>(a, m, st)
-               : launch_bwd_main_t<192, 128, 1, false>(a, m, st);
+  else if (a.Dqk == 192 && a.Dv == 128) {
+    // One CTA per key tile (single-buffered S^T / dP^T, no recompute) once its grid fills
+    // the SMs at least twice over; below that the head-dim split over two CTAs, which
+    // keeps twice as many SMs busy (measured at total_q = 4096, 128 key-tile CTAs on 148
+    // SMs: 1.51 ms against 1.22; at 16384, 512 CTAs: 11.8 against 13.1 ms).  The
+    // deterministic mode always splits.
+    int form = g_bwd_form.load(std::memory_order_relaxed);
+    if (form == SA_BWD_FORM_AUTO) {
+      int dev = 0, sms = 148;
+      if (cudaGetDevice(&dev) == cudaSuccess)
+        (void)cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      const int64_t ctas = static_cast<int64_t>(a.Tn) * a.HK * a.B;
+      form = ctas >= 2 * static_cast<int64_t>(sms) ? SA_BWD_FORM_WHOLE : SA_BWD_FORM_SPLIT;
+    }
+    rc = (a.det || form == SA_BWD_FORM_SPLIT) ? launch_bwd_main<192, 128, 2>(a, m, st)
+                                              : launch_bwd_main_t<192, 128, 1, false>(a, m, st);
+  }
   else if (a.Dqk == 256 && a.Dv == 256)
     rc = launch_bwd_pair(a, m, st);
   else

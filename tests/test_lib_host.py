@@ -114,6 +114,21 @@ def test_instrumentation_setters(lib):
     assert lib.sparse_attn_set_wait_limit_ns(0) == _lib.SA_OK
 
 
+def test_backward_form_setter(lib):
+    """The (192,128) backward's key-tile form: the three SA_BWD_FORM_* values are accepted,
+    anything else is refused with SA_ERR_INVALID; the binding maps the names and refuses
+    unknown ones."""
+    import index_sparse_attention_b200 as sa
+    for code in (_lib.SA_BWD_FORM_SPLIT, _lib.SA_BWD_FORM_WHOLE, _lib.SA_BWD_FORM_AUTO):
+        assert lib.sparse_attn_set_backward_form(code) == _lib.SA_OK
+    for bad in (-1, 3, 1 << 20):
+        assert lib.sparse_attn_set_backward_form(bad) == _lib.SA_ERR_INVALID
+    for name in ("split", "whole", "auto"):
+        sa.sparse_attn_set_backward_form(name)
+    with pytest.raises(ValueError):
+        sa.sparse_attn_set_backward_form("halves")
+
+
 def test_forward_form_setter(lib):
     """The forward's head-to-CTA form: the four SA_FWD_FORM_* values are accepted,
     anything else is refused with SA_ERR_INVALID; the binding maps the names and refuses
