@@ -93,3 +93,22 @@ def test_head_count_override_makes_a_gqa_workload():
             bench.get_workload(argparse.Namespace(workload=ns.workload, seq=0, heads=bad))
     ns.heads = ""
     assert bench.get_workload(ns) == I.WORKLOADS[ns.workload]
+
+
+def test_reported_backward_kernel_follows_the_library_rule():
+    """The roofline names the (192,128) backward instance the library picks: one CTA per
+    key tile when B * HK * ceil(Sk / 128) is at least twice the SM count, else (and in
+    deterministic mode, or when the split is forced) the head-dim split."""
+    from index_sparse_attention_b200 import inputs as I
+    w = I.WORKLOADS["indexsparse_gqa_q16384_hq32_hk4_d192_128_top2048"]  # 128 tiles x 4 heads
+    assert bench.bwd_kernel_name(w) == "sparse_bwd_kernel<192,128,1>"
+    assert bench.bwd_kernel_name(w, deterministic=True) == "sparse_bwd_kernel<192,128,2>"
+    assert bench.bwd_kernel_name(w, form="split") == "sparse_bwd_kernel<192,128,2>"
+    small = I.scaled(w, Sq=4096, Sk=4096)  # 32 tiles x 4 heads = 128 < 2 x 148
+    assert bench.bwd_kernel_name(small) == "sparse_bwd_kernel<192,128,2>"
+    assert bench.bwd_kernel_name(small, form="whole") == "sparse_bwd_kernel<192,128,1>"
+    edge = I.scaled(w, Sq=9472, Sk=9472)  # 74 tiles x 4 heads = 296 = 2 x 148
+    assert bench.bwd_kernel_name(edge) == "sparse_bwd_kernel<192,128,1>"
+    assert bench.bwd_kernel_name(I.scaled(w, Sq=9344, Sk=9344)) == "sparse_bwd_kernel<192,128,2>"
+    assert bench.bwd_kernel_name(I.WORKLOADS["long_causal_blocksparse_h16_s32768_d256"]) == \
+        "sparse_bwd_pair_kernel"
