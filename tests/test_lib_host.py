@@ -36,6 +36,23 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, n), f"{n} declared but not exported"
 
 
+def test_header_constants_match_the_binding():
+    """Every integer SA_* constant the header defines has the same value in the binding."""
+    import os
+    import re
+    hdr = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                            "include", "sparse_attn.h")).read()
+    defs = {}
+    for name, expr in re.findall(r"^#define (SA_[A-Z0-9_]+) ([^/\n]+)", hdr, re.M):
+        expr = expr.strip()
+        if re.fullmatch(r"[-+*()0-9u\s]+", expr):  # integer expressions only
+            defs[name] = eval(expr.replace("u", ""))
+    assert len(defs) >= 20
+    for name, value in defs.items():
+        assert hasattr(_lib, name), f"{name} missing from the binding"
+        assert getattr(_lib, name) == value, (name, getattr(_lib, name), value)
+
+
 def test_error_strings(lib):
     for code in (0, -1, -2, -3, -4, -5, -7, 12345):
         assert isinstance(_lib.error_string(code), str)
