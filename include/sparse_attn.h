@@ -47,8 +47,8 @@
  *    scratch address) is done on first use on each device, thread-safely.
  *  - Return value: SA_OK (0) or a negative SA_ERR_* code.  Errors found on the GPU
  *    (an index outside [-1, Sk), a pipeline wait that timed out) are OR-ed into the
- *    optional device int32 `dev_status` (bit 1: index, bit 2: timeout); read it after
- *    synchronising.  No C++ exception crosses this boundary.
+ *    optional device int32 `dev_status` as the flags SA_STATUS_INDEX (value 1) and
+ *    SA_STATUS_TIMEOUT (value 2); read it after synchronising.  No C++ exception crosses this boundary.
  */
 #ifndef SPARSE_ATTN_H_
 #define SPARSE_ATTN_H_
@@ -71,6 +71,10 @@ typedef struct CUstream_st *sa_stream_t; /* the same handle as cudaStream_t */
 #define SA_ERR_WORKSPACE (-7)   /* workspace missing or too small */
 #define SA_ERR_SCRATCH_LIMIT (-8) /* sparse_attn_bwd_noalloc: problem exceeds its fixed scratch */
 #define SA_ERR_DEVICE (-9)      /* the stream belongs to a device other than the current one */
+
+/* Flags OR-ed into the optional device status word (dev_status). */
+#define SA_STATUS_INDEX 1   /* an index outside [-1, Sk), or a top-k row range outside [0, cols) */
+#define SA_STATUS_TIMEOUT 2 /* a bounded pipeline wait ran out */
 
 #define SA_MODE_DENSE 0
 #define SA_MODE_BLOCK 1
@@ -111,8 +115,8 @@ typedef struct sa_block_sparse {
  *   idx   device int32 [B][Sq][HK][topk]: key positions in [0, Sk) or -1 (padding).
  *   out   host struct: B, HK, Sq, Sk, causal and the device buffers bitmap, cnt, idx,
  *         tcnt, tidx must be set by the caller; mode is set to SA_MODE_INDEX.
- * Fills the bitmap and all four lists.  Values < -1 or >= Sk are skipped and set bit 1
- * of *dev_status (when dev_status is not NULL).
+ * Fills the bitmap and all four lists.  Values < -1 or >= Sk are skipped and set
+ * SA_STATUS_INDEX in *dev_status (when dev_status is not NULL).
  */
 int index_to_block_sparse(const int32_t *idx, int32_t topk, sa_block_sparse *out,
                           int32_t *dev_status, sa_stream_t stream);
@@ -238,7 +242,7 @@ int sparse_attn_set_timing_events(void *const *events);
 /*
  * sparse_attn_set_wait_limit_ns -- test instrumentation (no counterpart on the pages).
  * Every pipeline wait inside the attention kernels is bounded: a wait that has not
- * completed after the limit gives up, sets bit 2 of *dev_status, and its CTA drains the
+ * completed after the limit gives up, sets SA_STATUS_TIMEOUT in *dev_status, and its CTA drains the
  * copies and tensor-core operations it has in flight and leaves (the outputs of that
  * call are then undefined, the CUDA context stays usable).  The default limit is 2 s.
  * This call sets the limit, in nanoseconds, for the calls enqueued after it (0 restores
@@ -333,7 +337,7 @@ int sparse_attn_set_backward_form(int form);
  *           smaller column, -0 equals +0, NaN ranks above +inf; when the range holds
  *           n < k columns, slots n..k-1 are -1.
  *   out_val optional device fp32 [rows][k]: the selected scores (-inf in -1 slots).
- * A row whose range is invalid yields k times -1 and sets bit 1 of *dev_status.  Needs
+ * A row whose range is invalid yields k times -1 and sets SA_STATUS_INDEX in *dev_status.  Needs
  * no workspace.  Returns SA_ERR_INVALID for a bad size, k or null pointer.
  */
 int topk_select(const float *scores, int64_t rows, int64_t cols, int64_t ld,

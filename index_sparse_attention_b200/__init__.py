@@ -318,8 +318,8 @@ def topk_select(scores, k, starts=None, ends=None, with_values=False, out_idx=No
 def sparse_attn_set_wait_limit_ns(ns):
     """Test instrumentation: the limit (ns) of every pipeline wait of the attention
     kernels enqueued after this call (0 restores the default of 2 s).  A wait that runs
-    out sets bit 2 of the device status word and its CTA leaves; see
-    include/sparse_attn.h."""
+    out sets the timeout flag (SA_STATUS_TIMEOUT, value 2) in the device status word and
+    its CTA leaves; see include/sparse_attn.h."""
     _lib.check("sparse_attn_set_wait_limit_ns", _lib.load().sparse_attn_set_wait_limit_ns(int(ns)))
 
 

@@ -31,6 +31,7 @@ SA_TILE = 128
 
 STATUS_INDEX = 1
 STATUS_TIMEOUT = 2
+SA_STATUS_INDEX, SA_STATUS_TIMEOUT = STATUS_INDEX, STATUS_TIMEOUT
 
 # every symbol include/sparse_attn.h declares
 EXPORTS = (

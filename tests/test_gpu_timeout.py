@@ -1,7 +1,7 @@
 """Bounded pipeline waits: a wait that runs out reports itself and the kernel still ends.
 
 Every mbarrier wait of the attention kernels gives up after a limit (2 s by default),
-sets bit 2 of the device status word, and its CTA drains the copies and tensor-core
+sets the timeout flag (value 2) in the device status word, and its CTA drains the copies and tensor-core
 operations it has in flight before it releases its resources and leaves.  These tests
 set a limit below 1 us through the C ABI (sparse_attn_set_wait_limit_ns), which makes a
 wait give up at its first test when its phase has not completed, so that ordinary
