@@ -180,9 +180,10 @@ size_t sparse_attn_bwd_workspace_size(const sparse_attn_params *p);
  * transposed lists) recomputing P = exp(scale S - LSE), accumulating dV += P^T dO and
  * dK += dS^T Q in tensor memory (dK scaled by softmax_scale as it is stored) and
  * adding dQ += dS K into an fp32 accumulator; the postprocess scales dQ by
- * softmax_scale and casts it to bf16 (MagiAttention PR #334, section 1 and section 3).  `workspace` is device memory of at least
- * sparse_attn_bwd_workspace_size() bytes, owned by the caller; its contents need not
- * be initialised.
+ * softmax_scale and casts it to bf16 (MagiAttention PR #334, section 1 and section 3).
+ * At head dims (192,128) a key tile takes one CTA or two (sparse_attn_set_backward_form).
+ * `workspace` is device memory of at least sparse_attn_bwd_workspace_size() bytes, owned
+ * by the caller; its contents need not be initialised.
  */
 int sparse_attn_bwd(const sparse_attn_params *p, void *workspace, size_t workspace_bytes,
                     sa_stream_t stream);
